@@ -1,0 +1,358 @@
+"""CPU oracle for the Grouped Query Experts (GQE) attention forward (prefill) pass.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.
+The product path (the CUDA library and its Python binding) never calls it and shares
+no code with it; this module imports nothing from the product package.
+
+Everything is float64 numpy. Each step is the plain definition, written in the order
+the sources give it; numpy's matmul and exp are the only library primitives used.
+There is no blocking or fusion, except that attention rows are processed in chunks of
+query rows to bound memory, which does not change any row's arithmetic.
+
+Sources (by page title and section):
+  [README]   "GQE: Grouped Query Experts" (FrontiersMindAI/GQE README):
+             Algorithm Overview, Usage, Parameters, Ablations.
+  [Summary]  "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention",
+             gist.science technical summary: Methodology (Architecture and Routing,
+             Output Construction), Training and Loss.
+  [Tutorial] "Grouped-query attention and mixture of experts" (CSE Roadmap):
+             Mixture of experts (MoE).
+
+Pins (tests/test_oracle_pins.py): brute-force routing on tiny inputs, closed forms of
+the gates and of the aux loss, torch's float64 scaled_dot_product_attention, the
+reduction to an independently written dense GQA layer at k = E, and the
+identical-experts collapse. Every function below is pinned; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+VARIANTS = ("gqe", "weighted_concat", "hard_concat")
+
+
+@dataclass
+class Layer:
+    """Shapes of one GQE layer ([README] Parameters)."""
+
+    dim: int
+    N: int
+    G: int
+    k: int
+    d_h: int
+    shared: bool = True
+    variant: str = "gqe"
+    causal: bool = True
+
+    def __post_init__(self):
+        if self.N % self.G != 0:  # [README] Parameters: N must be divisible by G
+            raise ValueError("num_query_experts must be divisible by num_kv_heads")
+        if not 1 <= self.k <= self.N // self.G:
+            raise ValueError("top_k must be in [1, N/G]")
+        if self.variant not in VARIANTS:
+            raise ValueError(f"unknown variant {self.variant!r}")
+
+    @property
+    def E(self) -> int:
+        return self.N // self.G
+
+    @property
+    def n_streams(self) -> int:
+        """Query streams computed per token: G*k routed plus the shared head."""
+        return self.G * self.k + (1 if self.shared else 0)
+
+    @property
+    def D_o(self) -> int:
+        """Width of the concatenated output Z (input width of W_o)."""
+        blocks = self.G * self.k + (1 if self.variant == "gqe" else 0) + (1 if self.shared else 0)
+        return blocks * self.d_h
+
+
+def default_head_dim(dim: int, N: int) -> int:
+    """[README] Parameters: head_dim defaults to dim // num_query_experts."""
+    return dim // N
+
+
+# ----------------------------------------------------------------------------------------
+# Step 1-3: router ([README] Algorithm Overview: softmax over the experts of each group,
+# then top-k; [Tutorial] Mixture of experts: mixing weights renormalised to sum to 1).
+# ----------------------------------------------------------------------------------------
+
+@dataclass
+class Routing:
+    logits: np.ndarray   # [M, N] float64
+    p: np.ndarray        # [M, G, E] per-group softmax, float64
+    sel: np.ndarray      # [M, G, k] int32, selected j in ascending order
+    p_sel: np.ndarray    # [M, G, k] p of the selected experts
+    gates: np.ndarray    # [M, G, k] p_sel renormalised within the group
+    w: np.ndarray        # [M, G, k] p_sel renormalised over all G*k selections (slot weights)
+    counts: np.ndarray   # [N] int64 tokens per expert
+    prob_sum: np.ndarray  # [N] float64 sum over tokens of p
+
+
+def router_logits(x: np.ndarray, W_r: np.ndarray) -> np.ndarray:
+    """l[t, e] = <x_t, W_r[e]> (no bias)."""
+    return x @ W_r.T
+
+
+def group_softmax(logits: np.ndarray, G: int) -> np.ndarray:
+    """Softmax over the E experts inside each of the G groups, with max subtraction."""
+    M, N = logits.shape
+    E = N // G
+    lg = logits.reshape(M, G, E)
+    z = np.exp(lg - lg.max(axis=2, keepdims=True))
+    return z / z.sum(axis=2, keepdims=True)
+
+
+def top_k_per_group(logits: np.ndarray, G: int, k: int) -> np.ndarray:
+    """The k largest experts of each group, listed in ascending expert index.
+
+    Ranking p equals ranking the logits (softmax is strictly increasing). The decision
+    is taken on the logits rounded to fp32, the GPU's precision; ties go to the lower
+    index. Returns int32 [M, G, k].
+    """
+    M, N = logits.shape
+    E = N // G
+    l32 = logits.astype(np.float32).reshape(M, G, E).astype(np.float64)
+    # Take the k experts one at a time: each time the largest logit not yet taken,
+    # the lowest index among equal maxima (argmax returns the first maximum).
+    taken = np.zeros((M, G, E), dtype=bool)
+    mi, gi = np.arange(M)[:, None], np.arange(G)[None, :]
+    for _ in range(k):
+        j = np.argmax(np.where(taken, -np.inf, l32), axis=2)
+        taken[mi, gi, j] = True
+    # List each selected set in ascending expert index.
+    chosen = np.zeros((M, G, k), dtype=np.int32)
+    for g in range(G):
+        chosen[:, g, :] = np.nonzero(taken[:, g, :])[1].reshape(M, k)
+    return chosen
+
+
+def route(x: np.ndarray, W_r: np.ndarray, G: int, k: int) -> Routing:
+    """Router, gates, slot weights and the statistics the load-balancing loss needs."""
+    M = x.shape[0]
+    N = W_r.shape[0]
+    E = N // G
+    logits = router_logits(x, W_r)
+    p = group_softmax(logits, G)
+    sel = top_k_per_group(logits, G, k)
+    p_sel = np.take_along_axis(p, sel.astype(np.int64), axis=2)
+    gates = p_sel / p_sel.sum(axis=2, keepdims=True)
+    w = p_sel / p_sel.sum(axis=(1, 2), keepdims=True)
+    counts = np.zeros(N, dtype=np.int64)
+    for g in range(G):
+        for r in range(k):
+            counts[g * E: (g + 1) * E] += np.bincount(sel[:, g, r], minlength=E)
+    prob_sum = p.reshape(M, N).sum(axis=0)
+    return Routing(logits, p, sel, p_sel, gates, w, counts, prob_sum)
+
+
+# ----------------------------------------------------------------------------------------
+# Step 4: projections ([README] Algorithm Overview: KV heads dense and unchanged, only the
+# selected query heads are computed; an always-on shared query head).
+# ----------------------------------------------------------------------------------------
+
+def kv_projection(x: np.ndarray, W_k: np.ndarray, W_v: np.ndarray, G: int, d_h: int):
+    """K[g], V[g] = x W_k[g]^T, x W_v[g]^T for every token. Returns [G, M, d_h] each."""
+    M = x.shape[0]
+    K = (x @ W_k.T).reshape(M, G, d_h).transpose(1, 0, 2).copy()
+    V = (x @ W_v.T).reshape(M, G, d_h).transpose(1, 0, 2).copy()
+    return K, V
+
+
+def routed_queries(x: np.ndarray, W_q: np.ndarray, sel: np.ndarray, G: int, E: int,
+                   d_h: int) -> np.ndarray:
+    """Q[s = g*k + r, t] = x_t W_q[g*E + sel[t,g,r]]^T, only for the selected pairs.
+
+    Returns [G*k, M, d_h]. Each expert's projection is applied only to the tokens that
+    selected it.
+    """
+    M = x.shape[0]
+    k = sel.shape[2]
+    Q = np.zeros((G * k, M, d_h))
+    for g in range(G):
+        for j in range(E):
+            Wqe = W_q[(g * E + j) * d_h:(g * E + j + 1) * d_h]
+            for r in range(k):
+                rows = np.nonzero(sel[:, g, r] == j)[0]
+                if rows.size:
+                    Q[g * k + r, rows] = x[rows] @ Wqe.T
+    return Q
+
+
+def shared_query(x: np.ndarray, W_shared: np.ndarray) -> np.ndarray:
+    """The always-on shared head's query for every token: [M, d_h]."""
+    return x @ W_shared.T
+
+
+def stream_kv_head(s: int, k: int, G: int) -> int:
+    """KV head read by query stream s: its group for routed streams, head 0 for the
+    shared stream (a stated reading: one extra head, and head 0 is the plainest)."""
+    return s // k if s < G * k else 0
+
+
+# ----------------------------------------------------------------------------------------
+# Step 5: softmax attention over the unchanged dense K/V.
+# ----------------------------------------------------------------------------------------
+
+def attention_rows(q: np.ndarray, t_pos: np.ndarray, K: np.ndarray, V: np.ndarray,
+                   causal: bool, chunk: int = 1024) -> np.ndarray:
+    """Softmax attention of query rows q [R, d_h] at positions t_pos [R] over one
+    sequence's keys K, V [T, d_h]: O = softmax(q K^T / sqrt(d_h)) V, keys u <= t only
+    when causal. Rows are independent; they are processed in chunks to bound memory."""
+    R, d_h = q.shape
+    T = K.shape[0]
+    out = np.empty((R, V.shape[1]))
+    scale = 1.0 / math.sqrt(d_h)
+    for a in range(0, R, chunk):
+        b = min(R, a + chunk)
+        s = (q[a:b] @ K.T) * scale
+        if causal:
+            u = np.arange(T)[None, :]
+            s = np.where(u <= t_pos[a:b, None], s, -np.inf)
+        s = s - s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        out[a:b] = (e @ V) / e.sum(axis=1, keepdims=True)
+    return out
+
+
+def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, B: int, T: int, k: int, G: int,
+              causal: bool) -> np.ndarray:
+    """All streams. Q [S, M, d_h], K/V [G, M, d_h]; returns O [S, M, d_h]."""
+    S, M, d_h = Q.shape
+    O = np.empty_like(Q)
+    pos = np.arange(T)
+    for s in range(S):
+        h = stream_kv_head(s, k, G)
+        for b in range(B):
+            rows = slice(b * T, (b + 1) * T)
+            O[s, rows] = attention_rows(Q[s, rows], pos, K[h, rows], V[h, rows], causal)
+    return O
+
+
+# ----------------------------------------------------------------------------------------
+# Step 6-7: output construction by variant ([Summary] Output Construction; [README]
+# Ablations) and the output projection.
+# ----------------------------------------------------------------------------------------
+
+def combine(O: np.ndarray, routing: Routing, layer: Layer) -> np.ndarray:
+    """Build Z [M, D_o] from the stream outputs O [S, M, d_h].
+
+    Column blocks: routed streams g-major then r; then the renormalised slot (variant
+    gqe only); then the shared stream (unweighted, whenever the shared head exists).
+      hard_concat:     routed outputs as they are.
+      weighted_concat: routed output (g, r) times the raw per-group softmax p of its expert.
+      gqe:             routed outputs as they are, plus slot = sum_{g,r} w * O.
+    """
+    G, k, d_h = layer.G, layer.k, layer.d_h
+    M = O.shape[1]
+    blocks = []
+    for g in range(G):
+        for r in range(k):
+            o = O[g * k + r]
+            if layer.variant == "weighted_concat":
+                o = o * routing.p_sel[:, g, r][:, None]
+            blocks.append(o)
+    if layer.variant == "gqe":
+        slot = np.zeros((M, d_h))
+        for g in range(G):
+            for r in range(k):
+                slot += routing.w[:, g, r][:, None] * O[g * k + r]
+        blocks.append(slot)
+    if layer.shared:
+        blocks.append(O[G * k])
+    return np.concatenate(blocks, axis=1)
+
+
+def output_projection(Z: np.ndarray, W_o: np.ndarray) -> np.ndarray:
+    """y = Z W_o^T."""
+    return Z @ W_o.T
+
+
+# ----------------------------------------------------------------------------------------
+# Step 8: Switch-style load-balancing loss ([README] Algorithm Overview; [Summary]
+# Training and Loss). The caller's 0.01 coefficient ([README] Usage) is not applied.
+# ----------------------------------------------------------------------------------------
+
+def aux_loss(counts: np.ndarray, prob_sum: np.ndarray, M: int, G: int, k: int) -> float:
+    """L = (1/G) sum_g E sum_j f_{g,j} Pbar_{g,j}, f = counts / (M k), Pbar = prob_sum / M."""
+    N = counts.shape[0]
+    E = N // G
+    f = counts.astype(np.float64).reshape(G, E) / (M * k)
+    P = prob_sum.reshape(G, E) / M
+    return float((E * (f * P).sum(axis=1)).mean())
+
+
+# ----------------------------------------------------------------------------------------
+# Whole layer.
+# ----------------------------------------------------------------------------------------
+
+@dataclass
+class Result:
+    routing: Routing
+    K: np.ndarray
+    V: np.ndarray
+    Q: np.ndarray          # [S, M, d_h]: routed streams then the shared stream
+    O: np.ndarray          # [S, M, d_h]
+    Z: np.ndarray          # [M, D_o]
+    y: np.ndarray          # [M, d]
+    aux: float
+    extra: dict = field(default_factory=dict)
+
+
+def forward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_shared,
+            W_o) -> Result:
+    """The full GQE attention forward pass on x [B*T, dim] (float64 arrays)."""
+    M = x.shape[0]
+    assert M == B * T
+    rt = route(x, W_r, layer.G, layer.k)
+    K, V = kv_projection(x, W_k, W_v, layer.G, layer.d_h)
+    Q = routed_queries(x, W_q, rt.sel, layer.G, layer.E, layer.d_h)
+    if layer.shared:
+        Q = np.concatenate([Q, shared_query(x, W_shared)[None]], axis=0)
+    O = attention(Q, K, V, B, T, layer.k, layer.G, layer.causal)
+    Z = combine(O, rt, layer)
+    y = output_projection(Z, W_o)
+    aux = aux_loss(rt.counts, rt.prob_sum, M, layer.G, layer.k)
+    return Result(rt, K, V, Q, O, Z, y, aux)
+
+
+def forward_rows(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_shared,
+                 W_o, rows: np.ndarray) -> dict:
+    """y for a subset of token rows only (the same steps restricted to those rows).
+
+    Routing and the aux loss use every token (the loss is a mean over all of them). K/V
+    are projected for each sequence's prefix that the sampled rows attend to. Returns a
+    dict with y [R, d], Z [R, D_o], sel/gates/w for the rows, counts, prob_sum and aux.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    M = x.shape[0]
+    rt = route(x, W_r, layer.G, layer.k)
+    aux = aux_loss(rt.counts, rt.prob_sum, M, layer.G, layer.k)
+    xs = x[rows]
+    sel = rt.sel[rows]
+    Q = routed_queries(xs, W_q, sel, layer.G, layer.E, layer.d_h)
+    if layer.shared:
+        Q = np.concatenate([Q, shared_query(xs, W_shared)[None]], axis=0)
+    S = Q.shape[0]
+    O = np.empty((S, rows.size, layer.d_h))
+    b_of = rows // T
+    t_of = rows % T
+    for b in np.unique(b_of):
+        m = np.nonzero(b_of == b)[0]
+        last = T if not layer.causal else int(t_of[m].max()) + 1
+        xb = x[b * T: b * T + last]
+        K, V = kv_projection(xb, W_k, W_v, layer.G, layer.d_h)
+        for s in range(S):
+            h = stream_kv_head(s, layer.k, layer.G)
+            O[s, m] = attention_rows(Q[s, m], t_of[m], K[h], V[h], layer.causal)
+    sub = Routing(rt.logits[rows], rt.p[rows], sel, rt.p_sel[rows], rt.gates[rows],
+                  rt.w[rows], rt.counts, rt.prob_sum)
+    Z = combine(O, sub, layer)
+    y = output_projection(Z, W_o)
+    return dict(y=y, Z=Z, O=O, sel=sel, gates=rt.gates[rows], w=rt.w[rows],
+                p_sel=rt.p_sel[rows], counts=rt.counts, prob_sum=rt.prob_sum, aux=aux,
+                routing=rt)
