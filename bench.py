@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""GQE attention prefill benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one gqe_forward over the workload (router, K/V/shared projection, bucketed
+routed Q projection, attention, output construction, W_o, aux loss) with its inputs
+already in HBM. Before each timed step the L2 cache is flushed by writing 256 MiB (the
+inputs of the default workload are smaller than L2); each step is timed with CUDA events
+on the launching stream, and the K step times are summed. Under torchrun every rank runs
+its own replica of the workload (the layer has no cross-sequence exchange), the time is
+the maximum over ranks and `value` counts the tokens of all ranks.
+
+Rank 0 prints one JSON line. Besides the metric it reports:
+  roofline      the attention kernel's achieved TFLOP/s (active FLOPs / its event-timed
+                duration) against the measured bf16 dense peak;
+  speedup_vs_kE the same kernels with every expert active (k = E), the in-run GQA
+                comparator;
+  e2e           the same metric through the public API with host buffers: pinned host x
+                copied in and y and the aux loss copied out inside each timed step;
+  cpu_baseline  the float64 CPU oracle on a bounded sample of the same workload (rank 0,
+                one GPU only).
+--impl reference times the CPU oracle alone (the only reference there is: the pages ship
+no code), one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from moe_query_head_b200 import workloads as W  # noqa: E402
+
+METRIC = "GQE prefill tokens/s @1 B200; % bf16 tensor peak (active FLOPs); speedup vs k=E"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_t16k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=8192,
+                    help="query rows in the oracle's bounded sample")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# ----------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        busy = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------------
+# The CPU oracle on a bounded sample (cpu_baseline and --impl reference).
+# ----------------------------------------------------------------------------------------
+
+def oracle_sample(inp: W.Inputs, n_rows: int) -> dict:
+    """Time the oracle's steps on the whole workload, except that the per-row steps (routed
+    and shared queries, attention, output construction, W_o) run on n_rows evenly spaced
+    token rows; the full-workload time is the whole-workload steps plus the per-row time
+    scaled by M / n_rows."""
+    import oracle
+    wl = inp.wl
+    f = inp.f64
+    x = f("x")
+    layer = oracle.Layer(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, shared=wl.shared,
+                         variant=wl.variant, causal=wl.causal)
+    t0 = time.perf_counter()
+    rt = oracle.route(x, f("W_r"), wl.G, wl.k)
+    oracle.aux_loss(rt.counts, rt.prob_sum, wl.M, wl.G, wl.k)
+    K, V = oracle.kv_projection(x, f("W_k"), f("W_v"), wl.G, wl.d_h)
+    t1 = time.perf_counter()
+    rows = np.linspace(0, wl.M - 1, n_rows).round().astype(np.int64)
+    xs = x[rows]
+    Q = oracle.routed_queries(xs, f("W_q"), rt.sel[rows], wl.G, wl.E, wl.d_h)
+    if wl.shared:
+        Q = np.concatenate([Q, oracle.shared_query(xs, f("W_shared"))[None]], axis=0)
+    O = np.empty((Q.shape[0], rows.size, wl.d_h))
+    for b in range(wl.B):
+        m = np.nonzero(rows // wl.T == b)[0]
+        if m.size == 0:
+            continue
+        tk = slice(b * wl.T, (b + 1) * wl.T)
+        for s in range(Q.shape[0]):
+            h = oracle.stream_kv_head(s, wl.k, wl.G)
+            O[s, m] = oracle.attention_rows(Q[s, m], rows[m] % wl.T, K[h, tk], V[h, tk], wl.causal)
+    sub = oracle.Routing(rt.logits[rows], rt.p[rows], rt.sel[rows], rt.p_sel[rows],
+                         rt.gates[rows], rt.w[rows], rt.counts, rt.prob_sum)
+    Z = oracle.combine(O, sub, layer)
+    oracle.output_projection(Z, f("W_o"))
+    t2 = time.perf_counter()
+    est = (t1 - t0) + (t2 - t1) * wl.M / rows.size
+    return {"whole_s": t1 - t0, "rows_s": t2 - t1, "rows": int(rows.size), "est_s": est,
+            "tokens_per_s": wl.M / est}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_sample_desc(wl, rows):
+    return (f"{wl.name}: routing, aux loss and K/V projection over all {wl.M} tokens; "
+            f"queries, attention, output construction and W_o on {rows} evenly spaced token "
+            f"rows, scaled by {wl.M}/{rows} (float64 numpy oracle)")
+
+
+# ----------------------------------------------------------------------------------------
+# Our arm.
+# ----------------------------------------------------------------------------------------
+
+def _upload(inp, torch):
+    out = {}
+    for n in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o"):
+        a = inp.raw(n)
+        if a is None:
+            out[n] = None
+        elif inp.wl.dtype == "bf16":
+            out[n] = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+        else:
+            out[n] = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return out
+
+
+def bench_ours(args, rank, world, dist):
+    import torch
+    from moe_query_head_b200 import gqe as G
+
+    wl = W.WORKLOADS[args.workload]
+    inp = W.generate(wl)
+    dev = _upload(inp, torch)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    code = G.GQE_BF16 if wl.dtype == "bf16" else G.GQE_F32
+    variant = W.VARIANT_IDS[wl.variant]
+    W_s = dev["W_shared"] if wl.shared else None
+
+    h = G.gqe_create(wl.dim, wl.N, wl.G, wl.k, wl.d_h, code, wl.M)
+    out = torch.empty((wl.M, wl.dim), dtype=tdt, device="cuda")
+    aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+    # the all-active comparator: same inputs, k = E, W_o of the wider concatenation
+    kE = wl.all_active()
+    hE = G.gqe_create(wl.dim, wl.N, wl.G, kE.k, wl.d_h, code, wl.M)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(wl.seed + 1000)
+    W_oE = (torch.randn((wl.dim, kE.D_o), generator=gen, device="cuda") * 0.02).to(tdt)
+    outE = torch.empty_like(out)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def fwd(handle, k, W_o, o):
+        G.gqe_forward(handle, dev["x"], wl.B, wl.T, dev["W_r"], dev["W_q"], dev["W_k"],
+                      dev["W_v"], W_s, W_o, wl.N, wl.G, k, wl.d_h, variant, int(wl.causal), o,
+                      aux)
+
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(G.GQE_NUM_STAGES + 1)]
+    for e in stage_ev:
+        e.record()
+    torch.cuda.synchronize()
+
+    def timed(fn, steps, stages=None):
+        s_ev = torch.cuda.Event(enable_timing=True)
+        e_ev = torch.cuda.Event(enable_timing=True)
+        total = 0.0
+        st_tot = np.zeros(G.GQE_NUM_STAGES)
+        for _ in range(steps):
+            flush.zero_()
+            s_ev.record()
+            fn()
+            e_ev.record()
+            torch.cuda.synchronize()
+            total += s_ev.elapsed_time(e_ev)
+            if stages:
+                for i in range(G.GQE_NUM_STAGES):
+                    st_tot[i] += stages[i].elapsed_time(stages[i + 1])
+        return total, st_tot
+
+    gpu_id = torch.cuda.get_device_properties(0).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+
+    # warm-up
+    for _ in range(args.warmup):
+        fwd(h, wl.k, dev["W_o"], out)
+        fwd(hE, kE.k, W_oE, outE)
+    torch.cuda.synchronize()
+    st = G.gqe_check_device_status(h)
+    if st != G.GQE_OK:
+        raise RuntimeError("device status after warm-up: " + G.status_str(st))
+
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    G.gqe_set_stage_events(h, stage_ev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms, stage_ms = timed(lambda: fwd(h, wl.k, dev["W_o"], out), args.steps, stage_ev)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    G.gqe_set_stage_events(h, None)
+    launches = G.gqe_kernel_launches(h)
+    totalE_ms, _ = timed(lambda: fwd(hE, kE.k, W_oE, outE), args.steps)
+
+    # end-to-end through the public API with host buffers
+    x_host = torch.empty(dev["x"].shape, dtype=tdt).pin_memory()
+    x_host.copy_(dev["x"].cpu())
+    y_host = torch.empty(out.shape, dtype=tdt).pin_memory()
+    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(dev["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        G.gqe_forward(h, x_dev, wl.B, wl.T, dev["W_r"], dev["W_q"], dev["W_k"], dev["W_v"],
+                      W_s, dev["W_o"], wl.N, wl.G, wl.k, wl.d_h, variant, int(wl.causal), out,
+                      aux)
+        y_host.copy_(out, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms, _ = timed(e2e_step, args.steps)
+    clocks = sampler.stop()
+    st = G.gqe_check_device_status(h)
+    if st != G.GQE_OK:
+        raise RuntimeError("device status after timing: " + G.status_str(st))
+
+    if dist:
+        import torch.distributed as td
+        t = torch.tensor([total_ms, totalE_ms, e2e_ms, stage_ms[5]], device="cuda",
+                         dtype=torch.float64)
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+        total_ms, totalE_ms, e2e_ms, att_ms_tot = [float(v) for v in t.cpu()]
+    else:
+        att_ms_tot = float(stage_ms[5])
+
+    peaks, peak_src = load_peaks()
+    ms = total_ms / args.steps
+    msE = totalE_ms / args.steps
+    tokens = wl.M * world
+    value = tokens / (total_ms / args.steps / 1e3)
+    flops = wl.active_flops()
+    S = wl.n_streams
+    att_flops = (2.0 * wl.B * wl.d_h * wl.T * (wl.T + 1) * S if wl.causal
+                 else 4.0 * wl.B * wl.d_h * wl.T * wl.T * S)
+    att_ms = att_ms_tot / args.steps
+    att_tflops = att_flops / (att_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded normal inputs and random-init weights of the layer shapes)",
+        "config": {"workload": wl.name, "dim": wl.dim, "N": wl.N, "G": wl.G, "k": wl.k,
+                   "d_h": wl.d_h, "B": wl.B, "T": wl.T, "variant": wl.variant,
+                   "shared": wl.shared, "causal": wl.causal,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "active_tflops": flops / (ms / 1e3) / 1e12,
+        "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / peak,
+        "speedup_vs_kE": msE / ms,
+        "kE_tokens_per_s": tokens / (msE / 1e3),
+        "stages_ms": {G.gqe_stage_name(i): float(stage_ms[i] / args.steps)
+                      for i in range(G.GQE_NUM_STAGES)},
+        "roofline": {"kernel": "attention", "bound": "tensor", "achieved": att_tflops,
+                     "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": None},
+        "e2e": {"value": tokens / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size() + 4)},
+        "gpu_launches": int(launches * args.steps),
+        "clocks": clocks,
+    }
+    G.gqe_destroy(h)
+    G.gqe_destroy(hE)
+    return res, inp
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = W.WORKLOADS[args.workload]
+        inp = W.generate(wl)
+        rows = max(16, min(args.cpu_rows, 256))
+        for _ in range(args.warmup):
+            oracle_sample(inp, rows)
+        samples = [oracle_sample(inp, rows) for _ in range(args.steps)]
+        est = sum(s["est_s"] for s in samples) / len(samples)
+        value = wl.M / est
+        res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+               "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": wl.name, "dim": wl.dim, "N": wl.N, "G": wl.G, "k": wl.k,
+                          "d_h": wl.d_h, "B": wl.B, "T": wl.T, "variant": wl.variant},
+               "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": cpu_sample_desc(wl, rows)},
+               "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return 0
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as td
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    else:
+        torch.cuda.set_device(0)
+    res, inp = bench_ours(args, rank, world, dist)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            s = oracle_sample(inp, args.cpu_rows)
+            res["cpu_baseline"] = {"value": s["tokens_per_s"], "unit": "tokens/s",
+                                   "cores": blas_threads(), "kind": "oracle",
+                                   "sample": cpu_sample_desc(inp.wl, s["rows"]),
+                                   "seconds": s["whole_s"] + s["rows_s"]}
+        print(json.dumps(res))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

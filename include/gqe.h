@@ -1,0 +1,178 @@
+/*
+ * gqe.h — C ABI of the Grouped Query Experts (GQE) attention forward (prefill) library.
+ *
+ * GQE is a mixture-of-experts layer on grouped-query attention ("GQE: Grouped Query
+ * Experts", FrontiersMindAI/GQE README, Algorithm Overview): N query-head experts in G
+ * groups, each group with one dense KV head. Per token and per group a router takes a
+ * softmax over the group's E = N/G experts and keeps the top k; only the selected query
+ * heads plus one always-on shared head are projected and attend over the dense K/V; the
+ * outputs are combined ("gqe", "weighted_concat", "hard_concat": README, Ablations and
+ * Parameters) and projected by W_o. A Switch-style load-balancing loss is reduced on the
+ * side (README, Algorithm Overview; gist.science summary, Training and Loss).
+ *
+ * Conventions for every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous, row-major,
+ *     16-byte aligned, in the handle's dtype (bf16 or fp32) unless stated otherwise.
+ *   - Weights use the nn.Linear layout [out, in]; y = x W^T; there are no biases.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Work is enqueued on it; no entry point synchronises the device except
+ *     gqe_check_device_status.
+ *   - Errors are reported by return code only. On an error return nothing has been
+ *     launched. No entry point aborts or throws.
+ *   - A handle may be used by one stream at a time.
+ */
+#ifndef GQE_H
+#define GQE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gqe_ctx* gqe_handle;
+
+typedef enum {
+    GQE_OK = 0,
+    GQE_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size, mismatch with create */
+    GQE_ERR_UNSUPPORTED = 2,  /* a shape this build does not implement (see gqe_create)   */
+    GQE_ERR_WORKSPACE = 3,    /* B*T larger than the handle's max_tokens                   */
+    GQE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed                          */
+    GQE_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up (see status below)      */
+} gqe_status;
+
+typedef enum {
+    GQE_VARIANT_GQE = 0,             /* routed blocks + renormalised slot + shared block */
+    GQE_VARIANT_WEIGHTED_CONCAT = 1, /* routed blocks scaled by raw router p + shared    */
+    GQE_VARIANT_HARD_CONCAT = 2      /* routed blocks as computed + shared               */
+} gqe_variant;
+
+typedef enum { GQE_BF16 = 0, GQE_F32 = 1 } gqe_dtype;
+
+/* Internal tensors that gqe_get_tensor can copy out (for tests and inspection). */
+typedef enum {
+    GQE_T_K = 0,      /* [G, M, d_h]       keys, dtype                                      */
+    GQE_T_V = 1,      /* [G, d_h, M]       values, stored transposed (token index fastest)  */
+    GQE_T_Q = 2,      /* [S, M, d_h]       query streams (routed g*k+r, then shared), dtype */
+    GQE_T_Z = 3,      /* [M, D_o]          concatenated attention output, dtype             */
+    GQE_T_PSEL = 4,   /* [M, G, k] float   router softmax p of each selected expert         */
+    GQE_T_W = 5,      /* [M, G, k] float   slot weights (p renormalised over all G*k)       */
+    GQE_T_LOGITS = 6  /* [M, N]    float   router logits                                    */
+} gqe_tensor;
+
+/*
+ * gqe_create — make a handle for one layer shape and allocate its device workspace.
+ *
+ *   dim         hidden size d ("dim", README Parameters), 16 <= dim, dim % 16 == 0 for bf16.
+ *   N           routed query-head experts ("num_query_experts"); N % G == 0 (README
+ *               Parameters), N <= 64.
+ *   G           GQA groups = dense KV heads ("num_kv_heads").
+ *   k           experts kept per group per token ("top_k"), 1 <= k <= min(N/G, 8).
+ *   d_h         head dimension ("head_dim"; its default dim/N is applied by the Python
+ *               binding, not here). bf16: d_h in {16, 32, 48, 64, 80, 96, 112, 128};
+ *               fp32: d_h % 4 == 0 and d_h <= 128.
+ *   dtype       GQE_BF16 (bf16 storage, fp32 accumulation) or GQE_F32.
+ *   max_tokens  the largest B*T any gqe_forward on this handle will use.
+ *
+ * Allocates (cudaMalloc, on the current device) the workspace for K, V, the query streams,
+ * Z, the routing tables and a device status word; the handle owns it until gqe_destroy.
+ * Returns GQE_ERR_INVALID_ARG / GQE_ERR_UNSUPPORTED for bad shapes and GQE_ERR_CUDA if an
+ * allocation fails (*h is then NULL).
+ */
+gqe_status gqe_create(gqe_handle* h, int dim, int N, int G, int k, int d_h, gqe_dtype dtype,
+                      int64_t max_tokens);
+
+/*
+ * gqe_forward — one GQE attention forward pass on B sequences of T tokens.
+ *
+ *   x         [B*T, dim]        input activations (token-major; sequence b owns rows b*T..).
+ *   W_r       [N, dim]          router; expert e = g*E + j belongs to group g.
+ *   W_q       [N*d_h, dim]      query projections; expert e owns rows e*d_h .. e*d_h+d_h-1.
+ *   W_k, W_v  [G*d_h, dim]      dense key / value projections; head g owns rows g*d_h...
+ *   W_shared  [d_h, dim]        always-on shared query head (README, Algorithm Overview;
+ *                               it reads KV head 0), or NULL for a layer without it.
+ *   W_o       [dim, D_o]        output projection, D_o = (G*k + [variant==GQE] +
+ *                               [W_shared != NULL]) * d_h. Z's column blocks are: routed
+ *                               streams g-major then rank r, then the slot (GQE only), then
+ *                               the shared stream.
+ *   N, G, k, d_h                must equal the values given to gqe_create.
+ *   variant   gqe_variant (gist.science summary, Output Construction; README Ablations).
+ *   causal    1: token t attends to positions <= t of its own sequence; 0: to all T.
+ *   out       [B*T, dim]        result y = Z W_o^T, written in the handle's dtype.
+ *   aux_loss  device float*     the Switch load-balancing loss (without the caller's 0.01
+ *                               coefficient, README Usage), or NULL to skip writing it.
+ *   stream    cudaStream_t      as void*.
+ *
+ * Routing per token and group: softmax over the E logits in fp32, top-k on the fp32
+ * logits with the lower expert index winning ties, selected experts listed in ascending
+ * index. Allocates nothing and does not synchronise. Returns GQE_ERR_WORKSPACE if
+ * B*T > max_tokens, GQE_ERR_INVALID_ARG for null required pointers, pointers not 16-byte
+ * aligned, B < 1, T < 1, or N/G/k/d_h different from the handle's.
+ */
+gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                       const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
+                       const void* W_o, int N, int G, int k, int d_h, int variant, int causal,
+                       void* out, float* aux_loss, void* stream);
+
+/*
+ * gqe_get_routing — copy the routing of the last gqe_forward on this handle.
+ *   sel        [M, G, k] int32   selected expert index j within the group, ascending.
+ *   gates      [M, G, k] float   p renormalised within the group (sums to 1 per group).
+ *   counts     [N] int32         tokens routed to each expert.
+ *   mean_prob  [N] float         mean over tokens of the router softmax p.
+ * Any pointer may be NULL (that output is skipped). Device pointers; enqueued on stream.
+ */
+gqe_status gqe_get_routing(gqe_handle h, int32_t* sel, float* gates, int32_t* counts,
+                           float* mean_prob, void* stream);
+
+/*
+ * gqe_get_tensor — copy an internal tensor of the last gqe_forward (see gqe_tensor for
+ * shapes) into the caller's device buffer dst of `bytes` bytes. Returns
+ * GQE_ERR_INVALID_ARG if `bytes` is smaller than the tensor.
+ */
+gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void* stream);
+
+/*
+ * gqe_check_device_status — synchronise `stream`, then read and clear the handle's device
+ * status word. Returns GQE_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * check (its output is then invalid), GQE_ERR_CUDA if the stream reports an error, else
+ * GQE_OK.
+ */
+gqe_status gqe_check_device_status(gqe_handle h, void* stream);
+
+/* gqe_set_spin_limit — iteration cap of the device-side waits (0 = default). For tests
+ * of the timeout path: a tiny limit makes the waits give up and report GQE_ERR_TIMEOUT. */
+gqe_status gqe_set_spin_limit(gqe_handle h, int64_t limit);
+
+/*
+ * gqe_set_stage_events — for measurement: record caller-created CUDA events (cudaEvent_t
+ * passed as void*) on the forward's stream around its stages. count = 0 turns recording
+ * off; otherwise count must be GQE_NUM_STAGES + 1: events[i] is recorded just before stage
+ * i and events[GQE_NUM_STAGES] after the last. The events must outlive the forwards that
+ * record them. Stage names: gqe_stage_name.
+ */
+#define GQE_NUM_STAGES 8
+gqe_status gqe_set_stage_events(gqe_handle h, void* const* events, int count);
+
+/* gqe_stage_name — "dense_proj", "route", "route_scan", "bucket", "qproj", "attention",
+ * "combine", "oproj" for i = 0..7; NULL otherwise. */
+const char* gqe_stage_name(int i);
+
+/* gqe_destroy — free the handle and its workspace (synchronises the device first). */
+void gqe_destroy(gqe_handle h);
+
+/* gqe_status_str — static text for a status code. */
+const char* gqe_status_str(int status);
+
+/* gqe_workspace_bytes — device bytes gqe_create would allocate for this shape, or -1. */
+int64_t gqe_workspace_bytes(int dim, int N, int G, int k, int d_h, gqe_dtype dtype,
+                            int64_t max_tokens);
+
+/* gqe_kernel_launches — kernels the last gqe_forward on this handle launched. */
+int gqe_kernel_launches(gqe_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQE_H */

@@ -1,0 +1,103 @@
+// Internal declarations shared by the GQE CUDA library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gqe.h"
+
+namespace gqe {
+
+// Tokens per router block: the per-block partial statistics are indexed by this.
+constexpr int kRouteBlock = 128;
+// Maximum sizes this build supports.
+constexpr int kMaxExperts = 64;
+constexpr int kMaxTopK = 8;
+
+// Device status word values (written by kernels whose bounded waits give up).
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 1;
+
+// ---------------------------------------------------------------------------------------
+// Element access helpers: every kernel computes in fp32; storage is float or bf16.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// Affine map from a GEMM output element (row m, column c) to memory: column c belongs to
+// head c / head_w at offset c % head_w; address = base + head*head_stride + m*row_stride
+// + (c % head_w)*col_stride (in elements of the output type).
+struct OutMap {
+  void* base;
+  int64_t head_stride;
+  int64_t row_stride;
+  int64_t col_stride;
+  int head_w;
+  int f32;  // 1: store float; 0: store the handle's storage type
+};
+
+// ---------------------------------------------------------------------------------------
+// The handle.
+// ---------------------------------------------------------------------------------------
+struct Workspace {
+  void* K = nullptr;        // [G, M, d_h]
+  void* Vt = nullptr;       // [G, d_h, M]
+  void* Q = nullptr;        // [S, M, d_h]
+  void* Z = nullptr;        // [M, D_o]
+  float* logits = nullptr;  // [M, N]
+  int32_t* sel = nullptr;   // [M, G, k]
+  float* psel = nullptr;    // [M, G, k]
+  float* gates = nullptr;   // [M, G, k]
+  float* w = nullptr;       // [M, G, k]
+  int32_t* part_counts = nullptr;  // [nblk, N]; after the scan: bucket base of (blk, e)
+  float* part_prob = nullptr;      // [nblk, N]
+  int32_t* counts = nullptr;       // [N]
+  float* mean_prob = nullptr;      // [N]
+  int32_t* offsets = nullptr;      // [N + 1] bucket start of each expert
+  int32_t* bucket = nullptr;       // [M * G * k] entries (token << 3) | rank, per expert
+  int32_t* status = nullptr;       // device status word
+  void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
+  void* base = nullptr;            // the single allocation
+  size_t bytes = 0;
+};
+
+}  // namespace gqe
+
+struct gqe_ctx {
+  int dim, N, G, k, d_h, E;
+  gqe_dtype dtype;
+  int64_t max_tokens;
+  int esz;  // bytes per stored element
+  int device;
+  int num_sms;
+  int64_t spin_limit;
+  gqe::Workspace ws;
+  // measurement: events recorded around the stages (GQE_NUM_STAGES + 1, or none)
+  cudaEvent_t stage_events[GQE_NUM_STAGES + 1] = {};
+  int n_stage_events = 0;
+  // state of the last forward
+  int last_M = 0, last_S = 0, last_Do = 0, last_launches = 0;
+};
+
+namespace gqe {
+
+// Launchers implemented in the .cu files. Each returns the number of kernels launched
+// (>= 0) or -1 if a launch failed.
+int launch_simt_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
+                           const void* W_v, const void* W_shared, cudaStream_t st);
+int launch_route_select(gqe_ctx* h, int M, cudaStream_t st);
+int launch_route_scan_aux(gqe_ctx* h, int M, float* aux_out, cudaStream_t st);
+int launch_bucket(gqe_ctx* h, int M, cudaStream_t st);
+int launch_simt_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);
+int launch_simt_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,
+                          int causal, int Do, cudaStream_t st);
+int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st);
+int launch_simt_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
+
+}  // namespace gqe

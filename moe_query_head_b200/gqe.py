@@ -1,0 +1,199 @@
+"""ctypes binding of the GQE C ABI (include/gqe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and passes torch tensors'
+device pointers and the current CUDA stream through unchanged; all computation happens in
+libgqe.so's kernels. If the library is missing, importing this module raises: there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqe.so")
+
+GQE_OK, GQE_ERR_INVALID_ARG, GQE_ERR_UNSUPPORTED, GQE_ERR_WORKSPACE, GQE_ERR_CUDA, \
+    GQE_ERR_TIMEOUT = range(6)
+GQE_BF16, GQE_F32 = 0, 1
+VARIANTS = {"gqe": 0, "weighted_concat": 1, "hard_concat": 2}
+TENSORS = {"K": 0, "V": 1, "Q": 2, "Z": 3, "PSEL": 4, "W": 5, "LOGITS": 6}
+
+EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
+            "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
+            "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
+            "gqe_stage_name")
+GQE_NUM_STAGES = 8
+
+
+class GQEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_str(status)}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"GQE CUDA library not built ({_LIB_PATH} missing); run "
+            "`python -m moe_query_head_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.gqe_create.argtypes = [ctypes.POINTER(P), I, I, I, I, I, I, I64]
+    lib.gqe_create.restype = I
+    lib.gqe_forward.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.gqe_forward.restype = I
+    lib.gqe_get_routing.argtypes = [P, P, P, P, P, P]
+    lib.gqe_get_routing.restype = I
+    lib.gqe_get_tensor.argtypes = [P, I, P, SZ, P]
+    lib.gqe_get_tensor.restype = I
+    lib.gqe_check_device_status.argtypes = [P, P]
+    lib.gqe_check_device_status.restype = I
+    lib.gqe_set_spin_limit.argtypes = [P, I64]
+    lib.gqe_set_spin_limit.restype = I
+    lib.gqe_destroy.argtypes = [P]
+    lib.gqe_destroy.restype = None
+    lib.gqe_status_str.argtypes = [I]
+    lib.gqe_status_str.restype = ctypes.c_char_p
+    lib.gqe_workspace_bytes.argtypes = [I, I, I, I, I, I, I64]
+    lib.gqe_workspace_bytes.restype = I64
+    lib.gqe_kernel_launches.argtypes = [P]
+    lib.gqe_kernel_launches.restype = I
+    lib.gqe_set_stage_events.argtypes = [P, ctypes.POINTER(P), I]
+    lib.gqe_set_stage_events.restype = I
+    lib.gqe_stage_name.argtypes = [I]
+    lib.gqe_stage_name.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.gqe_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != GQE_OK:
+        raise GQEError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def gqe_workspace_bytes(dim, N, G, k, d_h, dtype, max_tokens) -> int:
+    return int(lib.gqe_workspace_bytes(dim, N, G, k, d_h, dtype, max_tokens))
+
+
+def gqe_create(dim, N, G, k, d_h, dtype, max_tokens) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib.gqe_create(ctypes.byref(h), dim, N, G, k, d_h, dtype, max_tokens), "gqe_create")
+    return h
+
+
+def gqe_forward(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, variant, causal,
+                out, aux_loss=None, stream=None) -> None:
+    _check(lib.gqe_forward(h, _ptr(x), B, T, _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v),
+                           _ptr(W_shared), _ptr(W_o), N, G, k, d_h, variant, causal, _ptr(out),
+                           _ptr(aux_loss), _stream(stream)), "gqe_forward")
+
+
+def gqe_get_routing(h, sel=None, gates=None, counts=None, mean_prob=None, stream=None) -> None:
+    _check(lib.gqe_get_routing(h, _ptr(sel), _ptr(gates), _ptr(counts), _ptr(mean_prob),
+                               _stream(stream)), "gqe_get_routing")
+
+
+def gqe_get_tensor(h, which: str, dst, stream=None) -> None:
+    _check(lib.gqe_get_tensor(h, TENSORS[which], _ptr(dst), dst.numel() * dst.element_size(),
+                              _stream(stream)), "gqe_get_tensor")
+
+
+def gqe_check_device_status(h, stream=None) -> int:
+    return int(lib.gqe_check_device_status(h, _stream(stream)))
+
+
+def gqe_set_spin_limit(h, limit: int) -> None:
+    _check(lib.gqe_set_spin_limit(h, int(limit)), "gqe_set_spin_limit")
+
+
+def gqe_destroy(h) -> None:
+    lib.gqe_destroy(h)
+
+
+def gqe_kernel_launches(h) -> int:
+    return int(lib.gqe_kernel_launches(h))
+
+
+def gqe_stage_name(i: int):
+    r = lib.gqe_stage_name(int(i))
+    return None if r is None else r.decode()
+
+
+def gqe_set_stage_events(h, events) -> None:
+    """events: GQE_NUM_STAGES + 1 torch.cuda.Event(enable_timing=True) objects, each
+    already recorded once (torch creates the underlying cudaEvent_t lazily), or None."""
+    if not events:
+        _check(lib.gqe_set_stage_events(h, None, 0), "gqe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib.gqe_set_stage_events(h, arr, len(events)), "gqe_set_stage_events")
+
+
+class GQEAttention:
+    """One GQE attention layer shape on the current CUDA device.
+
+    The constructor arguments follow the module of the "GQE: Grouped Query Experts" README
+    (Usage, Parameters): dim, num_query_experts, num_kv_heads, top_k, head_dim (default
+    dim // num_query_experts), variant. Weights are passed to `forward` by the caller.
+    """
+
+    def __init__(self, dim, num_query_experts=16, num_kv_heads=8, top_k=1, head_dim=None,
+                 variant="gqe", dtype=torch.bfloat16, max_tokens=65536, shared=True,
+                 causal=True):
+        if num_query_experts % num_kv_heads != 0:
+            raise ValueError("num_query_experts must be divisible by num_kv_heads")
+        self.dim, self.N, self.G, self.k = dim, num_query_experts, num_kv_heads, top_k
+        self.d_h = head_dim if head_dim is not None else dim // num_query_experts
+        self.variant = variant
+        self.dtype = dtype
+        self.shared = shared
+        self.causal = causal
+        self.max_tokens = max_tokens
+        code = GQE_F32 if dtype == torch.float32 else GQE_BF16
+        self.handle = gqe_create(dim, self.N, self.G, self.k, self.d_h, code, max_tokens)
+        self.aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    @property
+    def D_o(self) -> int:
+        return (self.G * self.k + (self.variant == "gqe") + self.shared) * self.d_h
+
+    def forward(self, x, W_r, W_q, W_k, W_v, W_shared, W_o, B, T, out=None, stream=None):
+        if out is None:
+            out = torch.empty((B * T, self.dim), dtype=self.dtype, device=x.device)
+        gqe_forward(self.handle, x, B, T, W_r, W_q, W_k, W_v, W_shared if self.shared else None,
+                    W_o, self.N, self.G, self.k, self.d_h, VARIANTS[self.variant],
+                    int(self.causal), out, self.aux, stream)
+        return out
+
+    def collect_aux_loss(self):
+        """The load-balancing loss of the last forward, as a device scalar (the README's
+        collect_aux_loss; the caller applies its 0.01 coefficient)."""
+        return self.aux[0]
+
+    def close(self):
+        if self.handle:
+            gqe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
