@@ -159,6 +159,35 @@ gqe_status gqe_set_stage_events(gqe_handle h, void* const* events, int count);
  * "combine", "oproj" for i = 0..7; NULL otherwise. */
 const char* gqe_stage_name(int i);
 
+/*
+ * gqe_route_static — the router's selection and load statistics from precomputed router
+ * logits, allocating nothing. The paper has no counterpart: this entry point exists for
+ * callers that cannot call cudaMalloc (their device memory belongs to another allocator
+ * or a fixed budget, they are plug-in code handed only input and output buffers, or they
+ * cannot accept cudaMalloc's device-wide synchronisation), and so cannot create a handle.
+ *
+ *   logits     [M, N] float (device)  router logits x W_r^T.
+ *   sel        [M, G, k] int32        selected expert index j in its group, ascending
+ *                                     (top-k of the fp32 logits, lower index wins ties).
+ *   gates      [M, G, k] float        softmax probability renormalised within the group.
+ *   counts     [N] int32              tokens routed to each expert.
+ *   mean_prob  [N] float              mean over tokens of the per-group softmax p.
+ *   aux_loss   device float* or NULL  the Switch load-balancing loss (as gqe_forward).
+ *
+ * Scratch lives in one file-scope device array of 2.5 MiB (+256 B), held by every GPU that
+ * loads the library until the process exits. Limits: M <= 131072 and M*G*k <= 262144;
+ * larger calls return GQE_ERR_WORKSPACE and launch nothing. N <= 64, k <= 8
+ * (GQE_ERR_UNSUPPORTED otherwise). The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. All calls share the one array: calls whose kernels overlap
+ * on the GPU (different streams, or different threads without ordering) race and may
+ * return wrong results; order them on one stream. Every scratch element a call reads is
+ * written earlier in the same call, so nothing needs clearing between calls.
+ */
+gqe_status gqe_route_static(const float* logits, int M, int N, int G, int k, int32_t* sel,
+                            float* gates, int32_t* counts, float* mean_prob, float* aux_loss,
+                            void* stream);
+
 /* gqe_destroy — free the handle and its workspace (synchronises the device first). */
 void gqe_destroy(gqe_handle h);
 

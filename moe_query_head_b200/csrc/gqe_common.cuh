@@ -87,6 +87,19 @@ struct gqe_ctx {
 
 namespace gqe {
 
+// Router kernels (defined in route.cu), also launched by the static-scratch entry point.
+__global__ void __launch_bounds__(kRouteBlock)
+route_select_kernel(const float* __restrict__ logits, int M, int N, int G,
+                                    int k, int32_t* __restrict__ sel, float* __restrict__ psel,
+                                    float* __restrict__ gates, float* __restrict__ wslot,
+                                    int32_t* __restrict__ part_counts,
+                                    float* __restrict__ part_prob);
+__global__ void route_scan_aux_kernel(int32_t* __restrict__ part_counts,
+                                      const float* __restrict__ part_prob, int nblk, int M,
+                                      int N, int G, int k, int32_t* __restrict__ counts,
+                                      float* __restrict__ mean_prob,
+                                      int32_t* __restrict__ offsets, float* __restrict__ aux_out);
+
 // Launchers implemented in the .cu files. Each returns the number of kernels launched
 // (>= 0) or -1 if a launch failed.
 int launch_simt_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,

@@ -23,7 +23,7 @@ TENSORS = {"K": 0, "V": 1, "Q": 2, "Z": 3, "PSEL": 4, "W": 5, "LOGITS": 6}
 EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
-            "gqe_stage_name")
+            "gqe_stage_name", "gqe_route_static")
 GQE_NUM_STAGES = 8
 
 
@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
     lib.gqe_set_stage_events.restype = I
     lib.gqe_stage_name.argtypes = [I]
     lib.gqe_stage_name.restype = ctypes.c_char_p
+    lib.gqe_route_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P]
+    lib.gqe_route_static.restype = I
     return lib
 
 
@@ -129,6 +131,14 @@ def gqe_destroy(h) -> None:
 
 def gqe_kernel_launches(h) -> int:
     return int(lib.gqe_kernel_launches(h))
+
+
+def gqe_route_static(logits, M, N, G, k, sel, gates, counts, mean_prob, aux_loss=None,
+                     stream=None) -> None:
+    """Routing from precomputed logits with no device allocation (see include/gqe.h)."""
+    _check(lib.gqe_route_static(_ptr(logits), M, N, G, k, _ptr(sel), _ptr(gates), _ptr(counts),
+                                _ptr(mean_prob), _ptr(aux_loss), _stream(stream)),
+           "gqe_route_static")
 
 
 def gqe_stage_name(i: int):
