@@ -62,6 +62,8 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.mean_prob = (float*)take((size_t)N * 4);
   w.offsets = (int32_t*)take((size_t)(N + 1) * 4);
   w.bucket = (int32_t*)take((size_t)M * Gk * 4);
+  w.tile_list = (int2*)take((size_t)((M * Gk + 127) / 128 + N + 1) * sizeof(int2));
+  w.tile_count = (int32_t*)take(16);
   w.status = (int32_t*)take(16);
   w.wcat = take((size_t)(N + (2 * G + 1) * d_h) * dim * esz);
   (void)dim;
@@ -211,13 +213,18 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   };
   // mark() records stage event 0; each add() records the next event after its stage's
   // launches (the arguments are evaluated first), so event i precedes stage i.
-  bool ok = mark() && add(launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
+  // bf16: tensor-core (tcgen05) kernels for the projections; fp32: CUDA-core kernels.
+  const bool tc = h->dtype == GQE_BF16;
+  bool ok = mark() &&
+            add(tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)
+                   : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
             add(launch_route_select(h, M, st)) &&
             add(launch_route_scan_aux(h, M, aux_loss, st)) && add(launch_bucket(h, M, st)) &&
-            add(launch_simt_qproj(h, x, M, W_q, st)) &&
+            add(tc ? launch_tc_qproj(h, x, M, W_q, st) : launch_simt_qproj(h, x, M, W_q, st)) &&
             add(launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&
             add(launch_combine(h, M, variant, Do, st)) &&
-            add(launch_simt_oproj(h, M, Do, W_o, out, st));
+            add(tc ? launch_tc_oproj(h, M, Do, W_o, out, st)
+                   : launch_simt_oproj(h, M, Do, W_o, out, st));
   h->last_M = M;
   h->last_S = S;
   h->last_Do = Do;

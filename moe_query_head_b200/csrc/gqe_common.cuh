@@ -61,6 +61,8 @@ struct Workspace {
   float* mean_prob = nullptr;      // [N]
   int32_t* offsets = nullptr;      // [N + 1] bucket start of each expert
   int32_t* bucket = nullptr;       // [M * G * k] entries (token << 3) | rank, per expert
+  int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
+  int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* status = nullptr;       // device status word
   void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
   void* base = nullptr;            // the single allocation
@@ -112,5 +114,10 @@ int launch_simt_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int v
                           int causal, int Do, cudaStream_t st);
 int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st);
 int launch_simt_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
+// tcgen05 paths (bf16)
+int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
+                         const void* W_v, const void* W_shared, cudaStream_t st);
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);
+int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 
 }  // namespace gqe

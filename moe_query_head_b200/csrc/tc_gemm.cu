@@ -1,0 +1,531 @@
+// Tensor-core (tcgen05) GEMMs of the GQE forward pass, bf16 in, fp32 accumulation in TMEM:
+//
+//   dense projection  x [M, dim] times W_r, W_k, W_v, W_shared ([out, dim] each): router
+//                     logits (fp32), K [G, M, d_h], V stored transposed [G, d_h, M], and the
+//                     shared head's queries. KV heads are dense and routing-independent
+//                     ("GQE: Grouped Query Experts" README, Algorithm Overview).
+//   routed Q          for each expert e, the rows of x in e's bucket times W_q[e]; row i
+//                     lands in query stream g*k + r at its token position, so only the
+//                     selected (token, expert) pairs are projected (README, Algorithm
+//                     Overview: only the active query-head computation is reduced).
+//   output projection Z [M, D_o] times W_o [dim, D_o].
+//
+// One persistent kernel, one CTA per SM, 6 warps:
+//   warp 0     producer: TMA tile loads of A (or, for the routed projection, cp.async
+//              gathers of A rows written in the 128-byte swizzled layout) and of B;
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma (128 x BN x 16) and commits;
+//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator, conversion, stores.
+// Shared-memory stages are guarded by full/empty mbarriers; two TMEM accumulators let the
+// epilogue of one tile overlap the MMAs of the next.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gqe_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace gqe {
+
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;        // tile rows = MMA M = TMEM lanes
+constexpr int BN = 128;        // widest tile (MMA N)
+constexpr int BK = 64;         // one 128-byte swizzle atom of bf16 along K
+constexpr int STAGES = 6;
+constexpr int GATHER_LAG = 3;  // cp.async stages in flight before their barrier arrival
+constexpr int THREADS = 192;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int B_STAGE_BYTES = BN * BK * 2;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int MAX_PROBLEMS = 4;
+
+struct Problem {
+  int N;        // output columns of this problem
+  int n_tiles;  // ceil(N / BN)
+  int box_n;    // rows of B per TMA box (<= BN, multiple of 16)
+  OutMap out;
+};
+
+struct Params {
+  CUtensorMap tmap_a;                   // A [M, K] (unused when gathering)
+  CUtensorMap tmap_b[MAX_PROBLEMS];     // B [N_p, K] per problem
+  Problem prob[MAX_PROBLEMS];
+  int nprob;
+  int M, K;
+  int m_tiles;
+  int tiles_per_m;                      // sum of n_tiles over problems
+  int total_tiles;                      // dense: m_tiles * tiles_per_m
+  // routed projection (gather mode)
+  const __nv_bfloat16* x;               // A rows gathered from x [M, K]
+  const int32_t* bucket;                // entries (t << 3) | r
+  const int2* tile_list;                // (expert, first bucket slot) per tile
+  const int32_t* tile_count;            // number of tiles (device)
+  const int32_t* offsets;               // bucket offsets [N + 1]
+  __nv_bfloat16* Q;                     // query streams [S, M, d_h]
+  int E, k, d_h;
+  int32_t* status;
+  int64_t spin;
+};
+
+struct TileInfo {
+  int p;       // problem (dense) or expert (gather)
+  int m0;      // first row: token row (dense) or bucket slot (gather)
+  int rows;    // valid rows in the tile
+  int n0;      // first column within the problem
+  int n;       // MMA N (multiple of 16)
+};
+
+template <bool GATHER>
+__device__ __forceinline__ TileInfo tile_info(const Params& P, int tile) {
+  TileInfo ti;
+  if constexpr (GATHER) {
+    const int2 t = P.tile_list[tile];
+    ti.p = t.x;
+    ti.m0 = t.y;
+    const int end = P.offsets[t.x + 1];
+    ti.rows = min(BM, end - t.y);
+    ti.n0 = 0;
+    ti.n = P.prob[0].box_n;
+  } else {
+    const int mt = tile / P.tiles_per_m;
+    int r = tile % P.tiles_per_m;
+    int p = 0;
+    while (r >= P.prob[p].n_tiles) {
+      r -= P.prob[p].n_tiles;
+      ++p;
+    }
+    ti.p = p;
+    ti.m0 = mt * BM;
+    ti.rows = min(BM, P.M - ti.m0);
+    ti.n0 = r * BN;
+    const int rem = P.prob[p].N - ti.n0;
+    ti.n = min(BN, (rem + 15) / 16 * 16);
+  }
+  return ti;
+}
+
+__device__ __forceinline__ void set_timeout(const Params& P, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicExch(P.status, kStatusTimeout);
+}
+
+template <bool GATHER>
+__global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_constant__ Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int total = GATHER ? *P.tile_count : P.total_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], GATHER ? 33 : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!GATHER) prefetch_tmap(&P.tmap_a);
+    for (int p = 0; p < P.nprob; ++p) prefetch_tmap(&P.tmap_b[p]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int KB = (P.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;  // stages issued whose gather arrival is still pending (GATHER)
+    int pend_stage[GATHER_LAG + 1];
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      const TileInfo ti = tile_info<GATHER>(P, tile);
+      const int brow = GATHER ? ti.p * P.d_h : ti.n0;
+      const int tb = GATHER ? 0 : ti.p;
+      const uint32_t b_bytes = (uint32_t)P.prob[GATHER ? 0 : ti.p].box_n * BK * 2;
+      // gather mode: this lane's four rows of the tile and their source tokens
+      int64_t src_row[4];
+      if constexpr (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          src_row[i] = r < ti.rows ? (int64_t)(P.bucket[ti.m0 + r] >> 3) : -1;
+        }
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) {
+          if (lane == 0) set_timeout(P, abort_flag);
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], (GATHER ? 0u : (uint32_t)A_STAGE_BYTES) + b_bytes);
+          if (!GATHER) tma_load_2d(sA + stage * A_STAGE_BYTES, &P.tmap_a, kb * BK, ti.m0, &full[stage]);
+          tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[tb], kb * BK, brow, &full[stage]);
+        }
+        if constexpr (GATHER) {
+          const uint32_t base = smem_u32(sA + stage * A_STAGE_BYTES);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = lane + 32 * i;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int kcol = kb * BK + c * 8;
+              const bool ok_src = src_row[i] >= 0 && kcol < P.K;
+              const void* src = ok_src ? (const void*)(P.x + src_row[i] * P.K + kcol)
+                                       : (const void*)P.x;
+              const uint32_t dst = base + r * 128 + ((c ^ (r & 7)) << 4);
+              cp_async_16(dst, src, ok_src ? 16u : 0u);
+            }
+          }
+          cp_async_commit();
+          pend_stage[issued] = stage;
+          ++issued;
+          if (issued > GATHER_LAG) {
+            cp_async_wait<GATHER_LAG>();
+            fence_async_shared();
+            mbar_arrive(&full[pend_stage[0]]);
+#pragma unroll
+            for (int i = 0; i < GATHER_LAG; ++i) pend_stage[i] = pend_stage[i + 1];
+            --issued;
+          }
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if constexpr (GATHER) {
+      cp_async_wait<0>();
+      fence_async_shared();
+      for (int i = 0; i < issued; ++i) mbar_arrive(&full[pend_stage[i]]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
+      const TileInfo ti = tile_info<GATHER>(P, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1, P.spin);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        if (lane == 0) set_timeout(P, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      const uint32_t idesc = idesc_bf16_f32(BM, ti.n);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (lane == 0) ok = mbar_wait(&full[stage], phase, P.spin);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) {
+          if (lane == 0) set_timeout(P, abort_flag);
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc(a_addr + kk * 32, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(b_addr + kk * 32, 1024, kSwizzle128B);
+            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);  // frees the stage when these MMAs finish
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&acc_full[acc]);
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
+    const int row = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
+      const TileInfo ti = tile_info<GATHER>(P, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, P.spin);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        if (lane == 0) set_timeout(P, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const bool valid = row < ti.rows;
+      if constexpr (GATHER) {
+        __nv_bfloat16* dst = nullptr;
+        if (valid) {
+          const int ent = P.bucket[ti.m0 + row];
+          const int g = ti.p / P.E;
+          const int64_t s = (int64_t)g * P.k + (ent & 7);
+          dst = P.Q + (s * P.M + (ent >> 3)) * P.d_h;
+        }
+        for (int c0 = 0; c0 < ti.n; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(t_row + c0, r);
+          tmem_wait_ld();
+          if (valid && c0 < P.d_h) {
+            uint4 v0, v1;
+            v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
+            v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
+            v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
+            v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
+            v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
+            v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
+            v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
+            v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
+            *reinterpret_cast<uint4*>(dst + c0) = v0;
+            *reinterpret_cast<uint4*>(dst + c0 + 8) = v1;
+          }
+        }
+      } else {
+        const Problem& pr = P.prob[ti.p];
+        const OutMap& o = pr.out;
+        const int64_t m = ti.m0 + row;
+        for (int c0 = 0; c0 < ti.n; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(t_row + c0, r);
+          tmem_wait_ld();
+          if (!valid) continue;
+#pragma unroll
+          for (int g8 = 0; g8 < 2; ++g8) {
+            const int c = ti.n0 + c0 + g8 * 8;  // column within the problem
+            if (c >= pr.N) continue;
+            const int head = c / o.head_w, col = c % o.head_w;
+            const int64_t idx = head * o.head_stride + m * o.row_stride + (int64_t)col * o.col_stride;
+            const uint32_t* rv = r + g8 * 8;
+            if (o.f32) {
+              float* d = static_cast<float*>(o.base) + idx;
+              if (o.col_stride == 1 && c + 8 <= pr.N && ((reinterpret_cast<uintptr_t>(d) & 15) == 0)) {
+                *reinterpret_cast<uint4*>(d) = make_uint4(rv[0], rv[1], rv[2], rv[3]);
+                *reinterpret_cast<uint4*>(d + 4) = make_uint4(rv[4], rv[5], rv[6], rv[7]);
+              } else {
+                for (int j = 0; j < 8 && c + j < pr.N; ++j)
+                  d[(int64_t)j * o.col_stride] = __uint_as_float(rv[j]);
+              }
+            } else {
+              __nv_bfloat16* d = static_cast<__nv_bfloat16*>(o.base) + idx;
+              if (o.col_stride == 1 && c + 8 <= pr.N && ((reinterpret_cast<uintptr_t>(d) & 15) == 0)) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(rv[0]), __uint_as_float(rv[1]));
+                v.y = pack_bf16x2(__uint_as_float(rv[2]), __uint_as_float(rv[3]));
+                v.z = pack_bf16x2(__uint_as_float(rv[4]), __uint_as_float(rv[5]));
+                v.w = pack_bf16x2(__uint_as_float(rv[6]), __uint_as_float(rv[7]));
+                *reinterpret_cast<uint4*>(d) = v;
+              } else {
+                for (int j = 0; j < 8 && c + j < pr.N; ++j)
+                  d[(int64_t)j * o.col_stride] = __float2bfloat16_rn(__uint_as_float(rv[j]));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Tiles of the routed projection: each expert's bucket cut into runs of BM slots.
+__global__ void qproj_tiles_kernel(const int32_t* __restrict__ offsets, int N,
+                                   int2* __restrict__ tile_list, int32_t* __restrict__ tile_count) {
+  if (threadIdx.x != 0) return;
+  int n = 0;
+  for (int e = 0; e < N; ++e)
+    for (int s = offsets[e]; s < offsets[e + 1]; s += BM) tile_list[n++] = make_int2(e, s);
+  *tile_count = n;
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    cudaGetLastError();
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor map: `cols` contiguous elements per row, `rows` rows `ld` elements apart;
+// box of box_cols x box_rows with 128-byte swizzle (box_cols * 2 must be <= 128).
+bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t ld,
+                  uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  if (!encoder()) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATHER>
+int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
+  static bool configured[2] = {false, false};
+  if (!configured[GATHER]) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return -1;
+    configured[GATHER] = true;
+  }
+  tc_gemm_kernel<GATHER><<<grid, THREADS, SMEM_BYTES, st>>>(P);
+  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+}
+
+Problem make_problem(int N, OutMap out) {
+  Problem p;
+  p.N = N;
+  p.n_tiles = (N + BN - 1) / BN;
+  p.box_n = N >= BN ? BN : (N + 15) / 16 * 16;
+  p.out = out;
+  return p;
+}
+
+int64_t spin_limit(const gqe_ctx* h) { return h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22; }
+
+}  // namespace
+
+int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
+                         const void* W_v, const void* W_shared, cudaStream_t st) {
+  const int d_h = h->d_h, G = h->G, dim = h->dim;
+  const int S = G * h->k + (W_shared ? 1 : 0);
+  Params P;
+  memset(&P, 0, sizeof(P));
+  if (!tmap_bf16_2d(&P.tmap_a, x, dim, M, dim, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B)) return -1;
+  const void* Bs[4] = {W_r, W_k, W_v, W_shared};
+  const int Ns[4] = {h->N, G * d_h, G * d_h, d_h};
+  OutMap outs[4] = {
+      OutMap{h->ws.logits, 0, h->N, 1, 1 << 30, 1},
+      OutMap{h->ws.K, (int64_t)M * d_h, d_h, 1, d_h, 0},
+      OutMap{h->ws.Vt, (int64_t)d_h * M, 1, M, d_h, 0},
+      OutMap{static_cast<char*>(h->ws.Q) + (int64_t)(S - 1) * M * d_h * 2, 0, d_h, 1, d_h, 0}};
+  int np = 0;
+  for (int i = 0; i < 4; ++i) {
+    if (!Bs[i]) continue;
+    P.prob[np] = make_problem(Ns[i], outs[i]);
+    if (!tmap_bf16_2d(&P.tmap_b[np], Bs[i], dim, Ns[i], dim, BK, P.prob[np].box_n,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return -1;
+    ++np;
+  }
+  P.nprob = np;
+  P.M = M;
+  P.K = dim;
+  P.m_tiles = (M + BM - 1) / BM;
+  P.tiles_per_m = 0;
+  for (int i = 0; i < np; ++i) P.tiles_per_m += P.prob[i].n_tiles;
+  P.total_tiles = P.m_tiles * P.tiles_per_m;
+  P.status = h->ws.status;
+  P.spin = spin_limit(h);
+  const int grid = P.total_tiles < h->num_sms ? P.total_tiles : h->num_sms;
+  return launch<false>(h, P, grid, st);
+}
+
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st) {
+  qproj_tiles_kernel<<<1, 32, 0, st>>>(h->ws.offsets, h->N, h->ws.tile_list, h->ws.tile_count);
+  if (cudaGetLastError() != cudaSuccess) return -1;
+  Params P;
+  memset(&P, 0, sizeof(P));
+  P.prob[0] = make_problem(h->d_h, OutMap{});
+  if (!tmap_bf16_2d(&P.tmap_b[0], W_q, h->dim, (uint64_t)h->N * h->d_h, h->dim, BK,
+                    P.prob[0].box_n, CU_TENSOR_MAP_SWIZZLE_128B))
+    return -1;
+  P.nprob = 1;
+  P.M = M;
+  P.K = h->dim;
+  P.x = static_cast<const __nv_bfloat16*>(x);
+  P.bucket = h->ws.bucket;
+  P.tile_list = h->ws.tile_list;
+  P.tile_count = h->ws.tile_count;
+  P.offsets = h->ws.offsets;
+  P.Q = static_cast<__nv_bfloat16*>(h->ws.Q);
+  P.E = h->E;
+  P.k = h->k;
+  P.d_h = h->d_h;
+  P.status = h->ws.status;
+  P.spin = spin_limit(h);
+  const int max_tiles = (int)(((int64_t)M * h->G * h->k + BM - 1) / BM) + h->N;
+  const int grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
+  return launch<true>(h, P, grid, st) < 0 ? -1 : 2;
+}
+
+int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st) {
+  Params P;
+  memset(&P, 0, sizeof(P));
+  if (!tmap_bf16_2d(&P.tmap_a, h->ws.Z, Do, M, Do, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B)) return -1;
+  P.prob[0] = make_problem(h->dim, OutMap{out, 0, h->dim, 1, 1 << 30, 0});
+  if (!tmap_bf16_2d(&P.tmap_b[0], W_o, Do, h->dim, Do, BK, P.prob[0].box_n,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return -1;
+  P.nprob = 1;
+  P.M = M;
+  P.K = Do;
+  P.m_tiles = (M + BM - 1) / BM;
+  P.tiles_per_m = P.prob[0].n_tiles;
+  P.total_tiles = P.m_tiles * P.tiles_per_m;
+  P.status = h->ws.status;
+  P.spin = spin_limit(h);
+  const int grid = P.total_tiles < h->num_sms ? P.total_tiles : h->num_sms;
+  return launch<false>(h, P, grid, st);
+}
+
+}  // namespace gqe
