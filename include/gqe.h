@@ -53,7 +53,7 @@ typedef enum { GQE_BF16 = 0, GQE_F32 = 1 } gqe_dtype;
 /* Internal tensors that gqe_get_tensor can copy out (for tests and inspection). */
 typedef enum {
     GQE_T_K = 0,      /* [G, M, d_h]       keys, dtype                                      */
-    GQE_T_V = 1,      /* [G, d_h, M]       values, stored transposed (token index fastest)  */
+    GQE_T_V = 1,      /* [G, M, d_h]       values, dtype                                    */
     GQE_T_Q = 2,      /* [S, M, d_h]       query streams (routed g*k+r, then shared), dtype */
     GQE_T_Z = 3,      /* [M, D_o]          concatenated attention output, dtype             */
     GQE_T_PSEL = 4,   /* [M, G, k] float   router softmax p of each selected expert         */

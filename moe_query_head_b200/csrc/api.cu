@@ -48,7 +48,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   const int64_t nblk = (M + kRouteBlock - 1) / kRouteBlock;
   const int64_t Gk = (int64_t)G * k;
   w.K = take((size_t)G * M * d_h * esz);
-  w.Vt = take((size_t)G * M * d_h * esz);
+  w.V = take((size_t)G * M * d_h * esz);
   w.Q = take((size_t)S * M * d_h * esz);
   w.Z = take((size_t)M * Do * esz);
   w.logits = (float*)take((size_t)M * N * 4);
@@ -221,7 +221,8 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
             add(launch_route_select(h, M, st)) &&
             add(launch_route_scan_aux(h, M, aux_loss, st)) && add(launch_bucket(h, M, st)) &&
             add(tc ? launch_tc_qproj(h, x, M, W_q, st) : launch_simt_qproj(h, x, M, W_q, st)) &&
-            add(launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&
+            add(tc ? launch_tc_attention(h, B, T, S, has_shared, variant, causal, Do, st)
+                   : launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&
             add(launch_combine(h, M, variant, Do, st)) &&
             add(tc ? launch_tc_oproj(h, M, Do, W_o, out, st)
                    : launch_simt_oproj(h, M, Do, W_o, out, st));
@@ -257,7 +258,7 @@ gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void
   size_t n = 0;
   switch (which) {
     case GQE_T_K: src = h->ws.K; n = (size_t)h->G * M * h->d_h * h->esz; break;
-    case GQE_T_V: src = h->ws.Vt; n = (size_t)h->G * M * h->d_h * h->esz; break;
+    case GQE_T_V: src = h->ws.V; n = (size_t)h->G * M * h->d_h * h->esz; break;
     case GQE_T_Q: src = h->ws.Q; n = (size_t)h->last_S * M * h->d_h * h->esz; break;
     case GQE_T_Z: src = h->ws.Z; n = M * h->last_Do * h->esz; break;
     case GQE_T_PSEL: src = h->ws.psel; n = M * h->G * h->k * 4; break;

@@ -47,7 +47,7 @@ struct OutMap {
 // ---------------------------------------------------------------------------------------
 struct Workspace {
   void* K = nullptr;        // [G, M, d_h]
-  void* Vt = nullptr;       // [G, d_h, M]
+  void* V = nullptr;        // [G, M, d_h]
   void* Q = nullptr;        // [S, M, d_h]
   void* Z = nullptr;        // [M, D_o]
   float* logits = nullptr;  // [M, N]
@@ -119,5 +119,7 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
                          const void* W_v, const void* W_shared, cudaStream_t st);
 int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
+int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,
+                        int causal, int Do, cudaStream_t st);
 
 }  // namespace gqe

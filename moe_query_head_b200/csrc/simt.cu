@@ -156,7 +156,7 @@ constexpr int ATT_ROWS = 32, ATT_KEYS = 32;
 
 template <typename T, int DH>
 __global__ void __launch_bounds__(128)
-attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __restrict__ Vt,
+attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __restrict__ Vc,
                  T* __restrict__ Z, const float* __restrict__ psel, int M, int Tlen, int G,
                  int k, int Do, int shared_col, int weighted, int causal, float scale_log2) {
   constexpr int PD = DH / 4;
@@ -179,14 +179,13 @@ attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __r
   const int row0 = blockIdx.x * ATT_ROWS;
   const int kv_end = causal ? min(Tlen, row0 + ATT_ROWS) : Tlen;
   const T* Kh = Kc + (int64_t)kvh * M * DH + (int64_t)b * Tlen * DH;
-  const T* Vh = Vt + (int64_t)kvh * DH * M + (int64_t)b * Tlen;
+  const T* Vh = Vc + (int64_t)kvh * M * DH + (int64_t)b * Tlen * DH;
   for (int u0 = 0; u0 < kv_end; u0 += ATT_KEYS) {
     __syncthreads();
     for (int i = threadIdx.x; i < ATT_KEYS * DH; i += 128) {
       const int kr = i / DH, kc = i % DH;
       Ks[kr][kc] = (u0 + kr < Tlen) ? to_f32(Kh[(int64_t)(u0 + kr) * DH + kc]) : 0.f;
-      const int vc = i / ATT_KEYS, vr = i % ATT_KEYS;  // token index fastest in Vt
-      Vs[vr][vc] = (u0 + vr < Tlen) ? to_f32(Vh[(int64_t)vc * M + u0 + vr]) : 0.f;
+      Vs[kr][kc] = (u0 + kr < Tlen) ? to_f32(Vh[(int64_t)(u0 + kr) * DH + kc]) : 0.f;
     }
     __syncthreads();
     float sc[ATT_KEYS];
@@ -252,7 +251,7 @@ int dense_proj_t(gqe_ctx* h, const void* x, int M, const void* W_r, const void* 
   int n = 0;
   a.p[n++] = DenseProblem{W_r, h->N, OutMap{h->ws.logits, 0, h->N, 1, 1 << 30, 1}};
   a.p[n++] = DenseProblem{W_k, G * d_h, OutMap{h->ws.K, (int64_t)M * d_h, d_h, 1, d_h, 0}};
-  a.p[n++] = DenseProblem{W_v, G * d_h, OutMap{h->ws.Vt, (int64_t)d_h * M, 1, M, d_h, 0}};
+  a.p[n++] = DenseProblem{W_v, G * d_h, OutMap{h->ws.V, (int64_t)M * d_h, d_h, 1, d_h, 0}};
   if (W_shared) {
     void* qs = static_cast<char*>(h->ws.Q) + (int64_t)(S - 1) * M * d_h * h->esz;
     a.p[n++] = DenseProblem{W_shared, d_h, OutMap{qs, 0, d_h, 1, d_h, 0}};
@@ -273,7 +272,7 @@ void attention_launch(gqe_ctx* h, int B, int T_, int S, int shared_col, int weig
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   attention_kernel<T, DH><<<grid, 128, 0, st>>>(
       static_cast<const T*>(h->ws.Q), static_cast<const T*>(h->ws.K),
-      static_cast<const T*>(h->ws.Vt), static_cast<T*>(h->ws.Z), h->ws.psel, M, T_, h->G,
+      static_cast<const T*>(h->ws.V), static_cast<T*>(h->ws.Z), h->ws.psel, M, T_, h->G,
       h->k, Do, shared_col, weighted, causal, scale_log2);
 }
 

@@ -1,7 +1,7 @@
 // Tensor-core (tcgen05) GEMMs of the GQE forward pass, bf16 in, fp32 accumulation in TMEM:
 //
 //   dense projection  x [M, dim] times W_r, W_k, W_v, W_shared ([out, dim] each): router
-//                     logits (fp32), K [G, M, d_h], V stored transposed [G, d_h, M], and the
+//                     logits (fp32), K and V [G, M, d_h], and the
 //                     shared head's queries. KV heads are dense and routing-independent
 //                     ("GQE: Grouped Query Experts" README, Algorithm Overview).
 //   routed Q          for each expert e, the rows of x in e's bucket times W_q[e]; row i
@@ -444,6 +444,12 @@ int64_t spin_limit(const gqe_ctx* h) { return h->spin_limit > 0 ? h->spin_limit 
 
 }  // namespace
 
+bool tmap_bf16_2d_ext(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                      uint64_t ld, uint32_t box_cols, uint32_t box_rows,
+                      CUtensorMapSwizzle sw) {
+  return tmap_bf16_2d(m, ptr, cols, rows, ld, box_cols, box_rows, sw);
+}
+
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
                          const void* W_v, const void* W_shared, cudaStream_t st) {
   const int d_h = h->d_h, G = h->G, dim = h->dim;
@@ -456,7 +462,7 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   OutMap outs[4] = {
       OutMap{h->ws.logits, 0, h->N, 1, 1 << 30, 1},
       OutMap{h->ws.K, (int64_t)M * d_h, d_h, 1, d_h, 0},
-      OutMap{h->ws.Vt, (int64_t)d_h * M, 1, M, d_h, 0},
+      OutMap{h->ws.V, (int64_t)M * d_h, d_h, 1, d_h, 0},
       OutMap{static_cast<char*>(h->ws.Q) + (int64_t)(S - 1) * M * d_h * 2, 0, d_h, 1, d_h, 0}};
   int np = 0;
   for (int i = 0; i < 4; ++i) {

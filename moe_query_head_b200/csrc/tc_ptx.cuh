@@ -205,6 +205,20 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t sbo_bytes
   return d;
 }
 
+// MN-major operand: rows along K, each row holding (swizzle width) bytes of consecutive
+// MN elements. The MN extent is split into atoms `lbo_bytes` apart; 8-row groups along K
+// are `sbo_bytes` apart.
+__device__ __forceinline__ uint64_t smem_desc_mn(uint32_t saddr, uint32_t lbo_bytes,
+                                                 uint32_t sbo_bytes, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 accumulator, both
 // operands K-major, M = 128, N = n (multiple of 16, <= 256).
 __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int m, int n) {

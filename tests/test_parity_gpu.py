@@ -42,11 +42,11 @@ def test_tiny_f32_full_and_intermediates():
     run, ref, r, _ = _full_check(inp)
     tdt = torch.float32
     K = to_host_f64(run.tensor("K", (wl.G, wl.M, wl.d_h), tdt))
-    Vt = to_host_f64(run.tensor("V", (wl.G, wl.d_h, wl.M), tdt))
+    V = to_host_f64(run.tensor("V", (wl.G, wl.M, wl.d_h), tdt))
     Q = to_host_f64(run.tensor("Q", (wl.n_streams, wl.M, wl.d_h), tdt))
     Z = to_host_f64(run.tensor("Z", (wl.M, wl.D_o), tdt))
     assert rel_l2(K, ref.K) <= 1e-6
-    assert rel_l2(Vt, ref.V.transpose(0, 2, 1)) <= 1e-6
+    assert rel_l2(V, ref.V) <= 1e-6
     assert rel_l2(Q, ref.Q) <= 1e-6
     assert rel_l2(Z, ref.Z) <= 1e-5
     run.close()
@@ -116,14 +116,14 @@ def test_deterministic_and_kv_independent_of_routing():
     a.forward()
     assert torch.equal(y1, a.out), "two runs differ"
     K1 = a.tensor("K", (8, 333, 64), torch.bfloat16)
-    V1 = a.tensor("V", (8, 64, 333), torch.bfloat16)
+    V1 = a.tensor("V", (8, 333, 64), torch.bfloat16)
     for kw in (dict(variant="hard_concat"), dict(k=4)):
         # identical x and weights; only W_o takes the width of the other concatenation
         wl2 = base.with_(**kw)
         W_o = W.generate(wl2).W_o
         b = GpuRun(dataclasses.replace(inp, wl=wl2, W_o=W_o)).forward()
         assert torch.equal(K1, b.tensor("K", (8, 333, 64), torch.bfloat16))
-        assert torch.equal(V1, b.tensor("V", (8, 64, 333), torch.bfloat16))
+        assert torch.equal(V1, b.tensor("V", (8, 333, 64), torch.bfloat16))
         b.close()
     a.close()
 
