@@ -6,18 +6,21 @@
 // Every stream has one query per token, so the work is a grouped-query attention with
 // S = G*k + 1 query heads over G KV heads; the savings of GQE come from S < N + 1.
 //
-// Work item = (sequence b, stream s, 128-query tile); a persistent CTA per SM takes items
-// heaviest first (causal tiles near the end of the sequence have the most keys).
-//   warp 0     TMA: the Q tile once per item, then K and V tiles into a ring of stages;
-//   warp 1     TMEM owner; one lane issues S = Q K^T (A and B from shared memory) into
-//              one of two TMEM S buffers, then O += P V with P read from TMEM (the TS form)
-//              and V as an MN-major shared-memory operand;
-//   warps 2-5  softmax: one query row per thread, 128 scores per KV tile in registers,
-//              exp2 with the running row maximum, P written back over S as bf16 pairs.
-//              O is rescaled in TMEM only when a row maximum grows by more than 2^8
-//              (rare after the first tiles), so the common path never waits on P V. At
-//              the end of an item the same warps normalise O by the row sum, apply the
-//              weighted_concat scale if any, and store the row into its block of Z.
+// Work item = (sequence b, stream s, two consecutive 128-query tiles); a persistent CTA per
+// SM takes items heaviest first (causal tiles near the end of a sequence have the most
+// keys). The two query tiles share every K/V tile and are handled by two softmax
+// warpgroups that ping-pong: while one computes exponentials, the tensor core runs the
+// other's products, and each hides the other's waits.
+//   warp 0      TMA: both Q tiles once per item, then K and V tiles into a ring of stages;
+//   warp 1      TMEM owner; one lane issues, per query tile w, S_w = Q_w K^T (A and B from
+//               shared memory) into TMEM, and O_w += P_w V with P_w read from TMEM (the TS
+//               form) and V as an MN-major shared-memory operand;
+//   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: one query row per
+//               thread, 128 scores per KV tile in registers, exp2 against the running row
+//               maximum, P written back over S as bf16 pairs. O is rescaled in TMEM only
+//               when a row maximum grows by more than 2^8 (rare after the first tiles).
+//               At the end of an item the same warps normalise O by the row sum, apply the
+//               weighted_concat scale if any, and store the row into its block of Z.
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
@@ -33,9 +36,10 @@ namespace {
 
 using namespace tc;
 
-constexpr int THREADS = 192;
-constexpr int TQ = 128;   // queries per tile (MMA M, TMEM lanes)
-constexpr int TK = 128;   // keys per tile (S MMA N)
+constexpr int NWG = 2;                 // query tiles per item = softmax warpgroups
+constexpr int THREADS = 64 + NWG * 128;
+constexpr int TQ = 128;                // queries per tile (MMA M, TMEM lanes)
+constexpr int TK = 128;                // keys per tile (S MMA N)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int DH>
@@ -48,7 +52,14 @@ struct Cfg {
   static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;
   static constexpr int TILE_BYTES = 128 * DH * 2;   // one Q, K or V tile
   static constexpr int STAGES = DH <= 64 ? 4 : (DH <= 96 ? 3 : 2);
-  static constexpr int SMEM = TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
+  static constexpr int SMEM = NWG * TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
+  // TMEM columns (512): S_w at 128 w. For DH <= 64, P_w has columns of its own
+  // (256 + 64 w) and O_w sits at 384 + DH w, so S_w(j+1) can be computed while P_w(j) V
+  // is still being read. For larger DH, P_w overlays the first half of S_w and O_w sits at
+  // 256 + DH w; S_w(j+1) then waits for that product.
+  static constexpr bool SEP_P = DH <= 64;
+  static constexpr int O_COL = SEP_P ? 384 : 256;
+  __device__ static constexpr int p_col(int w) { return SEP_P ? 256 + 64 * w : 128 * w; }
 };
 
 struct Params {
@@ -56,7 +67,7 @@ struct Params {
   __nv_bfloat16* Z;
   const float* psel;
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
-  int nq, items;
+  int nq, npairs, items;
   float scale_log2;
   int32_t* status;
   int64_t spin;
@@ -69,27 +80,29 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 struct Item {
-  int b, s, qt;
+  int b, s, pair;
+  int nkv[NWG];  // KV tiles of each query tile (0: the tile is past the sequence end)
 };
 __device__ __forceinline__ Item decode(const Params& P, int i) {
   Item it;
   const int bs = P.B * P.S;
-  it.qt = P.causal ? P.nq - 1 - i / bs : i / bs;
+  it.pair = P.causal ? P.npairs - 1 - i / bs : i / bs;
   const int r = i % bs;
   it.s = r % P.S;
   it.b = r / P.S;
+#pragma unroll
+  for (int w = 0; w < NWG; ++w) {
+    const int qt = it.pair * NWG + w;
+    it.nkv[w] = qt >= P.nq ? 0 : (P.causal ? qt + 1 : P.nq);
+  }
   return it;
 }
-__device__ __forceinline__ int kv_tiles(const Params& P, const Item& it) {
-  return P.causal ? it.qt + 1 : P.nq;
-}
 
-// Waits (lane 0 polls, the warp follows); on giving up flags the timeout.
+// Waits with every lane polling (no divergence); the outcome is made warp-uniform. On
+// giving up, flags the timeout.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& P,
                                           volatile int* abort_flag) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, P.spin);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  const bool ok = !__any_sync(0xffffffffu, !mbar_wait(bar, parity, P.spin));
   if (!ok && (threadIdx.x & 31) == 0) {
     *abort_flag = 1;
     atomicExch(P.status, kStatusTimeout);
@@ -103,19 +116,19 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::TILE_BYTES;
+  uint8_t* sQ = smem;                              // NWG tiles
+  uint8_t* sKV = smem + NWG * C::TILE_BYTES;       // per stage: K tile, V tile
   uint64_t* bar = reinterpret_cast<uint64_t*>(sKV + C::STAGES * 2 * C::TILE_BYTES);
   uint64_t* q_full = bar;
   uint64_t* q_empty = bar + 1;
   uint64_t* kv_full = bar + 2;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* pv_done = p_ready + 2;
-  uint64_t* o_full = pv_done + 2;
-  uint64_t* o_free = o_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + 1);
+  uint64_t* s_full = kv_empty + C::STAGES;  // [NWG]
+  uint64_t* p_ready = s_full + NWG;         // [NWG]
+  uint64_t* pv_done = p_ready + NWG;        // [NWG]
+  uint64_t* o_full = pv_done + NWG;         // [NWG]
+  uint64_t* o_free = o_full + NWG;          // [NWG]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + NWG);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -126,13 +139,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_ready[b], 4);
-      mbar_init(&pv_done[b], 1);
+    for (int w = 0; w < NWG; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_ready[w], 4);
+      mbar_init(&pv_done[w], 1);
+      mbar_init(&o_full[w], 1);
+      mbar_init(&o_free[w], 4);
     }
-    mbar_init(o_full, 1);
-    mbar_init(o_free, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -148,8 +161,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_o = tmem + 256;
+  const uint32_t tmem = *tmem_holder;  // S_w at columns 128 w, O_w at 256 + DH w
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA loads
@@ -158,21 +170,28 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       uint32_t kv_phase = 0, q_phase = 0;
       for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
         const Item it = decode(P, i);
-        const int q0 = it.qt * TQ;
-        const int nkv = kv_tiles(P, it);
+        const int nk = max(it.nkv[0], it.nkv[1]);
         if (!mbar_wait(q_empty, q_phase ^ 1, P.spin)) {
           *abort_flag = 1;
           atomicExch(P.status, kStatusTimeout);
           break;
         }
         q_phase ^= 1;
-        mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-        const int qrow = it.s * P.M + it.b * P.T + q0;
+        int nq_tiles = 0;
 #pragma unroll
-        for (int c = 0; c < C::NC; ++c)
-          tma_load_2d(sQ + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow, q_full);
+        for (int w = 0; w < NWG; ++w) nq_tiles += it.nkv[w] > 0;
+        mbar_arrive_expect_tx(q_full, nq_tiles * C::TILE_BYTES);
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) {
+          if (it.nkv[w] == 0) continue;
+          const int qrow = it.s * P.M + it.b * P.T + (it.pair * NWG + w) * TQ;
+#pragma unroll
+          for (int c = 0; c < C::NC; ++c)
+            tma_load_2d(sQ + w * C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow,
+                        q_full);
+        }
         const int kvh = it.s < P.Sr ? it.s / P.k : 0;
-        for (int j = 0; j < nkv; ++j) {
+        for (int j = 0; j < nk; ++j) {
           if (!mbar_wait(&kv_empty[stage], kv_phase ^ 1, P.spin)) {
             *abort_flag = 1;
             atomicExch(P.status, kStatusTimeout);
@@ -196,125 +215,174 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
+    // This warp shares its sub-partition with two busy softmax warps, so it keeps its
+    // instruction count small: descriptors are built once, and each product's descriptor
+    // is a base plus a constant (the address field is the low 14 bits, in 16-byte units).
     const uint32_t idesc_s = idesc_bf16_f32(TQ, TK);
     const uint32_t idesc_pv = idesc_bf16_f32(TQ, DH) | (1u << 16);  // B (V) MN-major
-    const uint32_t q_addr = smem_u32(sQ);
+    const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t k_desc = smem_desc(smem_u32(sKV), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t v_desc =
+        smem_desc_mn(smem_u32(sKV + C::TILE_BYTES), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kStageStep = (2 * C::TILE_BYTES) >> 4;
+    constexpr uint32_t kTileStep = C::TILE_BYTES >> 4;
     int stage = 0;
     uint32_t kv_phase = 0, q_phase = 0;
-    uint32_t jt = 0;
-    int item_no = 0;
+    // per query tile: uses of s_full (= p_ready) / pv_done / o_full so far
+    uint32_t n_s[NWG] = {0, 0}, n_pv[NWG] = {0, 0}, n_o[NWG] = {0, 0};
     bool ok = true;
-    // O += P V for the KV tile held in `st`, whose S/P buffer is jt_ & 1.
-    auto issue_pv = [&](int st, uint32_t jt_, bool first) -> bool {
-      const int buf = jt_ & 1;
-      if (!warp_wait(&p_ready[buf], (jt_ >> 1) & 1, P, abort_flag)) return false;
-      if (first && item_no > 0 &&
-          !warp_wait(o_free, (item_no - 1) & 1, P, abort_flag))
-        return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t v_addr = smem_u32(sKV + st * 2 * C::TILE_BYTES + C::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < TK / 16; ++kk) {
-          // V as the MN-major B operand (N = head dim, K = keys): 16 keys are two 8-row
-          // groups (SBO apart) of every chunk; the chunks are the MN atoms (LBO apart).
-          const uint64_t vd = smem_desc_mn(v_addr + kk * 16 * C::ROW_BYTES, C::CHUNK_BYTES,
-                                           8 * C::ROW_BYTES, C::LAYOUT);
-          mma_ts(tmem_o, tmem + buf * 128 + kk * 8, vd, idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
-        }
-        mma_commit(&kv_empty[st]);
-        mma_commit(&pv_done[buf]);
-      }
-      __syncwarp();
-      return true;
-    };
+
+    // S_w = Q_w K^T for the K tile in stage `st` (lane 0 only).
+#define GQE_ISSUE_S(w, st)                                                                   \
+  do {                                                                                       \
+    const uint64_t qd = q_desc + (uint64_t)((w) * kTileStep);                                \
+    const uint64_t kd = k_desc + (uint64_t)((st) * kStageStep);                              \
+    _Pragma("unroll") for (int kk = 0; kk < DH / 16; ++kk) {                                 \
+      const uint32_t o = (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4; \
+      mma_ss(tmem + (w) * 128, qd + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);                   \
+    }                                                                                        \
+    mma_commit(&s_full[w]);                                                                  \
+  } while (0)
+    // O_w += P_w V for the V tile in stage `st` (lane 0 only). V is the MN-major B operand
+    // (N = head dim, K = keys): 16 keys are two 8-row groups of every chunk.
+#define GQE_ISSUE_PV(w, st, first)                                                           \
+  do {                                                                                       \
+    const uint64_t vd = v_desc + (uint64_t)((st) * kStageStep);                              \
+    _Pragma("unroll") for (int kk = 0; kk < TK / 16; ++kk)                                   \
+        mma_ts(tmem + C::O_COL + (w) * DH, tmem + C::p_col(w) + kk * 8,                      \
+               vd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_pv,                     \
+               ((first) && kk == 0) ? 0u : 1u);                                              \
+    mma_commit(&pv_done[w]);                                                                 \
+  } while (0)
+
     for (int i = blockIdx.x; i < P.items && ok && !*abort_flag; i += gridDim.x) {
       const Item it = decode(P, i);
-      const int nkv = kv_tiles(P, it);
+      const int nk = max(it.nkv[0], it.nkv[1]);
       if (!warp_wait(q_full, q_phase, P, abort_flag)) break;
       q_phase ^= 1;
-      tc_fence_after();
-      int pst = 0;
-      uint32_t pjt = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int buf = jt & 1;
-        if (!warp_wait(&kv_full[stage], kv_phase, P, abort_flag)) { ok = false; break; }
-        if (jt >= 2 && !warp_wait(&pv_done[buf], ((jt - 2) >> 1) & 1, P, abort_flag)) {
+      if (!warp_wait(&kv_full[stage], kv_phase, P, abort_flag)) break;
+#pragma unroll
+      for (int w = 0; w < NWG; ++w) {
+        if (it.nkv[w] == 0) continue;
+        if (!C::SEP_P && n_pv[w] > 0 &&
+            !warp_wait(&pv_done[w], (n_pv[w] - 1) & 1, P, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t k_addr = smem_u32(sKV + stage * 2 * C::TILE_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const int ch = (kk * 16) / C::CW, off = ((kk * 16) % C::CW) * 2;
-            const uint64_t qd = smem_desc(q_addr + ch * C::CHUNK_BYTES + off, 8 * C::ROW_BYTES, C::LAYOUT);
-            const uint64_t kd = smem_desc(k_addr + ch * C::CHUNK_BYTES + off, 8 * C::ROW_BYTES, C::LAYOUT);
-            mma_ss(tmem + buf * 128, qd, kd, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&s_full[buf]);
-          if (j == nkv - 1) mma_commit(q_empty);
-        }
-        __syncwarp();
-        if (j >= 1 && !issue_pv(pst, pjt, j == 1)) { ok = false; break; }
-        pst = stage;
-        pjt = jt;
-        ++jt;
-        if (++stage == C::STAGES) {
-          stage = 0;
-          kv_phase ^= 1;
-        }
+        if (lane == 0) GQE_ISSUE_S(w, stage);
+        ++n_s[w];
       }
       if (!ok) break;
-      if (!issue_pv(pst, pjt, nkv == 1)) break;
-      if (lane == 0) mma_commit(o_full);
+      if (nk == 1 && lane == 0) mma_commit(q_empty);
+      for (int j = 0; j < nk; ++j) {
+        const int cur = stage;
+        int nxt = stage + 1;
+        uint32_t nxt_phase = kv_phase;
+        if (nxt == C::STAGES) {
+          nxt = 0;
+          nxt_phase ^= 1;
+        }
+        bool next_loaded = false;
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) {
+          if (j >= it.nkv[w]) continue;
+          const bool more = j + 1 < it.nkv[w];
+          if (!warp_wait(&p_ready[w], (n_s[w] - 1) & 1, P, abort_flag)) { ok = false; break; }
+          if (j == 0 && n_o[w] > 0 &&
+              !warp_wait(&o_free[w], (n_o[w] - 1) & 1, P, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (more && !next_loaded) {
+            if (!warp_wait(&kv_full[nxt], nxt_phase, P, abort_flag)) { ok = false; break; }
+            next_loaded = true;
+          }
+          tc_fence_after();
+          if (C::SEP_P) {
+            // P_w has its own columns: the next S_w first (its softmax resumes sooner),
+            // then this tile's P_w V.
+            if (lane == 0) {
+              if (more) GQE_ISSUE_S(w, nxt);
+              GQE_ISSUE_PV(w, cur, j == 0);
+              if (!more) mma_commit(&o_full[w]);
+            }
+            ++n_pv[w];
+            if (more) ++n_s[w];
+          } else {
+            // P_w overlays S_w: S_w(j+1) waits for P_w(j) V.
+            if (lane == 0) {
+              GQE_ISSUE_PV(w, cur, j == 0);
+              if (!more) mma_commit(&o_full[w]);
+            }
+            ++n_pv[w];
+            if (more) {
+              if (!warp_wait(&pv_done[w], (n_pv[w] - 1) & 1, P, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              if (lane == 0) GQE_ISSUE_S(w, nxt);
+              ++n_s[w];
+            }
+          }
+          if (!more) ++n_o[w];
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          if (j + 2 == nk) mma_commit(q_empty);  // the item's last S products are issued
+          mma_commit(&kv_empty[cur]);
+        }
+        stage = nxt;
+        kv_phase = nxt_phase;
+      }
       __syncwarp();
-      ++item_no;
     }
+#undef GQE_ISSUE_S
+#undef GQE_ISSUE_PV
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int quarter = warp & 3;
+    const int w = (warp - 2) / 4;   // query tile of this warpgroup
+    const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint32_t jt = 0;
-    int item_no = 0;
+    const uint32_t t_s = tmem + lane_off + w * 128;
+    const uint32_t t_p = tmem + lane_off + C::p_col(w);
+    const uint32_t t_o = tmem + lane_off + C::O_COL + w * DH;
+    uint32_t n_s = 0, n_o = 0;
     const float cs = P.scale_log2;
     for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
       const Item it = decode(P, i);
-      const int q0 = it.qt * TQ;
+      const int nkv = it.nkv[w];
+      if (nkv == 0) continue;
+      const int q0 = (it.pair * NWG + w) * TQ;
       const int q = q0 + row;  // query position within the sequence
-      const int nkv = kv_tiles(P, it);
       float m_used = 0.f, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nkv; ++j, ++jt) {
-        const int buf = jt & 1;
-        if (!warp_wait(&s_full[buf], (jt >> 1) & 1, P, abort_flag)) { ok = false; break; }
+      for (int j = 0; j < nkv; ++j) {
+        if (!warp_wait(&s_full[w], n_s & 1, P, abort_flag)) { ok = false; break; }
+        ++n_s;
         tc_fence_after();
         float s[TK];
         {
-          uint32_t r[32];
+          uint32_t r[TK];
+          tmem_ld128_wait(t_s, r);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tmem + lane_off + buf * 128 + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
-          }
+          for (int c = 0; c < TK; ++c) s[c] = __uint_as_float(r[c]);
         }
         const int kv0 = j * TK;
-        const bool edge = (P.causal && kv0 + TK - 1 > q0) || (kv0 + TK > P.T);
-        if (edge) {
+        if ((P.causal && kv0 + TK - 1 > q0) || (kv0 + TK > P.T)) {
+          // keys past the sequence end, and (causal) keys after this query
+          const int lim = P.causal ? min(q + 1, P.T) : P.T;
 #pragma unroll
-          for (int c = 0; c < TK; ++c) {
-            const int key = kv0 + c;
-            if (key >= P.T || (P.causal && key > q)) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < TK; ++c)
+            if (kv0 + c >= lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row maximum: eight independent chains, then a tree
+        float mp[8];
 #pragma unroll
-        for (int c = 1; c < TK; ++c) mx = fmaxf(mx, s[c]);
+        for (int x = 0; x < 8; ++x) mp[x] = s[x];
+#pragma unroll
+        for (int c = 8; c < TK; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         float m_new = mx * cs;
         if (m_new == -INFINITY) m_new = 0.f;  // a row with every key masked
         bool need = false;
@@ -326,43 +394,57 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
           alpha = fast_exp2(m_used - m_new);
           m_used = m_new;
         }
+        // With separate P buffers, S_w(j) was issued without waiting for P_w(j-1) V: wait
+        // for that product before overwriting P_w or rescaling O_w.
+        if (C::SEP_P && n_s > 1 &&
+            !warp_wait(&pv_done[w], (n_s - 2) & 1, P, abort_flag)) {
+          ok = false;
+          break;
+        }
         if (__any_sync(0xffffffffu, need)) {
-          // O holds the sum through KV tile j-1: wait for that P V, then rescale in TMEM.
-          if (!warp_wait(&pv_done[buf ^ 1], ((jt - 1) >> 1) & 1, P, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+          // O_w holds the sum through KV tile j-1; that P V finished before S_w(j) was
+          // issued, so O_w can be rescaled in place now.
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 16) {
             uint32_t r[16];
-            tmem_ld16(tmem_o + lane_off + c0, r);
-            tmem_wait_ld();
+            tmem_ld16_wait(t_o + c0, r);
 #pragma unroll
             for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-            tmem_st16(tmem_o + lane_off + c0, r);
+            tmem_st16(t_o + c0, r);
           }
-          tmem_wait_st();
           l *= alpha;
         }
-        const float neg_m = -m_used;
+        // p = exp2(s * scale - m): packed FMA for the argument, MUFU ex2, four packed
+        // partial sums; P goes back over the first 64 columns of S_w as bf16 pairs.
+        const float2 cs2 = make_float2(cs, cs);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c0 = 0; c0 < TK; c0 += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const float p0 = fast_exp2(fmaf(s[c0 + 2 * x], cs, neg_m));
-            const float p1 = fast_exp2(fmaf(s[c0 + 2 * x + 1], cs, neg_m));
-            l += p0 + p1;
-            pk[x] = pack_bf16x2(p0, p1);
+            const float2 t = fma2(make_float2(s[c0 + 2 * x], s[c0 + 2 * x + 1]), cs2, nm2);
+            const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            lsum[x & 3] = add2(lsum[x & 3], p);
+            pk[x] = pack_bf16x2(p.x, p.y);
           }
-          tmem_st16(tmem + lane_off + buf * 128 + c0 / 2, pk);
+          tmem_st16(t_p + c0 / 2, pk);
+        }
+        {
+          const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
+          l += a.x + a.y;
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[buf]);
+        if (lane == 0) mbar_arrive(&p_ready[w]);
       }
       if (!ok) break;
-      // ---- epilogue: O / l into Z
-      if (!warp_wait(o_full, item_no & 1, P, abort_flag)) break;
+      // ---- epilogue: O_w / l into Z
+      if (!warp_wait(&o_full[w], n_o & 1, P, abort_flag)) break;
+      ++n_o;
       tc_fence_after();
       const bool valid = q < P.T;
       const int64_t tok = (int64_t)it.b * P.T + q;
@@ -378,8 +460,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
 #pragma unroll
       for (int c0 = 0; c0 < DH; c0 += 16) {
         uint32_t r[16];
-        tmem_ld16(tmem_o + lane_off + c0, r);
-        tmem_wait_ld();
+        tmem_ld16_wait(t_o + c0, r);
         if (valid) {
           uint4 v0, v1;
           v0.x = pack_bf16x2(__uint_as_float(r[0]) * scale, __uint_as_float(r[1]) * scale);
@@ -396,8 +477,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
-      ++item_no;
+      if (lane == 0) mbar_arrive(&o_free[w]);
     }
   }
   tc_fence_before();
@@ -442,7 +522,8 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
   P.weighted = weighted;
   P.causal = causal;
   P.nq = (T + TQ - 1) / TQ;
-  P.items = B * S * P.nq;
+  P.npairs = (P.nq + NWG - 1) / NWG;
+  P.items = B * S * P.npairs;
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   P.status = h->ws.status;
   P.spin = h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22;

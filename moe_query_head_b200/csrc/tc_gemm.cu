@@ -303,8 +303,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
         }
         for (int c0 = 0; c0 < ti.n; c0 += 16) {
           uint32_t r[16];
-          tmem_ld16(t_row + c0, r);
-          tmem_wait_ld();
+          tmem_ld16_wait(t_row + c0, r);
           if (valid && c0 < P.d_h) {
             uint4 v0, v1;
             v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
@@ -325,8 +324,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
         const int64_t m = ti.m0 + row;
         for (int c0 = 0; c0 < ti.n; c0 += 16) {
           uint32_t r[16];
-          tmem_ld16(t_row + c0, r);
-          tmem_wait_ld();
+          tmem_ld16_wait(t_row + c0, r);
           if (!valid) continue;
 #pragma unroll
           for (int g8 = 0; g8 < 2; ++g8) {
