@@ -96,7 +96,8 @@ route_select_kernel(const float* __restrict__ logits, int M, int N, int G,
                                     float* __restrict__ gates, float* __restrict__ wslot,
                                     int32_t* __restrict__ part_counts,
                                     float* __restrict__ part_prob);
-__global__ void route_scan_aux_kernel(int32_t* __restrict__ part_counts,
+__global__ void __launch_bounds__(1024)
+route_scan_aux_kernel(int32_t* __restrict__ part_counts,
                                       const float* __restrict__ part_prob, int nblk, int M,
                                       int N, int G, int k, int32_t* __restrict__ counts,
                                       float* __restrict__ mean_prob,

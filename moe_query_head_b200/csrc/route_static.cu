@@ -87,7 +87,7 @@ extern "C" gqe_status gqe_route_static(const float* logits, int M, int N, int G,
   route_select_kernel<<<nblk, kRouteBlock, 0, st>>>(logits, M, N, G, k, sel, psel, gates, wslot,
                                                      part_counts, part_prob);
   if (cudaGetLastError() != cudaSuccess) return GQE_ERR_CUDA;
-  route_scan_aux_kernel<<<1, kMaxExperts, 0, st>>>(part_counts, part_prob, nblk, M, N, G, k,
+  route_scan_aux_kernel<<<1, 1024, 0, st>>>(part_counts, part_prob, nblk, M, N, G, k,
                                                     counts, mean_prob, offsets, aux_loss);
   if (cudaGetLastError() != cudaSuccess) return GQE_ERR_CUDA;
   return GQE_OK;

@@ -230,16 +230,33 @@ attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __r
 
 // Variant gqe: the renormalised slot rho_t = sum_s w[t, s] * O[t, s] over the routed
 // streams, read back from Z's routed blocks and written to Z's slot block.
+// One thread per 16 bytes of the slot (8 bf16 or 4 fp32 values): 16-byte loads of every
+// routed block, fp32 accumulation, one 16-byte store.
 template <typename T>
 __global__ void slot_kernel(T* __restrict__ Z, const float* __restrict__ w, int M, int Sr,
                             int d_h, int Do) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int per_tok = d_h / VEC;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (int64_t)M * d_h) return;
-  const int64_t t = i / d_h;
-  const int c = (int)(i % d_h);
-  float acc = 0.f;
-  for (int s = 0; s < Sr; ++s) acc = fmaf(w[t * Sr + s], to_f32(Z[t * Do + s * d_h + c]), acc);
-  Z[t * Do + (int64_t)Sr * d_h + c] = from_f32<T>(acc);
+  if (i >= (int64_t)M * per_tok) return;
+  const int64_t t = i / per_tok;
+  const int c0 = (int)(i % per_tok) * VEC;
+  float acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+  const T* zt = Z + t * Do + c0;
+  for (int s = 0; s < Sr; ++s) {
+    const float ws = w[t * Sr + s];
+    const uint4 raw = *reinterpret_cast<const uint4*>(zt + (int64_t)s * d_h);
+    const T* val = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = fmaf(ws, to_f32(val[v]), acc[v]);
+  }
+  uint4 out;
+  T* o = reinterpret_cast<T*>(&out);
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) o[v] = from_f32<T>(acc[v]);
+  *reinterpret_cast<uint4*>(Z + t * Do + (int64_t)Sr * d_h + c0) = out;
 }
 
 template <typename T>
@@ -328,7 +345,7 @@ int launch_simt_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int v
 int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st) {
   if (variant != GQE_VARIANT_GQE) return 0;  // weighted_concat is applied in attention
   const int Sr = h->G * h->k;
-  const int64_t n = (int64_t)M * h->d_h;
+  const int64_t n = (int64_t)M * h->d_h / (16 / h->esz);
   const int blocks = (int)((n + 255) / 256);
   if (h->dtype == GQE_F32)
     slot_kernel<float><<<blocks, 256, 0, st>>>(static_cast<float*>(h->ws.Z), h->ws.w, M, Sr,

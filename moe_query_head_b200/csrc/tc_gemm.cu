@@ -34,11 +34,11 @@ constexpr int BM = 128;        // tile rows = MMA M = TMEM lanes
 constexpr int BN = 128;        // widest tile (MMA N)
 constexpr int BK = 64;         // one 128-byte swizzle atom of bf16 along K
 constexpr int STAGES = 6;
-constexpr int GATHER_LAG = 3;  // cp.async stages in flight before their barrier arrival
 constexpr int THREADS = 192;
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int B_STAGE_BYTES = BN * BK * 2;
-constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256 +
+                           BM * 4 /*gathered row indices*/;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_PROBLEMS = 4;
 
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], GATHER ? 33 : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    if (!GATHER) prefetch_tmap(&P.tmap_a);
+    prefetch_tmap(&P.tmap_a);
     for (int p = 0; p < P.nprob; ++p) prefetch_tmap(&P.tmap_b[p]);
   }
   tc_fence_before();
@@ -159,61 +159,40 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     // ------------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
-    int issued = 0;  // stages issued whose gather arrival is still pending (GATHER)
-    int pend_stage[GATHER_LAG + 1];
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
       const TileInfo ti = tile_info<GATHER>(P, tile);
       const int brow = GATHER ? ti.p * P.d_h : ti.n0;
       const int tb = GATHER ? 0 : ti.p;
       const uint32_t b_bytes = (uint32_t)P.prob[GATHER ? 0 : ti.p].box_n * BK * 2;
-      // gather mode: this lane's four rows of the tile and their source tokens
-      int64_t src_row[4];
+      // gather mode: lane l loads tile rows 4l .. 4l+3; their source token rows (rows past
+      // the tile's end repeat its first row: they are computed and never stored)
+      int g_rows[4] = {0, 0, 0, 0};
       if constexpr (GATHER) {
+        const int first = P.bucket[ti.m0] >> 3;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int r = lane + 32 * i;
-          src_row[i] = r < ti.rows ? (int64_t)(P.bucket[ti.m0 + r] >> 3) : -1;
+          const int r = 4 * lane + i;
+          g_rows[i] = r < ti.rows ? (P.bucket[ti.m0 + r] >> 3) : first;
         }
       }
       for (int kb = 0; kb < KB; ++kb) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        bool ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
+        ok = !__any_sync(0xffffffffu, !ok);
         if (!ok) {
           if (lane == 0) set_timeout(P, abort_flag);
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], (GATHER ? 0u : (uint32_t)A_STAGE_BYTES) + b_bytes);
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)A_STAGE_BYTES + b_bytes);
           if (!GATHER) tma_load_2d(sA + stage * A_STAGE_BYTES, &P.tmap_a, kb * BK, ti.m0, &full[stage]);
           tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[tb], kb * BK, brow, &full[stage]);
         }
         if constexpr (GATHER) {
-          const uint32_t base = smem_u32(sA + stage * A_STAGE_BYTES);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int kcol = kb * BK + c * 8;
-              const bool ok_src = src_row[i] >= 0 && kcol < P.K;
-              const void* src = ok_src ? (const void*)(P.x + src_row[i] * P.K + kcol)
-                                       : (const void*)P.x;
-              const uint32_t dst = base + r * 128 + ((c ^ (r & 7)) << 4);
-              cp_async_16(dst, src, ok_src ? 16u : 0u);
-            }
-          }
-          cp_async_commit();
-          pend_stage[issued] = stage;
-          ++issued;
-          if (issued > GATHER_LAG) {
-            cp_async_wait<GATHER_LAG>();
-            fence_async_shared();
-            mbar_arrive(&full[pend_stage[0]]);
-#pragma unroll
-            for (int i = 0; i < GATHER_LAG; ++i) pend_stage[i] = pend_stage[i + 1];
-            --issued;
-          }
+          // TMA row gather: four 128-byte row segments per lane into rows 4l .. 4l+3 of
+          // the 128-byte-swizzled A tile (the swizzle follows the destination address).
+          __syncwarp();
+          tma_gather4(sA + stage * A_STAGE_BYTES + lane * 4 * 128, &P.tmap_a, kb * BK,
+                      g_rows[0], g_rows[1], g_rows[2], g_rows[3], &full[stage]);
         }
         if (++stage == STAGES) {
           stage = 0;
@@ -221,13 +200,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
         }
       }
     }
-    if constexpr (GATHER) {
-      cp_async_wait<0>();
-      fence_async_shared();
-      for (int i = 0; i < issued; ++i) mbar_arrive(&full[pend_stage[i]]);
-    }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    const uint64_t a_desc0 = smem_desc(smem_u32(sA), 1024, kSwizzle128B);
+    const uint64_t b_desc0 = smem_desc(smem_u32(sB), 1024, kSwizzle128B);
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
@@ -236,8 +212,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1, P.spin);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ok = mbar_wait(&acc_empty[acc], acc_phase ^ 1, P.spin);
+      ok = !__any_sync(0xffffffffu, !ok);
       if (!ok) {
         if (lane == 0) set_timeout(P, abort_flag);
         break;
@@ -246,22 +222,20 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       const uint32_t d_tmem = tmem_base + acc * BN;
       const uint32_t idesc = idesc_bf16_f32(BM, ti.n);
       for (int kb = 0; kb < KB; ++kb) {
-        if (lane == 0) ok = mbar_wait(&full[stage], phase, P.spin);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ok = mbar_wait(&full[stage], phase, P.spin);
+        ok = !__any_sync(0xffffffffu, !ok);
         if (!ok) {
           if (lane == 0) set_timeout(P, abort_flag);
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE_BYTES);
+          // descriptor = base + offset in 16-byte units (K step: 32 bytes inside the atom)
+          const uint64_t ad = a_desc0 + (uint64_t)(stage * (A_STAGE_BYTES >> 4));
+          const uint64_t bd = b_desc0 + (uint64_t)(stage * (B_STAGE_BYTES >> 4));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc(a_addr + kk * 32, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(b_addr + kk * 32, 1024, kSwizzle128B);
-            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           mma_commit(&empty[stage]);  // frees the stage when these MMAs finish
         }
         __syncwarp();
@@ -284,8 +258,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_phase, P.spin);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ok = mbar_wait(&acc_full[acc], acc_phase, P.spin);
+      ok = !__any_sync(0xffffffffu, !ok);
       if (!ok) {
         if (lane == 0) set_timeout(P, abort_flag);
         break;
@@ -373,13 +347,29 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
 }
 
 // Tiles of the routed projection: each expert's bucket cut into runs of BM slots.
+// One thread per expert (N <= 64): tile counts, an exclusive scan, then each thread writes
+// its expert's tiles.
 __global__ void qproj_tiles_kernel(const int32_t* __restrict__ offsets, int N,
                                    int2* __restrict__ tile_list, int32_t* __restrict__ tile_count) {
-  if (threadIdx.x != 0) return;
-  int n = 0;
-  for (int e = 0; e < N; ++e)
-    for (int s = offsets[e]; s < offsets[e + 1]; s += BM) tile_list[n++] = make_int2(e, s);
-  *tile_count = n;
+  __shared__ int s_n[kMaxExperts + 1];
+  const int e = threadIdx.x;
+  const int beg = e < N ? offsets[e] : 0;
+  const int cnt = e < N ? offsets[e + 1] - beg : 0;
+  const int nt = (cnt + BM - 1) / BM;
+  if (e < kMaxExperts) s_n[e] = nt;
+  __syncthreads();
+  if (e == 0) {
+    int run = 0;
+    for (int i = 0; i < N; ++i) {
+      const int v = s_n[i];
+      s_n[i] = run;
+      run += v;
+    }
+    *tile_count = run;
+  }
+  __syncthreads();
+  if (e < N)
+    for (int i = 0; i < nt; ++i) tile_list[s_n[e] + i] = make_int2(e, beg + i * BM);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -485,10 +475,14 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
 }
 
 int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st) {
-  qproj_tiles_kernel<<<1, 32, 0, st>>>(h->ws.offsets, h->N, h->ws.tile_list, h->ws.tile_count);
+  qproj_tiles_kernel<<<1, kMaxExperts, 0, st>>>(h->ws.offsets, h->N, h->ws.tile_list,
+                                                 h->ws.tile_count);
   if (cudaGetLastError() != cudaSuccess) return -1;
   Params P;
   memset(&P, 0, sizeof(P));
+  // A: rows of x gathered four at a time (box one row high, 128 bytes wide)
+  if (!tmap_bf16_2d(&P.tmap_a, x, h->dim, M, h->dim, BK, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return -1;
   P.prob[0] = make_problem(h->d_h, OutMap{});
   if (!tmap_bf16_2d(&P.tmap_b[0], W_q, h->dim, (uint64_t)h->N * h->d_h, h->dim, BK,
                     P.prob[0].box_n, CU_TENSOR_MAP_SWIZZLE_128B))
