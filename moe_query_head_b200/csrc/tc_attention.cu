@@ -6,21 +6,23 @@
 // Every stream has one query per token, so the work is a grouped-query attention with
 // S = G*k + 1 query heads over G KV heads; the savings of GQE come from S < N + 1.
 //
-// Work item = (sequence b, stream s, two consecutive 128-query tiles); a persistent CTA per
-// SM takes items heaviest first (causal tiles near the end of a sequence have the most
-// keys). The two query tiles share every K/V tile and are handled by two softmax
-// warpgroups that ping-pong: while one computes exponentials, the tensor core runs the
-// other's products, and each hides the other's waits.
-//   warp 0      TMA: both Q tiles once per item, then K and V tiles into a ring of stages;
-//   warp 1      TMEM owner; one lane issues, per query tile w, S_w = Q_w K^T (A and B from
-//               shared memory) into TMEM, and O_w += P_w V with P_w read from TMEM (the TS
-//               form) and V as an MN-major shared-memory operand;
-//   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: one query row per
-//               thread, 128 scores per KV tile in registers, exp2 against the running row
-//               maximum, P written back over S as bf16 pairs. O is rescaled in TMEM only
-//               when a row maximum grows by more than 2^8 (rare after the first tiles).
-//               At the end of an item the same warps normalise O by the row sum, apply the
-//               weighted_concat scale if any, and store the row into its block of Z.
+// Work item = (sequence b, stream s, 128-query tile); persistent CTAs, two per SM, take
+// items heaviest first (causal tiles near the end of a sequence have the most keys). The
+// two CTAs of an SM interleave: while one computes exponentials the other's products run,
+// and each hides the other's waits. Per CTA:
+//   warp 0     TMA: the Q tile once per item, then K and V tiles into a ring of stages;
+//   warp 1     owns 256 TMEM columns; one lane issues S = Q K^T (A and B from shared
+//              memory) into TMEM and O += P V with P read from TMEM (the TS form) and V as
+//              an MN-major shared-memory operand;
+//   warps 2-5  softmax: one query row per thread, 128 scores per KV tile in registers,
+//              exp2 against the running row maximum, P written to TMEM as bf16 pairs. O is
+//              rescaled in TMEM only when a row maximum grows by more than 2^8 (rare after
+//              the first tiles). At the end of an item the same warps normalise O by the
+//              row sum, apply the weighted_concat scale if any, and store the row into its
+//              block of Z.
+// P has TMEM columns of its own: as soon as the softmax warps have pulled S(j) into
+// registers, S(j+1) is computed, so it is ready when they finish tile j. (Head dims above 64
+// run one CTA per SM with 512 TMEM columns; the shared memory of two would not fit.)
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
@@ -36,10 +38,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int NWG = 2;                 // query tiles per item = softmax warpgroups
-constexpr int THREADS = 64 + NWG * 128;
-constexpr int TQ = 128;                // queries per tile (MMA M, TMEM lanes)
-constexpr int TK = 128;                // keys per tile (S MMA N)
+constexpr int THREADS = 192;
+constexpr int TQ = 128;                    // queries per tile (MMA M, TMEM lanes)
+constexpr int TK = 128;                    // keys per tile (S MMA N)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int DH>
@@ -51,15 +52,16 @@ struct Cfg {
   static constexpr int ROW_BYTES = CW * 2;          // bytes per row inside a chunk
   static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;
   static constexpr int TILE_BYTES = 128 * DH * 2;   // one Q, K or V tile
-  static constexpr int STAGES = DH <= 64 ? 4 : (DH <= 96 ? 3 : 2);
-  static constexpr int SMEM = NWG * TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
-  // TMEM columns (512): S_w at 128 w. For DH <= 64, P_w has columns of its own
-  // (256 + 64 w) and O_w sits at 384 + DH w, so S_w(j+1) can be computed while P_w(j) V
-  // is still being read. For larger DH, P_w overlays the first half of S_w and O_w sits at
-  // 256 + DH w; S_w(j+1) then waits for that product.
-  static constexpr bool SEP_P = DH <= 64;
-  static constexpr int O_COL = SEP_P ? 384 : 256;
-  __device__ static constexpr int p_col(int w) { return SEP_P ? 256 + 64 * w : 128 * w; }
+  // Two CTAs per SM while both fit (TMEM 256 columns each, shared memory), else one.
+  static constexpr int CTAS = DH <= 64 ? 2 : 1;
+  static constexpr int TMEM_COLS = CTAS == 2 ? 256 : 512;
+  static constexpr int STAGES = DH <= 48 ? 4 : (DH <= 64 ? 2 : (DH <= 96 ? 3 : 2));
+  static constexpr int SMEM = TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
+  // TMEM columns: S at 0, P (bf16 pairs) at 128, O at 192.
+  static constexpr int P_COL = 128;
+  static constexpr int O_COL = 192;
+  static_assert(O_COL + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory budget");
 };
 
 struct Params {
@@ -67,7 +69,7 @@ struct Params {
   __nv_bfloat16* Z;
   const float* psel;
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
-  int nq, npairs, items;
+  int nq, items;
   float scale_log2;
   int32_t* status;
   int64_t spin;
@@ -80,21 +82,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 struct Item {
-  int b, s, pair;
-  int nkv[NWG];  // KV tiles of each query tile (0: the tile is past the sequence end)
+  int b, s, qt, nkv;
 };
 __device__ __forceinline__ Item decode(const Params& P, int i) {
   Item it;
   const int bs = P.B * P.S;
-  it.pair = P.causal ? P.npairs - 1 - i / bs : i / bs;
+  it.qt = P.causal ? P.nq - 1 - i / bs : i / bs;
   const int r = i % bs;
   it.s = r % P.S;
   it.b = r / P.S;
-#pragma unroll
-  for (int w = 0; w < NWG; ++w) {
-    const int qt = it.pair * NWG + w;
-    it.nkv[w] = qt >= P.nq ? 0 : (P.causal ? qt + 1 : P.nq);
-  }
+  it.nkv = P.causal ? it.qt + 1 : P.nq;
   return it;
 }
 
@@ -111,24 +108,26 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(THREADS, Cfg<DH>::CTAS)
+attn_kernel(const __grid_constant__ Params P) {
   using C = Cfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;                              // NWG tiles
-  uint8_t* sKV = smem + NWG * C::TILE_BYTES;       // per stage: K tile, V tile
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::TILE_BYTES;  // per stage: K tile, V tile
   uint64_t* bar = reinterpret_cast<uint64_t*>(sKV + C::STAGES * 2 * C::TILE_BYTES);
   uint64_t* q_full = bar;
   uint64_t* q_empty = bar + 1;
   uint64_t* kv_full = bar + 2;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;  // [NWG]
-  uint64_t* p_ready = s_full + NWG;         // [NWG]
-  uint64_t* pv_done = p_ready + NWG;        // [NWG]
-  uint64_t* o_full = pv_done + NWG;         // [NWG]
-  uint64_t* o_free = o_full + NWG;          // [NWG]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + NWG);
+  uint64_t* s_full = kv_empty + C::STAGES;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_ready = s_free + 1;
+  uint64_t* pv_done = p_ready + 1;
+  uint64_t* o_full = pv_done + 1;
+  uint64_t* o_free = o_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -139,18 +138,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int w = 0; w < NWG; ++w) {
-      mbar_init(&s_full[w], 1);
-      mbar_init(&p_ready[w], 4);
-      mbar_init(&pv_done[w], 1);
-      mbar_init(&o_full[w], 1);
-      mbar_init(&o_free[w], 4);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_ready, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -161,7 +159,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_holder;  // S_w at columns 128 w, O_w at 256 + DH w
+  const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA loads
@@ -170,41 +168,33 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       uint32_t kv_phase = 0, q_phase = 0;
       for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
         const Item it = decode(P, i);
-        const int nk = max(it.nkv[0], it.nkv[1]);
         if (!mbar_wait(q_empty, q_phase ^ 1, P.spin)) {
           *abort_flag = 1;
           atomicExch(P.status, kStatusTimeout);
           break;
         }
         q_phase ^= 1;
-        int nq_tiles = 0;
+        mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+        const int qrow = it.s * P.M + it.b * P.T + it.qt * TQ;
 #pragma unroll
-        for (int w = 0; w < NWG; ++w) nq_tiles += it.nkv[w] > 0;
-        mbar_arrive_expect_tx(q_full, nq_tiles * C::TILE_BYTES);
-#pragma unroll
-        for (int w = 0; w < NWG; ++w) {
-          if (it.nkv[w] == 0) continue;
-          const int qrow = it.s * P.M + it.b * P.T + (it.pair * NWG + w) * TQ;
-#pragma unroll
-          for (int c = 0; c < C::NC; ++c)
-            tma_load_2d(sQ + w * C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow,
-                        q_full);
-        }
+        for (int c = 0; c < C::NC; ++c)
+          tma_load_2d(sQ + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow, q_full);
         const int kvh = it.s < P.Sr ? it.s / P.k : 0;
-        for (int j = 0; j < nk; ++j) {
+        const int krow0 = kvh * P.M + it.b * P.T;
+        for (int j = 0; j < it.nkv; ++j) {
           if (!mbar_wait(&kv_empty[stage], kv_phase ^ 1, P.spin)) {
             *abort_flag = 1;
             atomicExch(P.status, kStatusTimeout);
             break;
           }
           mbar_arrive_expect_tx(&kv_full[stage], 2 * C::TILE_BYTES);
-          const int krow = kvh * P.M + it.b * P.T + j * TK;
           uint8_t* sK = sKV + stage * 2 * C::TILE_BYTES;
 #pragma unroll
           for (int c = 0; c < C::NC; ++c) {
-            tma_load_2d(sK + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW, krow, &kv_full[stage]);
-            tma_load_2d(sK + C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW, krow,
+            tma_load_2d(sK + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW, krow0 + j * TK,
                         &kv_full[stage]);
+            tma_load_2d(sK + C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW,
+                        krow0 + j * TK, &kv_full[stage]);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -215,9 +205,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
-    // This warp shares its sub-partition with two busy softmax warps, so it keeps its
-    // instruction count small: descriptors are built once, and each product's descriptor
-    // is a base plus a constant (the address field is the low 14 bits, in 16-byte units).
+    // Lean: descriptors are built once; each product's descriptor is a base plus a
+    // constant (the address field is the low 14 bits, in 16-byte units).
     const uint32_t idesc_s = idesc_bf16_f32(TQ, TK);
     const uint32_t idesc_pv = idesc_bf16_f32(TQ, DH) | (1u << 16);  // B (V) MN-major
     const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
@@ -225,56 +214,45 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
     const uint64_t v_desc =
         smem_desc_mn(smem_u32(sKV + C::TILE_BYTES), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
     constexpr uint32_t kStageStep = (2 * C::TILE_BYTES) >> 4;
-    constexpr uint32_t kTileStep = C::TILE_BYTES >> 4;
     int stage = 0;
     uint32_t kv_phase = 0, q_phase = 0;
-    // per query tile: uses of s_full (= p_ready) / pv_done / o_full so far
-    uint32_t n_s[NWG] = {0, 0}, n_pv[NWG] = {0, 0}, n_o[NWG] = {0, 0};
+    uint32_t n_sf = 0, n_p = 0, n_pv = 0, n_o = 0;  // uses of s_free / p_ready / pv_done / o_full
     bool ok = true;
 
-    // S_w = Q_w K^T for the K tile in stage `st` (lane 0 only).
-#define GQE_ISSUE_S(w, st)                                                                   \
+    // S = Q K^T for the K tile in stage `st` (lane 0 only).
+#define GQE_ISSUE_S(st)                                                                      \
   do {                                                                                       \
-    const uint64_t qd = q_desc + (uint64_t)((w) * kTileStep);                                \
     const uint64_t kd = k_desc + (uint64_t)((st) * kStageStep);                              \
     _Pragma("unroll") for (int kk = 0; kk < DH / 16; ++kk) {                                 \
       const uint32_t o = (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4; \
-      mma_ss(tmem + (w) * 128, qd + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);                   \
+      mma_ss(tmem, q_desc + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);                           \
     }                                                                                        \
-    mma_commit(&s_full[w]);                                                                  \
+    mma_commit(s_full);                                                                      \
   } while (0)
-    // O_w += P_w V for the V tile in stage `st` (lane 0 only). V is the MN-major B operand
+    // O += P V for the V tile in stage `st` (lane 0 only). V is the MN-major B operand
     // (N = head dim, K = keys): 16 keys are two 8-row groups of every chunk.
-#define GQE_ISSUE_PV(w, st, first)                                                           \
+#define GQE_ISSUE_PV(st, first)                                                              \
   do {                                                                                       \
     const uint64_t vd = v_desc + (uint64_t)((st) * kStageStep);                              \
     _Pragma("unroll") for (int kk = 0; kk < TK / 16; ++kk)                                   \
-        mma_ts(tmem + C::O_COL + (w) * DH, tmem + C::p_col(w) + kk * 8,                      \
+        mma_ts(tmem + C::O_COL, tmem + C::P_COL + kk * 8,                                    \
                vd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_pv,                     \
                ((first) && kk == 0) ? 0u : 1u);                                              \
-    mma_commit(&pv_done[w]);                                                                 \
+    mma_commit(pv_done);                                                                     \
   } while (0)
 
     for (int i = blockIdx.x; i < P.items && ok && !*abort_flag; i += gridDim.x) {
       const Item it = decode(P, i);
-      const int nk = max(it.nkv[0], it.nkv[1]);
+      const int nk = it.nkv;
       if (!warp_wait(q_full, q_phase, P, abort_flag)) break;
       q_phase ^= 1;
       if (!warp_wait(&kv_full[stage], kv_phase, P, abort_flag)) break;
-#pragma unroll
-      for (int w = 0; w < NWG; ++w) {
-        if (it.nkv[w] == 0) continue;
-        if (!C::SEP_P && n_pv[w] > 0 &&
-            !warp_wait(&pv_done[w], (n_pv[w] - 1) & 1, P, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) GQE_ISSUE_S(w, stage);
-        ++n_s[w];
+      tc_fence_after();
+      if (lane == 0) {
+        GQE_ISSUE_S(stage);
+        if (nk == 1) mma_commit(q_empty);
       }
-      if (!ok) break;
-      if (nk == 1 && lane == 0) mma_commit(q_empty);
+      __syncwarp();
       for (int j = 0; j < nk; ++j) {
         const int cur = stage;
         int nxt = stage + 1;
@@ -283,81 +261,59 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
           nxt = 0;
           nxt_phase ^= 1;
         }
-        bool next_loaded = false;
-#pragma unroll
-        for (int w = 0; w < NWG; ++w) {
-          if (j >= it.nkv[w]) continue;
-          const bool more = j + 1 < it.nkv[w];
-          if (!warp_wait(&p_ready[w], (n_s[w] - 1) & 1, P, abort_flag)) { ok = false; break; }
-          if (j == 0 && n_o[w] > 0 &&
-              !warp_wait(&o_free[w], (n_o[w] - 1) & 1, P, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (more && !next_loaded) {
-            if (!warp_wait(&kv_full[nxt], nxt_phase, P, abort_flag)) { ok = false; break; }
-            next_loaded = true;
-          }
+        const bool more = j + 1 < nk;
+        if (more) {
+          // S(j) is in the softmax registers: compute S(j+1) now.
+          if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!warp_wait(&kv_full[nxt], nxt_phase, P, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          if (C::SEP_P) {
-            // P_w has its own columns: the next S_w first (its softmax resumes sooner),
-            // then this tile's P_w V.
-            if (lane == 0) {
-              if (more) GQE_ISSUE_S(w, nxt);
-              GQE_ISSUE_PV(w, cur, j == 0);
-              if (!more) mma_commit(&o_full[w]);
-            }
-            ++n_pv[w];
-            if (more) ++n_s[w];
-          } else {
-            // P_w overlays S_w: S_w(j+1) waits for P_w(j) V.
-            if (lane == 0) {
-              GQE_ISSUE_PV(w, cur, j == 0);
-              if (!more) mma_commit(&o_full[w]);
-            }
-            ++n_pv[w];
-            if (more) {
-              if (!warp_wait(&pv_done[w], (n_pv[w] - 1) & 1, P, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              if (lane == 0) GQE_ISSUE_S(w, nxt);
-              ++n_s[w];
-            }
+          if (lane == 0) {
+            GQE_ISSUE_S(nxt);
+            if (j + 2 == nk) mma_commit(q_empty);
           }
-          if (!more) ++n_o[w];
+          __syncwarp();
         }
-        if (!ok) break;
+        if (!warp_wait(p_ready, n_p & 1, P, abort_flag)) { ok = false; break; }
+        ++n_p;
+        if (j == 0 && n_o > 0 && !warp_wait(o_free, (n_o - 1) & 1, P, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         if (lane == 0) {
-          if (j + 2 == nk) mma_commit(q_empty);  // the item's last S products are issued
+          GQE_ISSUE_PV(cur, j == 0);
+          if (!more) mma_commit(o_full);
           mma_commit(&kv_empty[cur]);
         }
+        __syncwarp();
+        ++n_pv;
+        if (!more) ++n_o;
         stage = nxt;
         kv_phase = nxt_phase;
       }
-      __syncwarp();
     }
 #undef GQE_ISSUE_S
 #undef GQE_ISSUE_PV
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int w = (warp - 2) / 4;   // query tile of this warpgroup
-    const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + w * 128;
-    const uint32_t t_p = tmem + lane_off + C::p_col(w);
-    const uint32_t t_o = tmem + lane_off + C::O_COL + w * DH;
-    uint32_t n_s = 0, n_o = 0;
+    const uint32_t t_s = tmem + lane_off;
+    const uint32_t t_p = tmem + lane_off + C::P_COL;
+    const uint32_t t_o = tmem + lane_off + C::O_COL;
+    uint32_t n_s = 0, n_o = 0;  // uses of s_full / o_full so far
     const float cs = P.scale_log2;
     for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
       const Item it = decode(P, i);
-      const int nkv = it.nkv[w];
-      if (nkv == 0) continue;
-      const int q0 = (it.pair * NWG + w) * TQ;
+      const int nkv = it.nkv;
+      const int q0 = it.qt * TQ;
       const int q = q0 + row;  // query position within the sequence
       float m_used = 0.f, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
-        if (!warp_wait(&s_full[w], n_s & 1, P, abort_flag)) { ok = false; break; }
+        if (!warp_wait(s_full, n_s & 1, P, abort_flag)) { ok = false; break; }
         ++n_s;
         tc_fence_after();
         float s[TK];
@@ -366,6 +322,12 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
           tmem_ld128_wait(t_s, r);
 #pragma unroll
           for (int c = 0; c < TK; ++c) s[c] = __uint_as_float(r[c]);
+        }
+        if (j + 1 < nkv) {
+          // S is in registers: the next S may be written.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
         }
         const int kv0 = j * TK;
         if ((P.causal && kv0 + TK - 1 > q0) || (kv0 + TK > P.T)) {
@@ -394,16 +356,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
           alpha = fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        // With separate P buffers, S_w(j) was issued without waiting for P_w(j-1) V: wait
-        // for that product before overwriting P_w or rescaling O_w.
-        if (C::SEP_P && n_s > 1 &&
-            !warp_wait(&pv_done[w], (n_s - 2) & 1, P, abort_flag)) {
+        // S(j) was issued without waiting for P(j-1) V: wait for that product before
+        // overwriting P or rescaling O.
+        if (j > 0 && !warp_wait(pv_done, (n_s - 2) & 1, P, abort_flag)) {
           ok = false;
           break;
         }
         if (__any_sync(0xffffffffu, need)) {
-          // O_w holds the sum through KV tile j-1; that P V finished before S_w(j) was
-          // issued, so O_w can be rescaled in place now.
+          tc_fence_after();
 #pragma unroll
           for (int c0 = 0; c0 < DH; c0 += 16) {
             uint32_t r[16];
@@ -415,7 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
           l *= alpha;
         }
         // p = exp2(s * scale - m): packed FMA for the argument, MUFU ex2, four packed
-        // partial sums; P goes back over the first 64 columns of S_w as bf16 pairs.
+        // partial sums; P goes to TMEM as bf16 pairs.
         const float2 cs2 = make_float2(cs, cs);
         const float2 nm2 = make_float2(-m_used, -m_used);
         float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -439,11 +399,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[w]);
+        if (lane == 0) mbar_arrive(p_ready);
       }
       if (!ok) break;
-      // ---- epilogue: O_w / l into Z
-      if (!warp_wait(&o_full[w], n_o & 1, P, abort_flag)) break;
+      // ---- epilogue: O / l into Z
+      if (!warp_wait(o_full, n_o & 1, P, abort_flag)) break;
       ++n_o;
       tc_fence_after();
       const bool valid = q < P.T;
@@ -477,14 +437,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_kernel(const __grid_constant_
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_free[w]);
+      if (lane == 0) mbar_arrive(o_free);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -522,12 +482,12 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
   P.weighted = weighted;
   P.causal = causal;
   P.nq = (T + TQ - 1) / TQ;
-  P.npairs = (P.nq + NWG - 1) / NWG;
-  P.items = B * S * P.npairs;
+  P.items = B * S * P.nq;
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   P.status = h->ws.status;
   P.spin = h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22;
-  const int grid = P.items < h->num_sms ? P.items : h->num_sms;
+  const int slots = C::CTAS * h->num_sms;
+  const int grid = P.items < slots ? P.items : slots;
   attn_kernel<DH><<<grid, THREADS, C::SMEM, st>>>(P);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }

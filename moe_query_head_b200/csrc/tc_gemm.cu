@@ -159,21 +159,35 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     // ------------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
+    // Gather mode: lane l loads tile rows 4l .. 4l+3. Their source token rows come from
+    // the bucket (rows past the tile's end repeat its first row: computed, never stored).
+    // The next tile's rows are fetched while this tile's stages are issued, and its list
+    // entry one tile earlier still, so no dependent global load waits at a tile boundary.
+    auto fetch_rows = [&](int2 t, int (&rows)[4]) {
+      const int n = min(BM, P.offsets[t.x + 1] - t.y);
+      const int first = P.bucket[t.y] >> 3;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        rows[i] = r < n ? (P.bucket[t.y + r] >> 3) : first;
+      }
+    };
+    int g_rows[4] = {0, 0, 0, 0};
+    int2 tl_next = make_int2(0, 0);
+    if constexpr (GATHER) {
+      if (blockIdx.x < total) fetch_rows(P.tile_list[blockIdx.x], g_rows);
+      if (blockIdx.x + gridDim.x < total) tl_next = P.tile_list[blockIdx.x + gridDim.x];
+    }
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
       const TileInfo ti = tile_info<GATHER>(P, tile);
       const int brow = GATHER ? ti.p * P.d_h : ti.n0;
       const int tb = GATHER ? 0 : ti.p;
       const uint32_t b_bytes = (uint32_t)P.prob[GATHER ? 0 : ti.p].box_n * BK * 2;
-      // gather mode: lane l loads tile rows 4l .. 4l+3; their source token rows (rows past
-      // the tile's end repeat its first row: they are computed and never stored)
-      int g_rows[4] = {0, 0, 0, 0};
+      int rows_next[4] = {0, 0, 0, 0};
+      int2 tl_after = make_int2(0, 0);
       if constexpr (GATHER) {
-        const int first = P.bucket[ti.m0] >> 3;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 4 * lane + i;
-          g_rows[i] = r < ti.rows ? (P.bucket[ti.m0 + r] >> 3) : first;
-        }
+        if (tile + gridDim.x < total) fetch_rows(tl_next, rows_next);
+        if (tile + 2 * gridDim.x < total) tl_after = P.tile_list[tile + 2 * gridDim.x];
       }
       for (int kb = 0; kb < KB; ++kb) {
         bool ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
@@ -199,6 +213,11 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
           phase ^= 1;
         }
       }
+      if constexpr (GATHER) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) g_rows[i] = rows_next[i];
+        tl_next = tl_after;
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -208,7 +227,14 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     uint32_t phase = 0;
     int it = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
-      const TileInfo ti = tile_info<GATHER>(P, tile);
+      // Only the MMA width is needed here: constant for the routed projection, so no
+      // tile-list load sits on this warp's path.
+      int n_mma;
+      if constexpr (GATHER) {
+        n_mma = P.prob[0].box_n;
+      } else {
+        n_mma = tile_info<false>(P, tile).n;
+      }
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       bool ok = true;
@@ -220,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
-      const uint32_t idesc = idesc_bf16_f32(BM, ti.n);
+      const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
       for (int kb = 0; kb < KB; ++kb) {
         ok = mbar_wait(&full[stage], phase, P.spin);
         ok = !__any_sync(0xffffffffu, !ok);
@@ -257,6 +283,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       const TileInfo ti = tile_info<GATHER>(P, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      const bool valid = row < ti.rows;
+      // gather mode: this row's bucket entry, loaded before the wait
+      const int ent = (GATHER && valid) ? P.bucket[ti.m0 + row] : 0;
       bool ok = true;
       ok = mbar_wait(&acc_full[acc], acc_phase, P.spin);
       ok = !__any_sync(0xffffffffu, !ok);
@@ -266,11 +295,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      const bool valid = row < ti.rows;
       if constexpr (GATHER) {
         __nv_bfloat16* dst = nullptr;
         if (valid) {
-          const int ent = P.bucket[ti.m0 + row];
           const int g = ti.p / P.E;
           const int64_t s = (int64_t)g * P.k + (ent & 7);
           dst = P.Q + (s * P.M + (ent >> 3)) * P.d_h;
