@@ -62,6 +62,24 @@ def parse_args():
     return a
 
 
+def attention_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu capture, if that capture was
+    taken on this workload and on the current attention source; else None."""
+    import hashlib
+    rec_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    src = os.path.join(ROOT, "moe_query_head_b200", "csrc", "tc_attention.cu")
+    try:
+        with open(rec_path) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if rec.get("source_sha256") != sha or rec.get("workload") != workload:
+        return None
+    return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -345,7 +363,9 @@ def bench_ours(args, rank, world, dist):
                       for i in range(G.GQE_NUM_STAGES)},
         "roofline": {"kernel": "attention", "bound": "tensor", "achieved": att_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
-                     "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": None},
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "traffic": attention_traffic(wl.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": {"value": tokens / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size() + 4)},
