@@ -64,6 +64,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.bucket = (int32_t*)take((size_t)M * Gk * 4);
   w.tile_list = (int2*)take((size_t)((M * Gk + 127) / 128 + N + 1) * sizeof(int2));
   w.tile_count = (int32_t*)take(16);
+  w.attn_counter = (int32_t*)take(16);
   w.status = (int32_t*)take(16);
   w.wcat = take((size_t)(N + (2 * G + 1) * d_h) * dim * esz);
   (void)dim;

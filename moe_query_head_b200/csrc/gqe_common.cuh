@@ -63,6 +63,7 @@ struct Workspace {
   int32_t* bucket = nullptr;       // [M * G * k] entries (token << 3) | rank, per expert
   int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
+  int32_t* attn_counter = nullptr; // attention work-item counter
   int32_t* status = nullptr;       // device status word
   void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
   void* base = nullptr;            // the single allocation

@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
+#include "exp2_fma.cuh"
 #include "tc_ptx.cuh"
 
 namespace gqe {
@@ -71,6 +72,7 @@ struct Params {
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
   int nq, items;
   float scale_log2;
+  int* next_item;  // global item counter (zero at launch); CTAs take items from it
   int32_t* status;
   int64_t spin;
 };
@@ -127,7 +129,10 @@ attn_kernel(const __grid_constant__ Params P) {
   uint64_t* pv_done = p_ready + 1;
   uint64_t* o_full = pv_done + 1;
   uint64_t* o_free = o_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_free + 1);
+  uint64_t* item_full = o_free + 1;   // [2] item ring, filled by the TMA warp
+  uint64_t* item_empty = item_full + 2;  // [2] read by the MMA warp and the softmax warps
+  volatile int* item_ring = reinterpret_cast<volatile int*>(item_empty + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(item_empty + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -144,6 +149,10 @@ attn_kernel(const __grid_constant__ Params P) {
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(o_free, 4);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&item_full[r], 1);
+      mbar_init(&item_empty[r], 5);  // the MMA warp and the four softmax warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -161,12 +170,43 @@ attn_kernel(const __grid_constant__ Params P) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // MMA and softmax warps: the next item index from the ring (warp-collective); the slot
+  // is released as soon as it has been read. -1 means no work is left.
+  auto next_item = [&](int& i, int& islot, uint32_t& iphase) -> bool {
+    if (!warp_wait(&item_full[islot], iphase, P, abort_flag)) return false;
+    i = item_ring[islot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[islot]);
+    if (++islot == 2) {
+      islot = 0;
+      iphase ^= 1;
+    }
+    return true;
+  };
+
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA loads
     if (lane == 0) {
       int stage = 0;
       uint32_t kv_phase = 0, q_phase = 0;
-      for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
+      int islot = 0;
+      uint32_t iphase = 0;
+      while (!*abort_flag) {
+        // claim the next item (heaviest first) and publish it to the other warps
+        if (!mbar_wait(&item_empty[islot], iphase ^ 1, P.spin)) {
+          *abort_flag = 1;
+          atomicExch(P.status, kStatusTimeout);
+          break;
+        }
+        int i = atomicAdd(P.next_item, 1);
+        if (i >= P.items) i = -1;
+        item_ring[islot] = i;
+        mbar_arrive(&item_full[islot]);
+        if (++islot == 2) {
+          islot = 0;
+          iphase ^= 1;
+        }
+        if (i < 0) break;
         const Item it = decode(P, i);
         if (!mbar_wait(q_empty, q_phase ^ 1, P.spin)) {
           *abort_flag = 1;
@@ -241,7 +281,12 @@ attn_kernel(const __grid_constant__ Params P) {
     mma_commit(pv_done);                                                                     \
   } while (0)
 
-    for (int i = blockIdx.x; i < P.items && ok && !*abort_flag; i += gridDim.x) {
+    int islot = 0;
+    uint32_t iphase = 0;
+    while (ok && !*abort_flag) {
+      int i;
+      if (!next_item(i, islot, iphase)) break;
+      if (i < 0) break;
       const Item it = decode(P, i);
       const int nk = it.nkv;
       if (!warp_wait(q_full, q_phase, P, abort_flag)) break;
@@ -305,7 +350,12 @@ attn_kernel(const __grid_constant__ Params P) {
     const uint32_t t_o = tmem + lane_off + C::O_COL;
     uint32_t n_s = 0, n_o = 0;  // uses of s_full / o_full so far
     const float cs = P.scale_log2;
-    for (int i = blockIdx.x; i < P.items && !*abort_flag; i += gridDim.x) {
+    int islot = 0;
+    uint32_t iphase = 0;
+    while (!*abort_flag) {
+      int i;
+      if (!next_item(i, islot, iphase)) break;
+      if (i < 0) break;
       const Item it = decode(P, i);
       const int nkv = it.nkv;
       const int q0 = it.qt * TQ;
@@ -337,14 +387,19 @@ attn_kernel(const __grid_constant__ Params P) {
           for (int c = 0; c < TK; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
         }
-        // row maximum: eight independent chains, then a tree
+        // row maximum: eight independent chains of three-input max, then a tree
         float mp[8];
+        static_assert(TK == 128, "the row-maximum schedule covers 128 columns");
 #pragma unroll
-        for (int x = 0; x < 8; ++x) mp[x] = s[x];
+        for (int x = 0; x < 8; ++x) mp[x] = fmax3(s[x], s[8 + x], s[16 + x]);        // 0..23
 #pragma unroll
-        for (int c = 8; c < TK; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        for (int c = 24; c < 120; c += 16)                                          // 24..119
+#pragma unroll
+          for (int x = 0; x < 8; ++x) mp[x] = fmax3(mp[x], s[c + x], s[c + 8 + x]);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mp[x] = fmaxf(mp[x], s[120 + x]);               // 120..127
+        const float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]),
+                               fmax3(fmax3(mp[3], mp[4], mp[5]), mp[6], mp[7]));
         float m_new = mx * cs;
         if (m_new == -INFINITY) m_new = 0.f;  // a row with every key masked
         bool need = false;
@@ -386,7 +441,9 @@ attn_kernel(const __grid_constant__ Params P) {
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
             const float2 t = fma2(make_float2(s[c0 + 2 * x], s[c0 + 2 * x + 1]), cs2, nm2);
-            const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            // one pair in four on the FMA pipe, the rest on MUFU
+            const float2 p = (x & 3) == 3 ? exp2_fma2(t)
+                                          : make_float2(fast_exp2(t.x), fast_exp2(t.y));
             lsum[x & 3] = add2(lsum[x & 3], p);
             pk[x] = pack_bf16x2(p.x, p.y);
           }
@@ -488,6 +545,8 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
   P.spin = h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22;
   const int slots = C::CTAS * h->num_sms;
   const int grid = P.items < slots ? P.items : slots;
+  P.next_item = h->ws.attn_counter;
+  if (cudaMemsetAsync(h->ws.attn_counter, 0, sizeof(int), st) != cudaSuccess) return -1;
   attn_kernel<DH><<<grid, THREADS, C::SMEM, st>>>(P);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }

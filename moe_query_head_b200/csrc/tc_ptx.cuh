@@ -199,6 +199,13 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
       : "memory");
 }
 
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Packed two-lane fp32 arithmetic (sm_100).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   uint64_t d;

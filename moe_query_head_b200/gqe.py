@@ -23,7 +23,7 @@ TENSORS = {"K": 0, "V": 1, "Q": 2, "Z": 3, "PSEL": 4, "W": 5, "LOGITS": 6}
 EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
-            "gqe_stage_name", "gqe_route_static")
+            "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma")
 GQE_NUM_STAGES = 8
 
 
@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     lib.gqe_stage_name.restype = ctypes.c_char_p
     lib.gqe_route_static.argtypes = [P, I, I, I, I, P, P, P, P, P, P]
     lib.gqe_route_static.restype = I
+    lib.gqe_exp2_fma.argtypes = [P, P, I, P]
+    lib.gqe_exp2_fma.restype = I
     return lib
 
 
@@ -139,6 +141,11 @@ def gqe_route_static(logits, M, N, G, k, sel, gates, counts, mean_prob, aux_loss
     _check(lib.gqe_route_static(_ptr(logits), M, N, G, k, _ptr(sel), _ptr(gates), _ptr(counts),
                                 _ptr(mean_prob), _ptr(aux_loss), _stream(stream)),
            "gqe_route_static")
+
+
+def gqe_exp2_fma(inp, out, stream=None) -> None:
+    """Diagnostic: the softmax's FMA-pipe exp2, elementwise (float32 device tensors)."""
+    _check(lib.gqe_exp2_fma(_ptr(inp), _ptr(out), inp.numel(), _stream(stream)), "gqe_exp2_fma")
 
 
 def gqe_stage_name(i: int):
