@@ -10,11 +10,12 @@
 //                     Overview: only the active query-head computation is reduced).
 //   output projection Z [M, D_o] times W_o [dim, D_o].
 //
-// One persistent kernel, one CTA per SM, 6 warps:
-//   warp 0     producer: TMA tile loads of A (or, for the routed projection, cp.async
-//              gathers of A rows written in the 128-byte swizzled layout) and of B;
-//   warp 1     allocates TMEM; one lane issues tcgen05.mma (128 x BN x 16) and commits;
-//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator, conversion, stores.
+// One persistent kernel, one CTA per SM:
+//   producers  dense: one warp issuing TMA tile loads of A and B. Routed projection: four
+//              warps gathering A rows through registers into the 128-byte swizzled
+//              layout (each warp fills every fourth stage), B by TMA;
+//   MMA warp   allocates TMEM; one lane issues tcgen05.mma (128 x BN x 16) and commits;
+//   4 warps    epilogue: tcgen05.ld of the fp32 accumulator, conversion, stores.
 // Shared-memory stages are guarded by full/empty mbarriers; two TMEM accumulators let the
 // epilogue of one tile overlap the MMAs of the next.
 #include <cudaTypedefs.h>
@@ -34,7 +35,14 @@ constexpr int BM = 128;        // tile rows = MMA M = TMEM lanes
 constexpr int BN = 128;        // widest tile (MMA N)
 constexpr int BK = 64;         // one 128-byte swizzle atom of bf16 along K
 constexpr int STAGES = 6;
-constexpr int THREADS = 192;
+// Warp roles: producers, one MMA-issuing warp, four epilogue warps.
+template <bool GATHER>
+struct Lay {
+  static constexpr int NPROD = GATHER ? 4 : 1;
+  static constexpr int MMA = NPROD;
+  static constexpr int EPI0 = NPROD + 1;
+  static constexpr int THREADS = (NPROD + 5) * 32;
+};
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int B_STAGE_BYTES = BN * BK * 2;
 constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256 +
@@ -113,7 +121,9 @@ __device__ __forceinline__ void set_timeout(const Params& P, volatile int* abort
 }
 
 template <bool GATHER>
-__global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(Lay<GATHER>::THREADS, 1)
+tc_gemm_kernel(const __grid_constant__ Params P) {
+  using L = Lay<GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -131,7 +141,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], GATHER ? 2 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -141,7 +151,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == L::MMA) {
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
@@ -155,71 +165,96 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
   const uint32_t tmem_base = *tmem_holder;
   const int KB = (P.K + BK - 1) / BK;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    // Gather mode: lane l loads tile rows 4l .. 4l+3. Their source token rows come from
-    // the bucket (rows past the tile's end repeat its first row: computed, never stored).
-    // The next tile's rows are fetched while this tile's stages are issued, and its list
-    // entry one tile earlier still, so no dependent global load waits at a tile boundary.
-    auto fetch_rows = [&](int2 t, int (&rows)[4]) {
-      const int n = min(BM, P.offsets[t.x + 1] - t.y);
-      const int first = P.bucket[t.y] >> 3;
+  if (warp < L::NPROD) {
+    // ------------------------------------------------------------------ producers
+    if constexpr (!GATHER) {
+      // One lane issues TMA tile loads of A and B.
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        const TileInfo ti = tile_info<false>(P, tile);
+        const uint32_t b_bytes = (uint32_t)P.prob[ti.p].box_n * BK * 2;
+        for (int kb = 0; kb < KB; ++kb) {
+          bool ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
+          ok = !__any_sync(0xffffffffu, !ok);
+          if (!ok) {
+            if (lane == 0) set_timeout(P, abort_flag);
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], (uint32_t)A_STAGE_BYTES + b_bytes);
+            tma_load_2d(sA + stage * A_STAGE_BYTES, &P.tmap_a, kb * BK, ti.m0, &full[stage]);
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[ti.p], kb * BK, ti.n0, &full[stage]);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    } else {
+      // Four producer warps; warp p fills every fourth stage of the CTA's stage sequence.
+      // A rows are gathered through registers: lane l moves 16-byte chunk l % 8 of rows
+      // 4 i + l / 8 (eight lanes per 128-byte row segment: coalesced loads, conflict-free
+      // stores into the 128-byte-swizzled slot). B (the expert's W_q rows) comes by TMA.
+      // The stage's full barrier takes two arrivals: the TMA's and this warp's.
+      const int pw = warp;
+      const int c = lane & 7;
+      uint32_t g = 0;  // position in the CTA's stage sequence
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        const int2 t = P.tile_list[tile];
+        const int n = min(BM, P.offsets[t.x + 1] - t.y);
+        const uint32_t b_bytes = (uint32_t)P.prob[0].box_n * BK * 2;
+        // source rows of this lane: r = 4 i + lane / 8 (rows past the tile's end repeat
+        // its first row: computed, never stored)
+        int src[BM / 4];
+        const int first = P.bucket[t.y] >> 3;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * lane + i;
-        rows[i] = r < n ? (P.bucket[t.y + r] >> 3) : first;
-      }
-    };
-    int g_rows[4] = {0, 0, 0, 0};
-    int2 tl_next = make_int2(0, 0);
-    if constexpr (GATHER) {
-      if (blockIdx.x < total) fetch_rows(P.tile_list[blockIdx.x], g_rows);
-      if (blockIdx.x + gridDim.x < total) tl_next = P.tile_list[blockIdx.x + gridDim.x];
-    }
-    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-      const TileInfo ti = tile_info<GATHER>(P, tile);
-      const int brow = GATHER ? ti.p * P.d_h : ti.n0;
-      const int tb = GATHER ? 0 : ti.p;
-      const uint32_t b_bytes = (uint32_t)P.prob[GATHER ? 0 : ti.p].box_n * BK * 2;
-      int rows_next[4] = {0, 0, 0, 0};
-      int2 tl_after = make_int2(0, 0);
-      if constexpr (GATHER) {
-        if (tile + gridDim.x < total) fetch_rows(tl_next, rows_next);
-        if (tile + 2 * gridDim.x < total) tl_after = P.tile_list[tile + 2 * gridDim.x];
-      }
-      for (int kb = 0; kb < KB; ++kb) {
-        bool ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
-        ok = !__any_sync(0xffffffffu, !ok);
-        if (!ok) {
-          if (lane == 0) set_timeout(P, abort_flag);
-          break;
+        for (int i = 0; i < BM / 4; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          src[i] = r < n ? (P.bucket[t.y + r] >> 3) : first;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], (uint32_t)A_STAGE_BYTES + b_bytes);
-          if (!GATHER) tma_load_2d(sA + stage * A_STAGE_BYTES, &P.tmap_a, kb * BK, ti.m0, &full[stage]);
-          tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[tb], kb * BK, brow, &full[stage]);
-        }
-        if constexpr (GATHER) {
-          // TMA row gather: four 128-byte row segments per lane into rows 4l .. 4l+3 of
-          // the 128-byte-swizzled A tile (the swizzle follows the destination address).
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          if ((int)(g % L::NPROD) != pw) continue;
+          const int stage = (int)(g % STAGES);
+          const uint32_t phase = (g / STAGES) & 1;
+          ok = !__any_sync(0xffffffffu, !mbar_wait(&empty[stage], phase ^ 1, P.spin));
+          if (!ok) {
+            if (lane == 0) set_timeout(P, abort_flag);
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], b_bytes);
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, t.x * P.d_h,
+                        &full[stage]);
+          }
+          uint8_t* dst = sA + stage * A_STAGE_BYTES;
+          const int kcol = kb * BK + c * 8;
+          const bool kok = kcol < P.K;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 v[BM / 8];
+#pragma unroll
+            for (int i = 0; i < BM / 8; ++i) {
+              const int ii = h * (BM / 8) + i;
+              v[i] = kok ? __ldg(reinterpret_cast<const uint4*>(P.x + (int64_t)src[ii] * P.K + kcol))
+                         : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < BM / 8; ++i) {
+              const int r = 4 * (h * (BM / 8) + i) + (lane >> 3);
+              *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = v[i];
+            }
+          }
+          fence_async_shared();  // these generic-proxy stores before the tensor core reads
           __syncwarp();
-          tma_gather4(sA + stage * A_STAGE_BYTES + lane * 4 * 128, &P.tmap_a, kb * BK,
-                      g_rows[0], g_rows[1], g_rows[2], g_rows[3], &full[stage]);
+          if (lane == 0) mbar_arrive(&full[stage]);
         }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if constexpr (GATHER) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) g_rows[i] = rows_next[i];
-        tl_next = tl_after;
+        if (!ok) break;
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == L::MMA) {
     // ------------------------------------------------------------------ MMA issuer
     const uint64_t a_desc0 = smem_desc(smem_u32(sA), 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(sB), 1024, kSwizzle128B);
@@ -367,7 +402,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_gemm_kernel(const __grid_consta
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == L::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -442,7 +477,7 @@ int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
       return -1;
     configured[GATHER] = true;
   }
-  tc_gemm_kernel<GATHER><<<grid, THREADS, SMEM_BYTES, st>>>(P);
+  tc_gemm_kernel<GATHER><<<grid, Lay<GATHER>::THREADS, SMEM_BYTES, st>>>(P);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
