@@ -14,7 +14,9 @@
 //   warp 1     owns 256 TMEM columns; one lane issues S = Q K^T (A and B from shared
 //              memory) into TMEM and O += P V with P read from TMEM (the TS form) and V as
 //              an MN-major shared-memory operand;
-//   warps 2-5  softmax: one query row per thread, 128 scores per KV tile in registers,
+//   warps 2-3  idle: with two CTAs per SM the launch gives every thread 128 registers;
+//              warps 0-3 drop to 48 (setmaxnreg) so that the softmax warpgroup can take 208;
+//   warps 4-7  softmax: one query row per thread, 128 scores per KV tile in registers,
 //              exp2 against the running row maximum, P written to TMEM as bf16 pairs. O is
 //              rescaled in TMEM only when a row maximum grows by more than 2^8 (rare after
 //              the first tiles). At the end of an item the same warps normalise O by the
@@ -39,7 +41,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int THREADS = 192;
+// Warps: 0 TMA, 1 MMA, 2-3 idle (they only hand their registers to the softmax
+// warpgroup), 4-7 softmax + epilogue.
+constexpr int THREADS = 256;
+constexpr int kSmallRegs = 48;   // warpgroup 0 after setmaxnreg.dec (two CTAs per SM)
+constexpr int kLargeRegs = 208;  // softmax warpgroup after setmaxnreg.inc
 constexpr int TQ = 128;                    // queries per tile (MMA M, TMEM lanes)
 constexpr int TK = 128;                    // keys per tile (S MMA N)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -184,6 +190,13 @@ attn_kernel(const __grid_constant__ Params P) {
     return true;
   };
 
+  // Two CTAs per SM launch with 128 registers per thread; warpgroup 0 (TMA, MMA and two
+  // idle warps) gives most of its share to the softmax warpgroup. The two counts add up
+  // to the launch allocation exactly: 48 * 128 + 208 * 128 = 256 * 128.
+  static_assert(kSmallRegs * 128 + kLargeRegs * 128 == THREADS * (65536 / (2 * THREADS)),
+                "register split must equal the launch allocation");
+  if (warp < 4) {
+  if constexpr (C::CTAS == 2) setmaxnreg_dec<kSmallRegs>();
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA loads
     if (lane == 0) {
@@ -340,8 +353,10 @@ attn_kernel(const __grid_constant__ Params P) {
     }
 #undef GQE_ISSUE_S
 #undef GQE_ISSUE_PV
+  }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
+    if constexpr (C::CTAS == 2) setmaxnreg_inc<kLargeRegs>();
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
