@@ -10,21 +10,24 @@
 // items heaviest first (causal tiles near the end of a sequence have the most keys). The
 // two CTAs of an SM interleave: while one computes exponentials the other's products run,
 // and each hides the other's waits. Per CTA:
-//   warp 0     TMA: the Q tile once per item, then K and V tiles into a ring of stages;
-//   warp 1     owns 256 TMEM columns; one lane issues S = Q K^T (A and B from shared
-//              memory) into TMEM and O += P V with P read from TMEM (the TS form) and V as
-//              an MN-major shared-memory operand;
-//   warps 2-3  idle: with two CTAs per SM the launch gives every thread 128 registers;
+//   warp 0     TMA: the Q tile once per item, then K tiles into their own ring;
+//   warp 1     owns the TMEM columns; one elected lane issues S = Q K^T (A and B from
+//              shared memory) into TMEM and O += P V with P read from TMEM (the TS form)
+//              and V as an MN-major shared-memory operand;
+//   warp 2     TMA: V tiles into a second ring (a K tile is released as soon as its S is
+//              done, so K runs ahead of the V tiles that the later P V products still hold);
+//   warp 3     idle. With two CTAs per SM the launch gives every thread 128 registers;
 //              warps 0-3 drop to 48 (setmaxnreg) so that the softmax warpgroup can take 208;
 //   warps 4-7  softmax: one query row per thread, 128 scores per KV tile in registers,
-//              exp2 against the running row maximum, P written to TMEM as bf16 pairs. O is
-//              rescaled in TMEM only when a row maximum grows by more than 2^8 (rare after
-//              the first tiles). At the end of an item the same warps normalise O by the
-//              row sum, apply the weighted_concat scale if any, and store the row into its
-//              block of Z.
-// P has TMEM columns of its own: as soon as the softmax warps have pulled S(j) into
-// registers, S(j+1) is computed, so it is ready when they finish tile j. (Head dims above 64
-// run one CTA per SM with 512 TMEM columns; the shared memory of two would not fit.)
+//              exp2 against the running row maximum, P kept in registers as bf16 pairs until
+//              the tile is done, then written to TMEM. O is rescaled in TMEM only when a row
+//              maximum grows by more than 2^8 (rare after the first tiles). At the end of an
+//              item the same warps normalise O by the row sum, apply the weighted_concat
+//              scale if any, and store the row into its block of Z.
+// P has TMEM columns of its own. S runs a tile ahead of the softmax warps: S(j+2) is issued
+// as soon as they hold S(j+1) in registers, before P(j) V, which they need only before they
+// write P(j+1). For head dims up to 48 the row sums come from the tensor core (a chunk of
+// ones after every V tile). Head dims above 64 run one CTA per SM with 512 TMEM columns.
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
@@ -41,7 +44,7 @@ namespace {
 
 using namespace tc;
 
-// Warps: 0 TMA, 1 MMA, 2-3 idle (they only hand their registers to the softmax
+// Warps: 0 Q/K loads, 1 MMA, 2 V loads, 3 idle (it only hands its registers to the softmax
 // warpgroup), 4-7 softmax + epilogue.
 constexpr int THREADS = 256;
 constexpr int kSmallRegs = 48;   // warpgroup 0 after setmaxnreg.dec (two CTAs per SM)
@@ -59,17 +62,34 @@ struct Cfg {
   static constexpr int ROW_BYTES = CW * 2;          // bytes per row inside a chunk
   static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;
   static constexpr int TILE_BYTES = 128 * DH * 2;   // one Q, K or V tile
+  // Small head dims let the tensor core form the softmax row sums: every V tile is
+  // followed by a constant chunk of ones, so O += P [V | 1] leaves sum_j P in the columns
+  // after the head dim (from the same bf16 P the product uses). Larger head dims keep the
+  // sums in registers (their products are already the larger cost).
+  static constexpr bool SUM_MMA = DH <= 48;
+  static constexpr int ONES_BYTES = SUM_MMA ? CHUNK_BYTES : 0;
+  static constexpr int N_PV = DH + (SUM_MMA ? 16 : 0);  // PV MMA width
+  static constexpr int V_BYTES = TILE_BYTES + ONES_BYTES;  // one V stage
   // Two CTAs per SM while both fit (TMEM 256 columns each, shared memory), else one.
   static constexpr int CTAS = DH <= 64 ? 2 : 1;
   static constexpr int TMEM_COLS = CTAS == 2 ? 256 : 512;
-  static constexpr int STAGES = DH <= 48 ? 4 : (DH <= 64 ? 2 : (DH <= 96 ? 3 : 2));
-  static constexpr int SMEM = TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
+  // Separate K and V rings: a K tile is released as soon as its S product is done, so K
+  // runs several tiles ahead of the V tiles that the later P V products hold.
+  static constexpr int K_STAGES = DH <= 48 ? 4 : 3;
+  static constexpr int V_STAGES = DH == 64 ? 2 : 3;
+  static constexpr int SMEM = TILE_BYTES * (1 + K_STAGES) + V_STAGES * V_BYTES + 1024 + 256;
   // TMEM columns: S at 0, P (bf16 pairs) at 128, O at 192.
   static constexpr int P_COL = 128;
   static constexpr int O_COL = 192;
-  static_assert(O_COL + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL + N_PV <= TMEM_COLS, "TMEM budget");
   static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory budget");
 };
+// Exponentials: of every 8 pairs of scores, this many go to the FMA-pipe polynomial and
+// the rest to the MUFU unit (16 results per SM per clock on B200).
+#ifndef GQE_ATTN_FMA_PAIRS_OF_8
+#define GQE_ATTN_FMA_PAIRS_OF_8 2
+#endif
+constexpr int kFmaPairsOf8 = GQE_ATTN_FMA_PAIRS_OF_8;
 
 struct Params {
   CUtensorMap tm_q, tm_k, tm_v;
@@ -123,31 +143,48 @@ attn_kernel(const __grid_constant__ Params P) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::TILE_BYTES;  // per stage: K tile, V tile
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sKV + C::STAGES * 2 * C::TILE_BYTES);
+  uint8_t* sK = smem + C::TILE_BYTES;                 // K ring
+  uint8_t* sV = sK + C::K_STAGES * C::TILE_BYTES;     // V ring: V tile[, ones chunk]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sV + C::V_STAGES * C::V_BYTES);
   uint64_t* q_full = bar;
   uint64_t* q_empty = bar + 1;
-  uint64_t* kv_full = bar + 2;
-  uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;
+  uint64_t* k_full = bar + 2;
+  uint64_t* k_empty = k_full + C::K_STAGES;
+  uint64_t* v_full = k_empty + C::K_STAGES;
+  uint64_t* v_empty = v_full + C::V_STAGES;
+  uint64_t* s_full = v_empty + C::V_STAGES;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_ready = s_free + 1;
   uint64_t* pv_done = p_ready + 1;
   uint64_t* o_full = pv_done + 1;
   uint64_t* o_free = o_full + 1;
-  uint64_t* item_full = o_free + 1;   // [2] item ring, filled by the TMA warp
-  uint64_t* item_empty = item_full + 2;  // [2] read by the MMA warp and the softmax warps
+  uint64_t* item_full = o_free + 1;   // [2] item ring, filled by the K/Q load warp
+  uint64_t* item_empty = item_full + 2;  // [2] read by the V load, MMA and softmax warps
   volatile int* item_ring = reinterpret_cast<volatile int*>(item_empty + 2);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(item_empty + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if constexpr (C::SUM_MMA) {
+    // the constant ones chunk after every stage's V tile (bf16 1.0 in every element, so
+    // the swizzle does not matter); TMA never writes it
+    for (int st = 0; st < C::V_STAGES; ++st) {
+      uint4* o = reinterpret_cast<uint4*>(sV + st * C::V_BYTES + C::TILE_BYTES);
+      for (int i = threadIdx.x; i < C::ONES_BYTES / 16; i += THREADS)
+        o[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    }
+    fence_async_shared();
+  }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < C::K_STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < C::V_STAGES; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
@@ -157,7 +194,7 @@ attn_kernel(const __grid_constant__ Params P) {
     mbar_init(o_free, 4);
     for (int r = 0; r < 2; ++r) {
       mbar_init(&item_full[r], 1);
-      mbar_init(&item_empty[r], 5);  // the MMA warp and the four softmax warps
+      mbar_init(&item_empty[r], 6);  // the V load warp, the MMA warp, four softmax warps
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -198,10 +235,10 @@ attn_kernel(const __grid_constant__ Params P) {
   if (warp < 4) {
   if constexpr (C::CTAS == 2) setmaxnreg_dec<kSmallRegs>();
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA loads
+    // ---------------------------------------------------------------- Q and K loads
     if (lane == 0) {
-      int stage = 0;
-      uint32_t kv_phase = 0, q_phase = 0;
+      int kst = 0;
+      uint32_t k_phase = 0, q_phase = 0;
       int islot = 0;
       uint32_t iphase = 0;
       while (!*abort_flag) {
@@ -235,23 +272,60 @@ attn_kernel(const __grid_constant__ Params P) {
         const int kvh = it.s < P.Sr ? it.s / P.k : 0;
         const int krow0 = kvh * P.M + it.b * P.T;
         for (int j = 0; j < it.nkv; ++j) {
-          if (!mbar_wait(&kv_empty[stage], kv_phase ^ 1, P.spin)) {
+          if (!mbar_wait(&k_empty[kst], k_phase ^ 1, P.spin)) {
             *abort_flag = 1;
             atomicExch(P.status, kStatusTimeout);
             break;
           }
-          mbar_arrive_expect_tx(&kv_full[stage], 2 * C::TILE_BYTES);
-          uint8_t* sK = sKV + stage * 2 * C::TILE_BYTES;
+          mbar_arrive_expect_tx(&k_full[kst], C::TILE_BYTES);
 #pragma unroll
-          for (int c = 0; c < C::NC; ++c) {
-            tma_load_2d(sK + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW, krow0 + j * TK,
-                        &kv_full[stage]);
-            tma_load_2d(sK + C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW,
-                        krow0 + j * TK, &kv_full[stage]);
+          for (int c = 0; c < C::NC; ++c)
+            tma_load_2d(sK + kst * C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW,
+                        krow0 + j * TK, &k_full[kst]);
+          if (++kst == C::K_STAGES) {
+            kst = 0;
+            k_phase ^= 1;
           }
-          if (++stage == C::STAGES) {
-            stage = 0;
-            kv_phase ^= 1;
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- V loads
+    if (lane == 0) {
+      int vst = 0;
+      uint32_t v_phase = 0;
+      int islot = 0;
+      uint32_t iphase = 0;
+      while (!*abort_flag) {
+        if (!mbar_wait(&item_full[islot], iphase, P.spin)) {
+          *abort_flag = 1;
+          atomicExch(P.status, kStatusTimeout);
+          break;
+        }
+        const int i = item_ring[islot];
+        mbar_arrive(&item_empty[islot]);
+        if (++islot == 2) {
+          islot = 0;
+          iphase ^= 1;
+        }
+        if (i < 0) break;
+        const Item it = decode(P, i);
+        const int kvh = it.s < P.Sr ? it.s / P.k : 0;
+        const int krow0 = kvh * P.M + it.b * P.T;
+        for (int j = 0; j < it.nkv; ++j) {
+          if (!mbar_wait(&v_empty[vst], v_phase ^ 1, P.spin)) {
+            *abort_flag = 1;
+            atomicExch(P.status, kStatusTimeout);
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[vst], C::TILE_BYTES);
+#pragma unroll
+          for (int c = 0; c < C::NC; ++c)
+            tma_load_2d(sV + vst * C::V_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW,
+                        krow0 + j * TK, &v_full[vst]);
+          if (++vst == C::V_STAGES) {
+            vst = 0;
+            v_phase ^= 1;
           }
         }
       }
@@ -261,39 +335,44 @@ attn_kernel(const __grid_constant__ Params P) {
     // Lean: descriptors are built once; each product's descriptor is a base plus a
     // constant (the address field is the low 14 bits, in 16-byte units).
     const uint32_t idesc_s = idesc_bf16_f32(TQ, TK);
-    const uint32_t idesc_pv = idesc_bf16_f32(TQ, DH) | (1u << 16);  // B (V) MN-major
+    const uint32_t idesc_pv = idesc_bf16_f32(TQ, C::N_PV) | (1u << 16);  // B (V) MN-major
     const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
-    const uint64_t k_desc = smem_desc(smem_u32(sKV), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t v_desc =
-        smem_desc_mn(smem_u32(sKV + C::TILE_BYTES), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
-    constexpr uint32_t kStageStep = (2 * C::TILE_BYTES) >> 4;
-    int stage = 0;
-    uint32_t kv_phase = 0, q_phase = 0;
-    uint32_t n_sf = 0, n_p = 0, n_pv = 0, n_o = 0;  // uses of s_free / p_ready / pv_done / o_full
+        smem_desc_mn(smem_u32(sV), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kKStep = C::TILE_BYTES >> 4;
+    constexpr uint32_t kVStep = C::V_BYTES >> 4;
+    int kst = 0, vst = 0;
+    uint32_t k_phase = 0, v_phase = 0, q_phase = 0;
+    uint32_t n_sf = 0, n_p = 0, n_o = 0;  // uses of s_free / p_ready / o_full
     bool ok = true;
 
-    // S = Q K^T for the K tile in stage `st` (lane 0 only).
-#define GQE_ISSUE_S(st)                                                                      \
-  do {                                                                                       \
-    const uint64_t kd = k_desc + (uint64_t)((st) * kStageStep);                              \
-    _Pragma("unroll") for (int kk = 0; kk < DH / 16; ++kk) {                                 \
-      const uint32_t o = (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4; \
-      mma_ss(tmem, q_desc + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);                           \
-    }                                                                                        \
-    mma_commit(s_full);                                                                      \
-  } while (0)
-    // O += P V for the V tile in stage `st` (lane 0 only). V is the MN-major B operand
-    // (N = head dim, K = keys): 16 keys are two 8-row groups of every chunk.
-#define GQE_ISSUE_PV(st, first)                                                              \
-  do {                                                                                       \
-    const uint64_t vd = v_desc + (uint64_t)((st) * kStageStep);                              \
-    _Pragma("unroll") for (int kk = 0; kk < TK / 16; ++kk)                                   \
-        mma_ts(tmem + C::O_COL, tmem + C::P_COL + kk * 8,                                    \
-               vd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_pv,                     \
-               ((first) && kk == 0) ? 0u : 1u);                                              \
-    mma_commit(pv_done);                                                                     \
-  } while (0)
-
+    // Order of issue per item: S(0), S(1); then for every tile j, once P(j) is ready,
+    // S(j+2) (as soon as the softmax warps hold S(j+1) in registers) and only then P(j) V.
+    // S therefore always runs a tile ahead of the softmax warps, and the products of P(j)
+    // V, which they need only before they write P(j+1), never delay the next S.
+    // S = Q K^T for the next K tile; its stage is released when the product is done.
+    auto issue_s = [&](bool last_s) -> bool {
+      if (!warp_wait(&k_full[kst], k_phase, P, abort_flag)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t kd = k_desc + (uint64_t)(kst * kKStep);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t o = (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4;
+          mma_ss(tmem, q_desc + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+        mma_commit(&k_empty[kst]);
+        if (last_s) mma_commit(q_empty);
+      }
+      __syncwarp();
+      if (++kst == C::K_STAGES) {
+        kst = 0;
+        k_phase ^= 1;
+      }
+      return true;
+    };
     int islot = 0;
     uint32_t iphase = 0;
     while (ok && !*abort_flag) {
@@ -304,55 +383,49 @@ attn_kernel(const __grid_constant__ Params P) {
       const int nk = it.nkv;
       if (!warp_wait(q_full, q_phase, P, abort_flag)) break;
       q_phase ^= 1;
-      if (!warp_wait(&kv_full[stage], kv_phase, P, abort_flag)) break;
-      tc_fence_after();
-      if (lane == 0) {
-        GQE_ISSUE_S(stage);
-        if (nk == 1) mma_commit(q_empty);
+      if (!issue_s(nk == 1)) break;  // S(0)
+      if (nk > 1) {
+        if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) break;  // S(0) is in registers
+        ++n_sf;
+        if (!issue_s(nk == 2)) break;  // S(1)
       }
-      __syncwarp();
       for (int j = 0; j < nk; ++j) {
-        const int cur = stage;
-        int nxt = stage + 1;
-        uint32_t nxt_phase = kv_phase;
-        if (nxt == C::STAGES) {
-          nxt = 0;
-          nxt_phase ^= 1;
-        }
-        const bool more = j + 1 < nk;
-        if (more) {
-          // S(j) is in the softmax registers: compute S(j+1) now.
-          if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) { ok = false; break; }
-          ++n_sf;
-          if (!warp_wait(&kv_full[nxt], nxt_phase, P, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            GQE_ISSUE_S(nxt);
-            if (j + 2 == nk) mma_commit(q_empty);
-          }
-          __syncwarp();
-        }
         if (!warp_wait(p_ready, n_p & 1, P, abort_flag)) { ok = false; break; }
         ++n_p;
+        if (j + 2 < nk) {
+          // the softmax warps take S(j+1) into registers right after P(j)
+          if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!issue_s(j + 3 == nk)) { ok = false; break; }  // S(j+2)
+        }
         if (j == 0 && n_o > 0 && !warp_wait(o_free, (n_o - 1) & 1, P, abort_flag)) {
           ok = false;
           break;
         }
+        if (!warp_wait(&v_full[vst], v_phase, P, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (lane == 0) {
-          GQE_ISSUE_PV(cur, j == 0);
-          if (!more) mma_commit(o_full);
-          mma_commit(&kv_empty[cur]);
+        const bool last = j + 1 == nk;
+        if (elect_one()) {
+          // O += P V (V: the MN-major B operand, N = head dim[+ ones], K = keys; 16 keys
+          // are two 8-row groups of every chunk)
+          const uint64_t vd = v_desc + (uint64_t)(vst * kVStep);
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk)
+            mma_ts(tmem + C::O_COL, tmem + C::P_COL + kk * 8,
+                   vd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_pv,
+                   (j == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(pv_done);
+          if (last) mma_commit(o_full);
+          mma_commit(&v_empty[vst]);
         }
         __syncwarp();
-        ++n_pv;
-        if (!more) ++n_o;
-        stage = nxt;
-        kv_phase = nxt_phase;
+        if (last) ++n_o;
+        if (++vst == C::V_STAGES) {
+          vst = 0;
+          v_phase ^= 1;
+        }
       }
     }
-#undef GQE_ISSUE_S
-#undef GQE_ISSUE_PV
   }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
@@ -426,8 +499,30 @@ attn_kernel(const __grid_constant__ Params P) {
           alpha = fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        // S(j) was issued without waiting for P(j-1) V: wait for that product before
-        // overwriting P or rescaling O.
+        // p = exp2(s * scale - m) with a packed FMA for the argument; most pairs on MUFU,
+        // kFmaPairsOf8 of every 8 on the FMA-pipe polynomial. P is kept in registers as
+        // bf16 pairs until the whole tile is done.
+        const float2 cs2 = make_float2(cs, cs);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        uint32_t pk[TK / 2];
+        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int x = 0; x < TK / 2; ++x) {
+          const float2 t = fma2(make_float2(s[2 * x], s[2 * x + 1]), cs2, nm2);
+          const float2 p = (x & 7) >= 8 - kFmaPairsOf8
+                               ? exp2_fma2(t)
+                               : make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          if constexpr (!C::SUM_MMA) lsum[x & 3] = add2(lsum[x & 3], p);
+          pk[x] = pack_bf16x2(p.x, p.y);
+        }
+        if constexpr (!C::SUM_MMA) {
+          const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
+          l = l * alpha + (a.x + a.y);  // alpha = 1 unless this row's maximum moved on
+        }
+        // S(j) was issued without waiting for P(j-1) V, and the exponentials above did not
+        // need it either: only now wait for that product before overwriting P or
+        // rescaling O.
         if (j > 0 && !warp_wait(pv_done, (n_s - 2) & 1, P, abort_flag)) {
           ok = false;
           break;
@@ -435,38 +530,20 @@ attn_kernel(const __grid_constant__ Params P) {
         if (__any_sync(0xffffffffu, need)) {
           tc_fence_after();
 #pragma unroll
-          for (int c0 = 0; c0 < DH; c0 += 16) {
+          for (int c0 = 0; c0 < C::N_PV; c0 += 16) {
             uint32_t r[16];
             tmem_ld16_wait(t_o + c0, r);
 #pragma unroll
             for (int x = 0; x < 16; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
             tmem_st16(t_o + c0, r);
           }
-          l *= alpha;
         }
-        // p = exp2(s * scale - m): packed FMA for the argument, MUFU ex2, four packed
-        // partial sums; P goes to TMEM as bf16 pairs.
-        const float2 cs2 = make_float2(cs, cs);
-        const float2 nm2 = make_float2(-m_used, -m_used);
-        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c0 = 0; c0 < TK; c0 += 32) {
-          uint32_t pk[16];
+        for (int c0 = 0; c0 < TK / 2; c0 += 16) {
+          uint32_t r[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float2 t = fma2(make_float2(s[c0 + 2 * x], s[c0 + 2 * x + 1]), cs2, nm2);
-            // one pair in four on the FMA pipe, the rest on MUFU
-            const float2 p = (x & 3) == 3 ? exp2_fma2(t)
-                                          : make_float2(fast_exp2(t.x), fast_exp2(t.y));
-            lsum[x & 3] = add2(lsum[x & 3], p);
-            pk[x] = pack_bf16x2(p.x, p.y);
-          }
-          tmem_st16(t_p + c0 / 2, pk);
-        }
-        {
-          const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
-          l += a.x + a.y;
+          for (int x = 0; x < 16; ++x) r[x] = pk[c0 + x];
+          tmem_st16(t_p + c0, r);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -480,6 +557,11 @@ attn_kernel(const __grid_constant__ Params P) {
       tc_fence_after();
       const bool valid = q < P.T;
       const int64_t tok = (int64_t)it.b * P.T + q;
+      if constexpr (C::SUM_MMA) {
+        uint32_t r[16];
+        tmem_ld16_wait(t_o + DH, r);
+        l = __uint_as_float(r[0]);
+      }
       float scale = 1.f / l;
       int col;
       if (it.s < P.Sr) {
