@@ -181,7 +181,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
             if (lane == 0) set_timeout(P, abort_flag);
             break;
           }
-          if (lane == 0) {
+          if (elect_one()) {
             mbar_arrive_expect_tx(&full[stage], (uint32_t)A_STAGE_BYTES + b_bytes);
             tma_load_2d(sA + stage * A_STAGE_BYTES, &P.tmap_a, kb * BK, ti.m0, &full[stage]);
             tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[ti.p], kb * BK, ti.n0, &full[stage]);
@@ -224,7 +224,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
             if (lane == 0) set_timeout(P, abort_flag);
             break;
           }
-          if (lane == 0) {
+          if (elect_one()) {
             mbar_arrive_expect_tx(&full[stage], b_bytes);
             tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, t.x * P.d_h,
                         &full[stage]);
@@ -290,7 +290,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
           // descriptor = base + offset in 16-byte units (K step: 32 bytes inside the atom)
           const uint64_t ad = a_desc0 + (uint64_t)(stage * (A_STAGE_BYTES >> 4));
           const uint64_t bd = b_desc0 + (uint64_t)(stage * (B_STAGE_BYTES >> 4));
@@ -306,7 +306,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
         }
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(&acc_full[acc]);
+      if (elect_one()) mma_commit(&acc_full[acc]);
       __syncwarp();
     }
   } else {
