@@ -152,11 +152,11 @@ gqe_status gqe_set_spin_limit(gqe_handle h, int64_t limit);
  * i and events[GQE_NUM_STAGES] after the last. The events must outlive the forwards that
  * record them. Stage names: gqe_stage_name.
  */
-#define GQE_NUM_STAGES 8
+#define GQE_NUM_STAGES 6
 gqe_status gqe_set_stage_events(gqe_handle h, void* const* events, int count);
 
-/* gqe_stage_name — "dense_proj", "route", "route_scan", "bucket", "qproj", "attention",
- * "combine", "oproj" for i = 0..7; NULL otherwise. */
+/* gqe_stage_name — "dense_proj", "route", "qproj", "attention", "combine", "oproj" for
+ * i = 0..5; NULL otherwise. */
 const char* gqe_stage_name(int i);
 
 /*

@@ -65,6 +65,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.tile_list = (int2*)take((size_t)((M * Gk + 127) / 128 + N + 1) * sizeof(int2));
   w.tile_count = (int32_t*)take(16);
   w.attn_counter = (int32_t*)take(16);
+  w.grid_sync = (int32_t*)take(16);
   w.status = (int32_t*)take(16);
   w.wcat = take((size_t)(N + (2 * G + 1) * d_h) * dim * esz);
   (void)dim;
@@ -130,7 +131,9 @@ gqe_status gqe_create(gqe_handle* out, int dim, int N, int G, int k, int d_h, gq
   layout(h->ws, static_cast<char*>(base), dim, N, G, k, d_h, h->esz, max_tokens);
   h->ws.base = base;
   h->ws.bytes = bytes;
-  if (cudaMemset(h->ws.status, 0, 16) != cudaSuccess) {
+  // Everything starts at zero: counters, the status word, and index arrays (so no stale
+  // value can ever name a token or expert outside the current call's range).
+  if (cudaMemset(base, 0, bytes) != cudaSuccess) {
     cudaFree(base);
     delete h;
     return GQE_ERR_CUDA;
@@ -170,8 +173,8 @@ gqe_status gqe_set_stage_events(gqe_handle h, void* const* events, int count) {
 }
 
 const char* gqe_stage_name(int i) {
-  static const char* names[GQE_NUM_STAGES] = {"dense_proj", "route", "route_scan", "bucket",
-                                               "qproj", "attention", "combine", "oproj"};
+  static const char* names[GQE_NUM_STAGES] = {"dense_proj", "route", "qproj",
+                                               "attention", "combine", "oproj"};
   return (i >= 0 && i < GQE_NUM_STAGES) ? names[i] : nullptr;
 }
 
@@ -219,8 +222,7 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   bool ok = mark() &&
             add(tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)
                    : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
-            add(launch_route_select(h, M, st)) &&
-            add(launch_route_scan_aux(h, M, aux_loss, st)) && add(launch_bucket(h, M, st)) &&
+            add(launch_route_fused(h, M, aux_loss, st)) &&
             add(tc ? launch_tc_qproj(h, x, M, W_q, st) : launch_simt_qproj(h, x, M, W_q, st)) &&
             add(tc ? launch_tc_attention(h, B, T, S, has_shared, variant, causal, Do, st)
                    : launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&

@@ -64,6 +64,7 @@ struct Workspace {
   int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* attn_counter = nullptr; // attention work-item counter
+  int32_t* grid_sync = nullptr;    // grid-barrier counters of the fused routing kernel
   int32_t* status = nullptr;       // device status word
   void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
   void* base = nullptr;            // the single allocation
@@ -86,6 +87,8 @@ struct gqe_ctx {
   int n_stage_events = 0;
   // state of the last forward
   int last_M = 0, last_S = 0, last_Do = 0, last_launches = 0;
+  // resident-CTA capacity of the fused routing kernel (0 until its first launch)
+  int route_cap = 0;
 };
 
 namespace gqe {
@@ -109,6 +112,7 @@ route_scan_aux_kernel(int32_t* __restrict__ part_counts,
 int launch_simt_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
                            const void* W_v, const void* W_shared, cudaStream_t st);
 int launch_route_select(gqe_ctx* h, int M, cudaStream_t st);
+int launch_route_fused(gqe_ctx* h, int M, float* aux_out, cudaStream_t st);
 int launch_route_scan_aux(gqe_ctx* h, int M, float* aux_out, cudaStream_t st);
 int launch_bucket(gqe_ctx* h, int M, cudaStream_t st);
 int launch_simt_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);

@@ -8,20 +8,20 @@
 
 namespace gqe {
 
-// One thread per token; the block's logits [128, N] are staged in shared memory (one
-// coalesced copy) and every per-token array lives there too, so nothing spills to local
-// memory. Writes sel / p_sel / gates / w [M, G, k] and this block's per-expert token
-// counts and probability sums to part_counts / part_prob [blockIdx, N] (summed later in a
-// fixed order, so the result does not depend on scheduling).
-__global__ void __launch_bounds__(kRouteBlock)
-route_select_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
-                    int32_t* __restrict__ sel, float* __restrict__ psel,
-                    float* __restrict__ gates, float* __restrict__ wslot,
-                    int32_t* __restrict__ part_counts, float* __restrict__ part_prob) {
-  __shared__ float s_p[kRouteBlock][kMaxExperts + 1];          // logits, then probabilities
-  __shared__ unsigned char s_hit[kRouteBlock][kMaxExperts + 1];  // selected experts
+// Selection for one block of kRouteBlock tokens, one thread per token. The block's logits
+// [128, N] are staged in shared memory (one coalesced copy) and every per-token array lives
+// there too, so nothing spills to local memory. Writes sel / p_sel / gates / w [M, G, k] and
+// this block's per-expert token counts and probability sums to part_counts / part_prob
+// [blk, N] (summed later in a fixed order, so the result does not depend on scheduling).
+// Leaves the block's selection flags in s_hit.
+__device__ void select_block(const float* __restrict__ logits, int blk, int M, int N, int G,
+                             int k, int32_t* __restrict__ sel, float* __restrict__ psel,
+                             float* __restrict__ gates, float* __restrict__ wslot,
+                             int32_t* __restrict__ part_counts, float* __restrict__ part_prob,
+                             float (*s_p)[kMaxExperts + 1],
+                             unsigned char (*s_hit)[kMaxExperts + 1]) {
   const int E = N / G;
-  const int t0 = blockIdx.x * kRouteBlock;
+  const int t0 = blk * kRouteBlock;
   const int tid = threadIdx.x;
   const int t = t0 + tid;
   const bool valid = t < M;
@@ -105,9 +105,20 @@ route_select_kernel(const float* __restrict__ logits, int M, int N, int G, int k
       ps += s_p[i][tid];
       c += s_hit[i][tid];
     }
-    part_prob[(int64_t)blockIdx.x * N + tid] = ps;
-    part_counts[(int64_t)blockIdx.x * N + tid] = c;
+    part_prob[(int64_t)blk * N + tid] = ps;
+    part_counts[(int64_t)blk * N + tid] = c;
   }
+}
+
+__global__ void __launch_bounds__(kRouteBlock)
+route_select_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
+                    int32_t* __restrict__ sel, float* __restrict__ psel,
+                    float* __restrict__ gates, float* __restrict__ wslot,
+                    int32_t* __restrict__ part_counts, float* __restrict__ part_prob) {
+  __shared__ float s_p[kRouteBlock][kMaxExperts + 1];          // logits, then probabilities
+  __shared__ unsigned char s_hit[kRouteBlock][kMaxExperts + 1];  // selected experts
+  select_block(logits, blockIdx.x, M, N, G, k, sel, psel, gates, wslot, part_counts, part_prob,
+               s_p, s_hit);
 }
 
 // One block of 32 warps; warp w handles experts w and w + 32. Lane l sums a contiguous run
@@ -210,6 +221,377 @@ bucket_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ base,
     const int slot = base[(int64_t)blockIdx.x * N + e] + before;
     bucket[slot] = (t << 3) | rank;
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// The whole routing stage in one cooperative launch: selection, the per-expert statistics
+// and Switch loss, the expert buckets and the routed-projection tile list. Persistent CTAs
+// of kFusedThreads (all resident, guaranteed by the cooperative launch) take blocks of
+// kRouteBlock tokens in turn; two grid barriers separate the phases. Per token and group
+// the arithmetic is that of select_block (same operations in the same order), so the
+// selections, gates and statistics equal route_select_kernel's; only the work is spread
+// over one thread per (token, group) and the loads are batched.
+// ---------------------------------------------------------------------------------------
+constexpr int kFusedThreads = 512;
+
+// Dynamic shared memory of the fused kernel for N experts in G groups.
+__host__ __device__ inline int fused_smem_bytes(int N, int G) {
+  const int sel_bytes = kRouteBlock * N * 4 + kRouteBlock * G * 4 + kRouteBlock * N;
+  const int bucket_bytes = kRouteBlock * N + 4 * N + 4 * N * (kRouteBlock / 32);
+  const int scan_bytes = 8 * kFusedThreads + 8 * kMaxExperts + 4 * kFusedThreads + 12 * (kMaxExperts + 1);
+  const int a = (sel_bytes + 15) / 16 * 16;
+  return a + (bucket_bytes > scan_bytes ? bucket_bytes : scan_bytes) + 64;
+}
+
+// Grid-wide barrier on a counter that is zero at launch; the i-th barrier waits for
+// i * gridDim.x arrivals. Bounded: gives up after `spin` polls and reports it.
+__device__ bool grid_barrier(int32_t* ctr, int target, int64_t spin) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1);
+    int ok = 0;
+    for (int64_t i = 0; i < spin; ++i) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= target) {
+        ok = 1;
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Selection of one token block, one thread per (token, group). Leaves the probabilities in
+// s_p [128][N], the chosen experts' ranks + 1 in s_hit [128][N] (0 = not chosen) and writes
+// sel / p_sel / gates / w and the block's part_counts / part_prob.
+__device__ void fused_select(const float* __restrict__ logits, int blk, int M, int N, int G,
+                             int k, int32_t* __restrict__ sel, float* __restrict__ psel,
+                             float* __restrict__ gates, float* __restrict__ wslot,
+                             int32_t* __restrict__ part_counts, float* __restrict__ part_prob,
+                             float* s_p, unsigned char* s_hit, float* s_psum) {
+  const int E = N / G;
+  const int tid = threadIdx.x;
+  const int t0 = blk * kRouteBlock;
+  const int rows = min(kRouteBlock, M - t0);
+  const float* src = logits + (int64_t)t0 * N;
+#pragma unroll 4
+  for (int i = tid; i < kRouteBlock * N; i += kFusedThreads) {
+    s_p[i] = i < rows * N ? __ldcg(src + i) : 0.f;
+    s_hit[i] = 0;
+  }
+  __syncthreads();
+  for (int pi = tid; pi < kRouteBlock * G; pi += kFusedThreads) {
+    const int tl = pi / G, g = pi % G;
+    const int t = t0 + tl;
+    float* lg = s_p + tl * N + g * E;
+    unsigned char* hit = s_hit + tl * N + g * E;
+    if (t >= M) {
+      for (int j = 0; j < E; ++j) lg[j] = 0.f;
+      s_psum[tl * G + g] = 0.f;
+      continue;
+    }
+    // top-k on the logits (ties: the lowest index), then the group softmax in place
+    uint64_t taken = 0;
+    for (int r = 0; r < k; ++r) {
+      int best = -1;
+      float bv = 0.f;
+      for (int j = 0; j < E; ++j) {
+        if (taken >> j & 1ull) continue;
+        if (best < 0 || lg[j] > bv) {
+          best = j;
+          bv = lg[j];
+        }
+      }
+      taken |= 1ull << best;
+    }
+    float mx = lg[0];
+    for (int j = 1; j < E; ++j) mx = fmaxf(mx, lg[j]);
+    float den = 0.f;
+    for (int j = 0; j < E; ++j) {
+      const float z = expf(lg[j] - mx);
+      lg[j] = z;
+      den += z;
+    }
+    const float inv = 1.f / den;
+    float psum = 0.f;
+    for (int j = 0; j < E; ++j) {
+      lg[j] *= inv;
+      if (taken >> j & 1ull) psum += lg[j];
+    }
+    const float ginv = 1.f / psum;
+    int r = 0;
+    for (int j = 0; j < E; ++j) {
+      if (!(taken >> j & 1ull)) continue;
+      hit[j] = (unsigned char)(r + 1);
+      const int64_t o = (int64_t)t * G * k + g * k + r;
+      sel[o] = j;
+      psel[o] = lg[j];
+      gates[o] = lg[j] * ginv;
+      ++r;
+    }
+    s_psum[tl * G + g] = psum;
+  }
+  __syncthreads();
+  // slot weights: p of each selection renormalised over the token's G*k selections
+  for (int pi = tid; pi < kRouteBlock * G; pi += kFusedThreads) {
+    const int tl = pi / G, g = pi % G;
+    const int t = t0 + tl;
+    if (t >= M) continue;
+    float p_tot = 0.f;
+    for (int gg = 0; gg < G; ++gg) p_tot += s_psum[tl * G + gg];
+    const float winv = 1.f / p_tot;
+    int r = 0;
+    for (int j = 0; j < E; ++j)
+      if (s_hit[tl * N + g * E + j])
+        wslot[(int64_t)t * G * k + g * k + r++] = s_p[tl * N + g * E + j] * winv;
+  }
+  // per-expert sums over the block's tokens, in token order
+  if (tid < N) {
+    float ps = 0.f;
+    int c = 0;
+    for (int i = 0; i < kRouteBlock; ++i) {
+      ps += s_p[i * N + tid];
+      c += s_hit[i * N + tid] != 0;
+    }
+    part_prob[(int64_t)blk * N + tid] = ps;
+    part_counts[(int64_t)blk * N + tid] = c;
+  }
+  __syncthreads();
+}
+
+// Scan of the per-block statistics by one CTA. Thread (e, c) sums a fixed run of router
+// blocks for expert e (kFusedThreads / N threads per expert, loads in batches of eight);
+// the runs combine in run order (probabilities in double), so the result does not depend
+// on scheduling. Writes counts / mean_prob / offsets and the Switch loss
+//   L = (1/G) sum_g E sum_j f_{g,j} Pbar_{g,j},  f = c / (M k),  Pbar = prob_sum / M,
+// turns part_counts into each (block, expert)'s first bucket slot, and lists the
+// routed-projection tiles: each expert's bucket cut into runs of 128 slots.
+__device__ void fused_scan(int32_t* __restrict__ part_counts, const float* __restrict__ part_prob,
+                           int nblk, int M, int N, int G, int k, int32_t* __restrict__ counts,
+                           float* __restrict__ mean_prob, int32_t* __restrict__ offsets,
+                           float* __restrict__ aux_out, int2* __restrict__ tile_list,
+                           int32_t* __restrict__ tile_count, uint8_t* smem) {
+  double* s_ppart = reinterpret_cast<double*>(smem);                 // [kFusedThreads]
+  double* s_term = s_ppart + kFusedThreads;                          // [kMaxExperts]
+  int* s_cpart = reinterpret_cast<int*>(s_term + kMaxExperts);      // [kFusedThreads]
+  int* s_cnt = s_cpart + kFusedThreads;                              // [kMaxExperts]
+  int* s_off = s_cnt + kMaxExperts;                                  // [kMaxExperts + 1]
+  int* s_nt = s_off + kMaxExperts + 1;                               // [kMaxExperts + 1]
+  const int tid = threadIdx.x;
+  const int tpe = max(1, kFusedThreads / N);  // threads per expert
+  const int e = tid / tpe, c = tid % tpe;
+  const bool act = e < N;
+  const int chunk = (nblk + tpe - 1) / tpe;
+  const int b0 = min(nblk, c * chunk), b1 = min(nblk, b0 + chunk);
+  if (act) {
+    int cs = 0;
+    double ps = 0.0;
+    for (int b = b0; b < b1; b += 8) {
+      int cv[8];
+      float pv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = b + u < b1;
+        cv[u] = in ? __ldcg(part_counts + (int64_t)(b + u) * N + e) : 0;
+        pv[u] = in ? __ldcg(part_prob + (int64_t)(b + u) * N + e) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        cs += cv[u];
+        if (b + u < b1) ps += (double)pv[u];
+      }
+    }
+    s_cpart[tid] = cs;
+    s_ppart[tid] = ps;
+  }
+  __syncthreads();
+  if (act && c == 0) {
+    int tot = 0;
+    double ps = 0.0;
+    for (int i = 0; i < tpe; ++i) {
+      const int v = s_cpart[tid + i];
+      s_cpart[tid + i] = tot;  // exclusive prefix of the runs
+      tot += v;
+      ps += s_ppart[tid + i];
+    }
+    counts[e] = tot;
+    mean_prob[e] = (float)(ps / M);
+    s_cnt[e] = tot;
+    s_term[e] = (double)(N / G) * ((double)tot / ((double)M * k)) * (ps / M);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int off = 0, nt = 0;
+    for (int x = 0; x < N; ++x) {
+      s_off[x] = off;
+      offsets[x] = off;
+      s_nt[x] = nt;
+      nt += (s_cnt[x] + 127) / 128;
+      off += s_cnt[x];
+    }
+    offsets[N] = off;
+    *tile_count = nt;
+    if (aux_out != nullptr) {
+      double L = 0.0;
+      for (int x = 0; x < N; ++x) L += s_term[x];
+      aux_out[0] = (float)(L / G);
+    }
+  }
+  __syncthreads();
+  if (act) {
+    int run = s_off[e] + s_cpart[tid];
+    for (int b = b0; b < b1; b += 8) {
+      int cv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        cv[u] = b + u < b1 ? __ldcg(part_counts + (int64_t)(b + u) * N + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (b + u < b1) part_counts[(int64_t)(b + u) * N + e] = run;
+        run += cv[u];
+      }
+    }
+  }
+  for (int x = tid; x < N; x += kFusedThreads) {
+    const int nt = (s_cnt[x] + 127) / 128;
+    for (int i = 0; i < nt; ++i) tile_list[s_nt[x] + i] = make_int2(x, s_off[x] + i * 128);
+  }
+}
+
+// Bucket entries of one token block: entry (t << 3) | r for every selection, at the
+// expert's base slot for this block plus the number of earlier tokens of the block that
+// chose the same expert (so each expert's bucket is in token order); one warp ballot per
+// expert gives those counts. s_hit holds the block's ranks + 1 if `have_hits`, else they are
+// read back from sel.
+__device__ void fused_bucket(const int32_t* __restrict__ sel, const int32_t* __restrict__ base,
+                             int blk, int M, int N, int G, int k, int32_t* __restrict__ bucket,
+                             unsigned char* s_hit, bool have_hits, uint8_t* scratch) {
+  constexpr int kWarps = kRouteBlock / 32;
+  unsigned char* s_lb = scratch;                                      // [128][N] lanes before
+  int* s_base = reinterpret_cast<int*>(scratch + ((kRouteBlock * N + 15) / 16 * 16));  // [N]
+  int* s_warp = s_base + N;                                           // [N][kWarps]
+  const int E = N / G;
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int t = blk * kRouteBlock + tid;
+  if (!have_hits) {
+    for (int i = tid; i < kRouteBlock * N; i += kFusedThreads) s_hit[i] = 0;
+    __syncthreads();
+    for (int pi = tid; pi < kRouteBlock * G; pi += kFusedThreads) {
+      const int tl = pi / G, g = pi % G;
+      const int tt = blk * kRouteBlock + tl;
+      if (tt >= M) continue;
+      for (int r = 0; r < k; ++r)
+        s_hit[tl * N + g * E + __ldcg(sel + (int64_t)tt * G * k + g * k + r)] =
+            (unsigned char)(r + 1);
+    }
+  }
+  if (tid < N) s_base[tid] = __ldcg(base + (int64_t)blk * N + tid);
+  __syncthreads();
+  if (tid < kRouteBlock) {
+    for (int e = 0; e < N; ++e) {
+      const unsigned ball = __ballot_sync(0xffffffffu, s_hit[tid * N + e] != 0);
+      s_lb[tid * N + e] = (unsigned char)__popc(ball & ((1u << lane) - 1u));
+      if (lane == 0) s_warp[e * kWarps + warp] = __popc(ball);
+    }
+  }
+  __syncthreads();
+  if (tid < kRouteBlock && t < M) {
+    for (int e = 0; e < N; ++e) {
+      const int r1 = s_hit[tid * N + e];
+      if (!r1) continue;
+      int before = s_lb[tid * N + e];
+      for (int w = 0; w < warp; ++w) before += s_warp[e * kWarps + w];
+      bucket[s_base[e] + before] = (t << 3) | (r1 - 1);
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kFusedThreads)
+route_fused_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
+                   int32_t* __restrict__ sel, float* __restrict__ psel,
+                   float* __restrict__ gates, float* __restrict__ wslot,
+                   int32_t* __restrict__ part_counts, float* __restrict__ part_prob,
+                   int32_t* __restrict__ counts, float* __restrict__ mean_prob,
+                   int32_t* __restrict__ offsets, float* __restrict__ aux_out,
+                   int32_t* __restrict__ bucket, int2* __restrict__ tile_list,
+                   int32_t* __restrict__ tile_count, int32_t* __restrict__ grid_ctr,
+                   int32_t* __restrict__ status, int64_t spin) {
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  float* s_p = reinterpret_cast<float*>(dsmem);                         // [128][N]
+  float* s_psum = s_p + kRouteBlock * N;                                // [128][G]
+  unsigned char* s_hit = reinterpret_cast<unsigned char*>(s_psum + kRouteBlock * G);  // [128][N]
+  uint8_t* scratch = dsmem + ((kRouteBlock * N * 4 + kRouteBlock * G * 4 + kRouteBlock * N + 15) / 16 * 16);
+  const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x)
+    fused_select(logits, blk, M, N, G, k, sel, psel, gates, wslot, part_counts, part_prob, s_p,
+                 s_hit, s_psum);
+  if (!grid_barrier(grid_ctr, gridDim.x, spin)) {
+    if (threadIdx.x == 0) atomicExch(status, kStatusTimeout);
+    return;
+  }
+  if (blockIdx.x == 0)
+    fused_scan(part_counts, part_prob, nblk, M, N, G, k, counts, mean_prob, offsets, aux_out,
+               tile_list, tile_count, scratch);
+  if (!grid_barrier(grid_ctr, 2 * gridDim.x, spin)) {
+    if (threadIdx.x == 0) atomicExch(status, kStatusTimeout);
+    return;
+  }
+  // a CTA that selected a single block still holds that block's ranks in shared memory
+  const bool single = nblk <= (int)gridDim.x;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x)
+    fused_bucket(sel, part_counts, blk, M, N, G, k, bucket, s_hit, single, scratch);
+}
+
+int launch_route_fused(gqe_ctx* h, int M, float* aux_out, cudaStream_t st) {
+  const int smem = fused_smem_bytes(h->N, h->G);
+  if (h->route_cap == 0) {
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel, kFusedThreads,
+                                                      smem) != cudaSuccess ||
+        per_sm < 1)
+      return -1;
+    h->route_cap = per_sm * h->num_sms;
+  }
+  const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
+  int grid = nblk < h->route_cap ? nblk : h->route_cap;
+  if (cudaMemsetAsync(h->ws.grid_sync, 0, 16, st) != cudaSuccess) return -1;
+  const float* logits = h->ws.logits;
+  int32_t* sel = h->ws.sel;
+  float* psel = h->ws.psel;
+  float* gates = h->ws.gates;
+  float* wslot = h->ws.w;
+  int32_t* pc = h->ws.part_counts;
+  float* pp = h->ws.part_prob;
+  int32_t* counts = h->ws.counts;
+  float* mp = h->ws.mean_prob;
+  int32_t* offs = h->ws.offsets;
+  int32_t* bucket = h->ws.bucket;
+  int2* tl = h->ws.tile_list;
+  int32_t* tc = h->ws.tile_count;
+  int32_t* gs = h->ws.grid_sync;
+  int32_t* status = h->ws.status;
+  // The grid barriers wait only for co-resident CTAs of this launch (the cooperative launch
+  // guarantees that they all run), so they use a fixed generous bound rather than the
+  // handle's spin limit: a test that shortens the other kernels' waits leaves the routing
+  // complete and consistent.
+  int64_t spin = (int64_t)1 << 26;
+  int N = h->N, G = h->G, k = h->k;
+  void* args[] = {&logits, &M, &N, &G, &k, &sel, &psel, &gates, &wslot, &pc, &pp, &counts,
+                  &mp, &offs, &aux_out, &bucket, &tl, &tc, &gs, &status, &spin};
+  if (cudaLaunchCooperativeKernel((const void*)route_fused_kernel, dim3(grid),
+                                  dim3(kFusedThreads), args, smem, st) != cudaSuccess)
+    return -1;
+  return 1;
 }
 
 int launch_route_select(gqe_ctx* h, int M, cudaStream_t st) {

@@ -119,8 +119,8 @@ qproj_kernel(const T* __restrict__ x, int M, int K, const T* __restrict__ Wq, in
     const int m = m0 + ty + 16 * i;
     if (m >= cnt) continue;
     const int ent = bucket[beg + m];
-    const int64_t t = ent >> 3;
-    const int s = g * k + (ent & 7);
+    const int64_t t = min(ent >> 3, M - 1);
+    const int s = g * k + min(ent & 7, k - 1);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx + 16 * j;

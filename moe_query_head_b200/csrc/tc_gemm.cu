@@ -208,11 +208,13 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
         // source rows of this lane: r = 4 i + lane / 8 (rows past the tile's end repeat
         // its first row: computed, never stored)
         int src[BM / 4];
-        const int first = P.bucket[t.y] >> 3;
+        // (token indices are clamped to the call's rows: defence against a bucket that a
+        // failed routing pass left stale; a complete pass never needs it)
+        const int first = min(P.bucket[t.y] >> 3, P.M - 1);
 #pragma unroll
         for (int i = 0; i < BM / 4; ++i) {
           const int r = 4 * i + (lane >> 3);
-          src[i] = r < n ? (P.bucket[t.y + r] >> 3) : first;
+          src[i] = r < n ? min(P.bucket[t.y + r] >> 3, P.M - 1) : first;
         }
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++g) {
@@ -334,8 +336,8 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
         __nv_bfloat16* dst = nullptr;
         if (valid) {
           const int g = ti.p / P.E;
-          const int64_t s = (int64_t)g * P.k + (ent & 7);
-          dst = P.Q + (s * P.M + (ent >> 3)) * P.d_h;
+          const int64_t s = (int64_t)g * P.k + min(ent & 7, P.k - 1);
+          dst = P.Q + (s * P.M + min(ent >> 3, P.M - 1)) * P.d_h;
         }
         for (int c0 = 0; c0 < ti.n; c0 += 16) {
           uint32_t r[16];
@@ -406,32 +408,6 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
-}
-
-// Tiles of the routed projection: each expert's bucket cut into runs of BM slots.
-// One thread per expert (N <= 64): tile counts, an exclusive scan, then each thread writes
-// its expert's tiles.
-__global__ void qproj_tiles_kernel(const int32_t* __restrict__ offsets, int N,
-                                   int2* __restrict__ tile_list, int32_t* __restrict__ tile_count) {
-  __shared__ int s_n[kMaxExperts + 1];
-  const int e = threadIdx.x;
-  const int beg = e < N ? offsets[e] : 0;
-  const int cnt = e < N ? offsets[e + 1] - beg : 0;
-  const int nt = (cnt + BM - 1) / BM;
-  if (e < kMaxExperts) s_n[e] = nt;
-  __syncthreads();
-  if (e == 0) {
-    int run = 0;
-    for (int i = 0; i < N; ++i) {
-      const int v = s_n[i];
-      s_n[i] = run;
-      run += v;
-    }
-    *tile_count = run;
-  }
-  __syncthreads();
-  if (e < N)
-    for (int i = 0; i < nt; ++i) tile_list[s_n[e] + i] = make_int2(e, beg + i * BM);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -536,10 +512,8 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   return launch<false>(h, P, grid, st);
 }
 
+// The tile list (expert, first bucket slot) and its length come from the routing stage.
 int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st) {
-  qproj_tiles_kernel<<<1, kMaxExperts, 0, st>>>(h->ws.offsets, h->N, h->ws.tile_list,
-                                                 h->ws.tile_count);
-  if (cudaGetLastError() != cudaSuccess) return -1;
   Params P;
   memset(&P, 0, sizeof(P));
   // A: rows of x gathered four at a time (box one row high, 128 bytes wide)
@@ -565,7 +539,7 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStrea
   P.spin = spin_limit(h);
   const int max_tiles = (int)(((int64_t)M * h->G * h->k + BM - 1) / BM) + h->N;
   const int grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
-  return launch<true>(h, P, grid, st) < 0 ? -1 : 2;
+  return launch<true>(h, P, grid, st);
 }
 
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st) {

@@ -24,7 +24,7 @@ EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
             "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma")
-GQE_NUM_STAGES = 8
+GQE_NUM_STAGES = 6
 
 
 class GQEError(RuntimeError):
