@@ -87,7 +87,7 @@ struct Cfg {
 // Exponentials: of every 8 pairs of scores, this many go to the FMA-pipe polynomial and
 // the rest to the MUFU unit (16 results per SM per clock on B200).
 #ifndef GQE_ATTN_FMA_PAIRS_OF_8
-#define GQE_ATTN_FMA_PAIRS_OF_8 2
+#define GQE_ATTN_FMA_PAIRS_OF_8 3
 #endif
 constexpr int kFmaPairsOf8 = GQE_ATTN_FMA_PAIRS_OF_8;
 
