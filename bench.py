@@ -316,14 +316,15 @@ def bench_ours(args, rank, world, dist):
     if st != G.GQE_OK:
         raise RuntimeError("device status after timing: " + G.status_str(st))
 
+    att_i = [G.gqe_stage_name(i) for i in range(G.GQE_NUM_STAGES)].index("attention")
     if dist:
         import torch.distributed as td
-        t = torch.tensor([total_ms, totalE_ms, e2e_ms, stage_ms[5]], device="cuda",
+        t = torch.tensor([total_ms, totalE_ms, e2e_ms, stage_ms[att_i]], device="cuda",
                          dtype=torch.float64)
         td.all_reduce(t, op=td.ReduceOp.MAX)
         total_ms, totalE_ms, e2e_ms, att_ms_tot = [float(v) for v in t.cpu()]
     else:
-        att_ms_tot = float(stage_ms[5])
+        att_ms_tot = float(stage_ms[att_i])
 
     peaks, peak_src = load_peaks()
     ms = total_ms / args.steps
