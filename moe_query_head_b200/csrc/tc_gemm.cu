@@ -141,7 +141,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], GATHER ? 2 : 1);
+      mbar_init(&full[s], GATHER ? 33 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -194,10 +194,11 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       }
     } else {
       // Four producer warps; warp p fills every fourth stage of the CTA's stage sequence.
-      // A rows are gathered through registers: lane l moves 16-byte chunk l % 8 of rows
-      // 4 i + l / 8 (eight lanes per 128-byte row segment: coalesced loads, conflict-free
-      // stores into the 128-byte-swizzled slot). B (the expert's W_q rows) comes by TMA.
-      // The stage's full barrier takes two arrivals: the TMA's and this warp's.
+      // A rows are gathered by asynchronous 16-byte copies (cp.async, no registers, many
+      // stages in flight): lane l moves chunk l % 8 of rows 4 i + l / 8 (eight lanes per
+      // 128-byte row segment: coalesced reads, conflict-free writes into the
+      // 128-byte-swizzled slot). B (the expert's W_q rows) comes by TMA. The stage's full
+      // barrier takes 33 arrivals: the TMA's, and one per lane when its copies complete.
       const int pw = warp;
       const int c = lane & 7;
       uint32_t g = 0;  // position in the CTA's stage sequence
@@ -231,30 +232,23 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
             tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, t.x * P.d_h,
                         &full[stage]);
           }
-          uint8_t* dst = sA + stage * A_STAGE_BYTES;
+          const uint32_t dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const int kcol = kb * BK + c * 8;
-          const bool kok = kcol < P.K;
+          // columns past K are zero-filled (nothing is read; the address stays in range)
+          const uint32_t nbytes = kcol < P.K ? 16u : 0u;
+          const int kc = kcol < P.K ? kcol : 0;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint4 v[BM / 8];
-#pragma unroll
-            for (int i = 0; i < BM / 8; ++i) {
-              const int ii = h * (BM / 8) + i;
-              v[i] = kok ? __ldg(reinterpret_cast<const uint4*>(P.x + (int64_t)src[ii] * P.K + kcol))
-                         : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < BM / 8; ++i) {
-              const int r = 4 * (h * (BM / 8) + i) + (lane >> 3);
-              *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = v[i];
-            }
+          for (int i = 0; i < BM / 4; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), P.x + (int64_t)src[i] * P.K + kc,
+                        nbytes);
           }
-          fence_async_shared();  // these generic-proxy stores before the tensor core reads
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[stage]);
+          cp_async_mbar_arrive_noinc(&full[stage]);
         }
         if (!ok) break;
       }
+      // no copy of this warp may still be writing when the CTA leaves
+      cp_async_wait<0>();
     }
   } else if (warp == L::MMA) {
     // ------------------------------------------------------------------ MMA issuer
@@ -291,6 +285,9 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           if (lane == 0) set_timeout(P, abort_flag);
           break;
         }
+        // gathered rows were written by the generic proxy (cp.async): make them visible
+        // to the tensor core's reads
+        if constexpr (GATHER) fence_async_shared();
         tc_fence_after();
         if (elect_one()) {
           // descriptor = base + offset in 16-byte units (K step: 32 bytes inside the atom)
