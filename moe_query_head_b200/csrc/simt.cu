@@ -245,12 +245,23 @@ __global__ void slot_kernel(T* __restrict__ Z, const float* __restrict__ w, int 
 #pragma unroll
   for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
   const T* zt = Z + t * Do + c0;
-  for (int s = 0; s < Sr; ++s) {
-    const float ws = w[t * Sr + s];
-    const uint4 raw = *reinterpret_cast<const uint4*>(zt + (int64_t)s * d_h);
-    const T* val = reinterpret_cast<const T*>(&raw);
+  // eight streams per batch: all their loads are issued before the first use
+  for (int s0 = 0; s0 < Sr; s0 += 8) {
+    uint4 raw[8];
+    float ws[8];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = fmaf(ws, to_f32(val[v]), acc[v]);
+    for (int u = 0; u < 8; ++u) {
+      const bool in = s0 + u < Sr;
+      ws[u] = in ? w[t * Sr + s0 + u] : 0.f;
+      raw[u] = in ? *reinterpret_cast<const uint4*>(zt + (int64_t)(s0 + u) * d_h)
+                  : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const T* val = reinterpret_cast<const T*>(&raw[u]);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(ws[u], to_f32(val[v]), acc[v]);
+    }
   }
   uint4 out;
   T* o = reinterpret_cast<T*>(&out);
