@@ -80,6 +80,20 @@ def attention_traffic(workload: str):
     return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
 
 
+def reduce_max_over_ranks(values, dist, device):
+    """Each value's maximum over all ranks (times of a multi-GPU run are the slowest
+    rank's). `dist` is torch.distributed with an initialised process group."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, total_ms: float, steps: int):
+    """Tokens of all ranks per second of the (max-over-ranks) time of one step."""
+    return tokens_per_rank * world / (total_ms / steps / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -318,11 +332,8 @@ def bench_ours(args, rank, world, dist):
 
     att_i = [G.gqe_stage_name(i) for i in range(G.GQE_NUM_STAGES)].index("attention")
     if dist:
-        import torch.distributed as td
-        t = torch.tensor([total_ms, totalE_ms, e2e_ms, stage_ms[att_i]], device="cuda",
-                         dtype=torch.float64)
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        total_ms, totalE_ms, e2e_ms, att_ms_tot = [float(v) for v in t.cpu()]
+        total_ms, totalE_ms, e2e_ms, att_ms_tot = reduce_max_over_ranks(
+            [total_ms, totalE_ms, e2e_ms, stage_ms[att_i]], dist, "cuda")
     else:
         att_ms_tot = float(stage_ms[att_i])
 
@@ -330,7 +341,7 @@ def bench_ours(args, rank, world, dist):
     ms = total_ms / args.steps
     msE = totalE_ms / args.steps
     tokens = wl.M * world
-    value = tokens / (total_ms / args.steps / 1e3)
+    value = whole_job_tokens_per_s(wl.M, world, total_ms, args.steps)
     flops = wl.active_flops()
     S = wl.n_streams
     att_flops = (2.0 * wl.B * wl.d_h * wl.T * (wl.T + 1) * S if wl.causal

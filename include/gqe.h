@@ -196,6 +196,18 @@ gqe_status gqe_route_static(const float* logits, int M, int N, int G, int k, int
  */
 gqe_status gqe_exp2_fma(const float* in, float* out, int n, void* stream);
 
+/*
+ * gqe_selftest_timeout — diagnostic of the failure-detection path (failure made on purpose,
+ * without any GPU fault): launches one warp that waits, with the bounded mbarrier wait the
+ * pipeline kernels use and an iteration cap of `spin` (>= 1), on a barrier phase that nothing
+ * completes. When the cap runs out the warp writes the timeout code into h's device status
+ * word, as a pipeline kernel that gave up would, and returns. The next
+ * gqe_check_device_status(h) reports GQE_ERR_TIMEOUT and clears the word; the handle and
+ * the CUDA context stay usable. Stream-ordered; GQE_ERR_INVALID_ARG for a null handle or
+ * spin < 1.
+ */
+gqe_status gqe_selftest_timeout(gqe_handle h, int64_t spin, void* stream);
+
 /* gqe_destroy — free the handle and its workspace (synchronises the device first). */
 void gqe_destroy(gqe_handle h);
 

@@ -23,7 +23,7 @@ TENSORS = {"K": 0, "V": 1, "Q": 2, "Z": 3, "PSEL": 4, "W": 5, "LOGITS": 6}
 EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
-            "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma")
+            "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma", "gqe_selftest_timeout")
 GQE_NUM_STAGES = 6
 
 
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     lib.gqe_route_static.restype = I
     lib.gqe_exp2_fma.argtypes = [P, P, I, P]
     lib.gqe_exp2_fma.restype = I
+    lib.gqe_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
+    lib.gqe_selftest_timeout.restype = I
     return lib
 
 
@@ -141,6 +143,11 @@ def gqe_route_static(logits, M, N, G, k, sel, gates, counts, mean_prob, aux_loss
     _check(lib.gqe_route_static(_ptr(logits), M, N, G, k, _ptr(sel), _ptr(gates), _ptr(counts),
                                 _ptr(mean_prob), _ptr(aux_loss), _stream(stream)),
            "gqe_route_static")
+
+
+def gqe_selftest_timeout(h, spin: int, stream=None) -> None:
+    """Makes one bounded device wait run out on purpose (see include/gqe.h)."""
+    _check(lib.gqe_selftest_timeout(h, spin, _stream(stream)), "gqe_selftest_timeout")
 
 
 def gqe_exp2_fma(inp, out, stream=None) -> None:
