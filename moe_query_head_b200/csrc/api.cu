@@ -61,11 +61,11 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.counts = (int32_t*)take((size_t)N * 4);
   w.mean_prob = (float*)take((size_t)N * 4);
   w.offsets = (int32_t*)take((size_t)(N + 1) * 4);
-  w.bucket = (int32_t*)take((size_t)M * Gk * 4);
+  w.bucket = (int32_t*)take((size_t)M * N * 4);  // expert e owns slots [e M, (e + 1) M)
   w.tile_list = (int2*)take((size_t)((M * Gk + 127) / 128 + N + 1) * sizeof(int2));
   w.tile_count = (int32_t*)take(16);
   w.attn_counter = (int32_t*)take(16);
-  w.grid_sync = (int32_t*)take(16);
+  w.cursor = (int32_t*)take((kMaxExperts + 4) * 4);
   w.status = (int32_t*)take(16);
   w.wcat = take((size_t)(N + (2 * G + 1) * d_h) * dim * esz);
   (void)dim;

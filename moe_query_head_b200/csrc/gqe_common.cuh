@@ -59,12 +59,14 @@ struct Workspace {
   float* part_prob = nullptr;      // [nblk, N]
   int32_t* counts = nullptr;       // [N]
   float* mean_prob = nullptr;      // [N]
-  int32_t* offsets = nullptr;      // [N + 1] bucket start of each expert
-  int32_t* bucket = nullptr;       // [M * G * k] entries (token << 3) | rank, per expert
+  int32_t* offsets = nullptr;      // [N + 1] bucket start of each expert (e M)
+  int32_t* bucket = nullptr;       // [N * M] entries (token << 3) | rank; expert e's run of
+                                   // counts[e] entries starts at e M
   int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* attn_counter = nullptr; // attention work-item counter
-  int32_t* grid_sync = nullptr;    // grid-barrier counters of the fused routing kernel
+  int32_t* cursor = nullptr;       // [kMaxExperts] bucket cursors, then the routing ticket
+                                   // (zero between calls)
   int32_t* status = nullptr;       // device status word
   void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
   void* base = nullptr;            // the single allocation
@@ -87,8 +89,6 @@ struct gqe_ctx {
   int n_stage_events = 0;
   // state of the last forward
   int last_M = 0, last_S = 0, last_Do = 0, last_launches = 0;
-  // resident-CTA capacity of the fused routing kernel (0 until its first launch)
-  int route_cap = 0;
 };
 
 namespace gqe {

@@ -224,58 +224,45 @@ bucket_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ base,
 }
 
 // ---------------------------------------------------------------------------------------
-// The whole routing stage in one cooperative launch: selection, the per-expert statistics
-// and Switch loss, the expert buckets and the routed-projection tile list. Persistent CTAs
-// of kFusedThreads (all resident, guaranteed by the cooperative launch) take blocks of
-// kRouteBlock tokens in turn; two grid barriers separate the phases. Per token and group
-// the arithmetic is that of select_block (same operations in the same order), so the
-// selections, gates and statistics equal route_select_kernel's; only the work is spread
-// over one thread per (token, group) and the loads are batched.
+// The whole routing stage in one pass, without a grid barrier: selection, the expert
+// buckets, the per-expert statistics and Switch loss, and the routed-projection tile list.
+// CTAs of kFusedThreads take blocks of kRouteBlock tokens. Per token and group the
+// arithmetic is that of select_block (same operations in the same order), so selections,
+// gates and statistics equal route_select_kernel's; the work is spread over one thread per
+// (token, group).
+//
+// Buckets: expert e owns slots [e M, e M + count_e) of the bucket array (room for every
+// token). A block claims a contiguous run of each expert's slots with one integer atomic on
+// the expert's cursor, so the order of tokens inside a bucket depends on scheduling; every
+// routed query row is computed on its own (its value does not depend on which rows share
+// its tile), so the results do not. The last CTA to finish (an atomic ticket) turns the
+// cursors into counts, reduces the per-block probability sums in block order (the same
+// arithmetic as the scan of route_scan_aux_kernel), writes the Switch loss and the tile
+// list, and sets the cursors and the ticket back to zero for the next call.
 // ---------------------------------------------------------------------------------------
 constexpr int kFusedThreads = 512;
 
-// Dynamic shared memory of the fused kernel for N experts in G groups.
+// Scratch after the selection arrays: the bucket phase's arrays, the block's counts, and
+// the last CTA's reduction arrays.
+__host__ __device__ inline int fused_bucket_bytes(int N) {
+  return ((kRouteBlock * N + 15) / 16 * 16 + 4 * N + 4 * N * (kRouteBlock / 32) + 15) / 16 * 16;
+}
+constexpr int kStatsBytes = 8 * kFusedThreads + 8 * kMaxExperts + 4 * kFusedThreads +
+                            4 * kMaxExperts + 2 * 4 * (kMaxExperts + 1);
 __host__ __device__ inline int fused_smem_bytes(int N, int G) {
   const int sel_bytes = kRouteBlock * N * 4 + kRouteBlock * G * 4 + kRouteBlock * N;
-  const int bucket_bytes = kRouteBlock * N + 4 * N + 4 * N * (kRouteBlock / 32);
-  const int scan_bytes = 8 * kFusedThreads + 8 * kMaxExperts + 4 * kFusedThreads + 12 * (kMaxExperts + 1);
-  const int a = (sel_bytes + 15) / 16 * 16;
-  return a + (bucket_bytes > scan_bytes ? bucket_bytes : scan_bytes) + 64;
-}
-
-// Grid-wide barrier on a counter that is zero at launch; the i-th barrier waits for
-// i * gridDim.x arrivals. Bounded: gives up after `spin` polls and reports it.
-__device__ bool grid_barrier(int32_t* ctr, int target, int64_t spin) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1);
-    int ok = 0;
-    for (int64_t i = 0; i < spin; ++i) {
-      int v;
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-      if (v >= target) {
-        ok = 1;
-        break;
-      }
-      __nanosleep(32);
-    }
-    __threadfence();
-    s_ok = ok;
-  }
-  __syncthreads();
-  return s_ok != 0;
+  return (sel_bytes + 15) / 16 * 16 + fused_bucket_bytes(N) + 4 * kMaxExperts + kStatsBytes + 64;
 }
 
 // Selection of one token block, one thread per (token, group). Leaves the probabilities in
-// s_p [128][N], the chosen experts' ranks + 1 in s_hit [128][N] (0 = not chosen) and writes
-// sel / p_sel / gates / w and the block's part_counts / part_prob.
+// s_p [128][N], the chosen experts' ranks + 1 in s_hit [128][N] (0 = not chosen) and the
+// block's per-expert token counts in s_count [N]; writes sel / p_sel / gates / w and the
+// block's part_counts / part_prob.
 __device__ void fused_select(const float* __restrict__ logits, int blk, int M, int N, int G,
                              int k, int32_t* __restrict__ sel, float* __restrict__ psel,
                              float* __restrict__ gates, float* __restrict__ wslot,
                              int32_t* __restrict__ part_counts, float* __restrict__ part_prob,
-                             float* s_p, unsigned char* s_hit, float* s_psum) {
+                             float* s_p, unsigned char* s_hit, float* s_psum, int* s_count) {
   const int E = N / G;
   const int tid = threadIdx.x;
   const int t0 = blk * kRouteBlock;
@@ -362,117 +349,20 @@ __device__ void fused_select(const float* __restrict__ logits, int blk, int M, i
     }
     part_prob[(int64_t)blk * N + tid] = ps;
     part_counts[(int64_t)blk * N + tid] = c;
+    s_count[tid] = c;
   }
   __syncthreads();
-}
-
-// Scan of the per-block statistics by one CTA. Thread (e, c) sums a fixed run of router
-// blocks for expert e (kFusedThreads / N threads per expert, loads in batches of eight);
-// the runs combine in run order (probabilities in double), so the result does not depend
-// on scheduling. Writes counts / mean_prob / offsets and the Switch loss
-//   L = (1/G) sum_g E sum_j f_{g,j} Pbar_{g,j},  f = c / (M k),  Pbar = prob_sum / M,
-// turns part_counts into each (block, expert)'s first bucket slot, and lists the
-// routed-projection tiles: each expert's bucket cut into runs of 128 slots.
-__device__ void fused_scan(int32_t* __restrict__ part_counts, const float* __restrict__ part_prob,
-                           int nblk, int M, int N, int G, int k, int32_t* __restrict__ counts,
-                           float* __restrict__ mean_prob, int32_t* __restrict__ offsets,
-                           float* __restrict__ aux_out, int2* __restrict__ tile_list,
-                           int32_t* __restrict__ tile_count, uint8_t* smem) {
-  double* s_ppart = reinterpret_cast<double*>(smem);                 // [kFusedThreads]
-  double* s_term = s_ppart + kFusedThreads;                          // [kMaxExperts]
-  int* s_cpart = reinterpret_cast<int*>(s_term + kMaxExperts);      // [kFusedThreads]
-  int* s_cnt = s_cpart + kFusedThreads;                              // [kMaxExperts]
-  int* s_off = s_cnt + kMaxExperts;                                  // [kMaxExperts + 1]
-  int* s_nt = s_off + kMaxExperts + 1;                               // [kMaxExperts + 1]
-  const int tid = threadIdx.x;
-  const int tpe = max(1, kFusedThreads / N);  // threads per expert
-  const int e = tid / tpe, c = tid % tpe;
-  const bool act = e < N;
-  const int chunk = (nblk + tpe - 1) / tpe;
-  const int b0 = min(nblk, c * chunk), b1 = min(nblk, b0 + chunk);
-  if (act) {
-    int cs = 0;
-    double ps = 0.0;
-    for (int b = b0; b < b1; b += 8) {
-      int cv[8];
-      float pv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool in = b + u < b1;
-        cv[u] = in ? __ldcg(part_counts + (int64_t)(b + u) * N + e) : 0;
-        pv[u] = in ? __ldcg(part_prob + (int64_t)(b + u) * N + e) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        cs += cv[u];
-        if (b + u < b1) ps += (double)pv[u];
-      }
-    }
-    s_cpart[tid] = cs;
-    s_ppart[tid] = ps;
-  }
-  __syncthreads();
-  if (act && c == 0) {
-    int tot = 0;
-    double ps = 0.0;
-    for (int i = 0; i < tpe; ++i) {
-      const int v = s_cpart[tid + i];
-      s_cpart[tid + i] = tot;  // exclusive prefix of the runs
-      tot += v;
-      ps += s_ppart[tid + i];
-    }
-    counts[e] = tot;
-    mean_prob[e] = (float)(ps / M);
-    s_cnt[e] = tot;
-    s_term[e] = (double)(N / G) * ((double)tot / ((double)M * k)) * (ps / M);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int off = 0, nt = 0;
-    for (int x = 0; x < N; ++x) {
-      s_off[x] = off;
-      offsets[x] = off;
-      s_nt[x] = nt;
-      nt += (s_cnt[x] + 127) / 128;
-      off += s_cnt[x];
-    }
-    offsets[N] = off;
-    *tile_count = nt;
-    if (aux_out != nullptr) {
-      double L = 0.0;
-      for (int x = 0; x < N; ++x) L += s_term[x];
-      aux_out[0] = (float)(L / G);
-    }
-  }
-  __syncthreads();
-  if (act) {
-    int run = s_off[e] + s_cpart[tid];
-    for (int b = b0; b < b1; b += 8) {
-      int cv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        cv[u] = b + u < b1 ? __ldcg(part_counts + (int64_t)(b + u) * N + e) : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (b + u < b1) part_counts[(int64_t)(b + u) * N + e] = run;
-        run += cv[u];
-      }
-    }
-  }
-  for (int x = tid; x < N; x += kFusedThreads) {
-    const int nt = (s_cnt[x] + 127) / 128;
-    for (int i = 0; i < nt; ++i) tile_list[s_nt[x] + i] = make_int2(x, s_off[x] + i * 128);
-  }
 }
 
 // Bucket entries of one token block: entry (t << 3) | r for every selection, at the
 // expert's base slot for this block plus the number of earlier tokens of the block that
-// chose the same expert (so each expert's bucket is in token order); one warp ballot per
-// expert gives those counts. s_hit holds the block's ranks + 1 if `have_hits`, else they are
-// read back from sel.
+// chose the same expert; one warp ballot per expert gives those counts. s_hit holds the
+// block's ranks + 1 if `have_hits`, else they are read back from sel; the bases are in
+// shared memory if `have_bases`, else read from `base` [blk][N].
 __device__ void fused_bucket(const int32_t* __restrict__ sel, const int32_t* __restrict__ base,
                              int blk, int M, int N, int G, int k, int32_t* __restrict__ bucket,
-                             unsigned char* s_hit, bool have_hits, uint8_t* scratch) {
+                             unsigned char* s_hit, bool have_hits, bool have_bases,
+                             uint8_t* scratch) {
   constexpr int kWarps = kRouteBlock / 32;
   unsigned char* s_lb = scratch;                                      // [128][N] lanes before
   int* s_base = reinterpret_cast<int*>(scratch + ((kRouteBlock * N + 15) / 16 * 16));  // [N]
@@ -492,7 +382,7 @@ __device__ void fused_bucket(const int32_t* __restrict__ sel, const int32_t* __r
             (unsigned char)(r + 1);
     }
   }
-  if (tid < N) s_base[tid] = __ldcg(base + (int64_t)blk * N + tid);
+  if (!have_bases && tid < N) s_base[tid] = __ldcg(base + (int64_t)blk * N + tid);
   __syncthreads();
   if (tid < kRouteBlock) {
     for (int e = 0; e < N; ++e) {
@@ -514,6 +404,76 @@ __device__ void fused_bucket(const int32_t* __restrict__ sel, const int32_t* __r
   __syncthreads();
 }
 
+// The last CTA's reduction. Thread (e, c) sums a fixed run of router blocks for expert e
+// (kFusedThreads / N threads per expert, loads in batches of eight); the runs combine in run
+// order (probabilities in double), so the result does not depend on scheduling. Writes
+// counts (the cursors' final values), mean_prob, offsets (e M), the Switch loss
+//   L = (1/G) sum_g E sum_j f_{g,j} Pbar_{g,j},  f = c / (M k),  Pbar = prob_sum / M,
+// and the routed-projection tiles (each expert's bucket cut into runs of 128 slots), then
+// zeroes the cursors.
+__device__ void finalize_routing(const float* __restrict__ part_prob, int nblk, int M, int N,
+                                 int G, int k, int32_t* __restrict__ cursor,
+                                 int32_t* __restrict__ counts, float* __restrict__ mean_prob,
+                                 int32_t* __restrict__ offsets, float* __restrict__ aux_out,
+                                 int2* __restrict__ tile_list, int32_t* __restrict__ tile_count,
+                                 uint8_t* st) {
+  double* s_ppart = reinterpret_cast<double*>(st);                   // [kFusedThreads]
+  double* s_term = s_ppart + kFusedThreads;                          // [kMaxExperts]
+  int* s_cnt = reinterpret_cast<int*>(s_term + kMaxExperts);        // [kMaxExperts]
+  int* s_nt = s_cnt + kMaxExperts;                                   // [kMaxExperts + 1]
+  const int tid = threadIdx.x;
+  const int tpe = max(1, kFusedThreads / N);
+  const int e = tid / tpe, c = tid % tpe;
+  const bool act = e < N;
+  const int chunk = (nblk + tpe - 1) / tpe;
+  const int b0 = min(nblk, c * chunk), b1 = min(nblk, b0 + chunk);
+  if (act) {
+    double ps = 0.0;
+    for (int b = b0; b < b1; b += 8) {
+      float pv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        pv[u] = b + u < b1 ? __ldcg(part_prob + (int64_t)(b + u) * N + e) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (b + u < b1) ps += (double)pv[u];
+    }
+    s_ppart[tid] = ps;
+  }
+  if (tid < N) s_cnt[tid] = __ldcg(cursor + tid);
+  __syncthreads();
+  if (act && c == 0) {
+    double ps = 0.0;
+    for (int i = 0; i < tpe; ++i) ps += s_ppart[tid + i];
+    const int tot = s_cnt[e];
+    counts[e] = tot;
+    offsets[e] = e * M;
+    mean_prob[e] = (float)(ps / M);
+    s_term[e] = (double)(N / G) * ((double)tot / ((double)M * k)) * (ps / M);
+    cursor[e] = 0;  // ready for the next call
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nt = 0;
+    for (int x = 0; x < N; ++x) {
+      s_nt[x] = nt;
+      nt += (s_cnt[x] + 127) / 128;
+    }
+    offsets[N] = N * M;
+    *tile_count = nt;
+    if (aux_out != nullptr) {
+      double L = 0.0;
+      for (int x = 0; x < N; ++x) L += s_term[x];
+      aux_out[0] = (float)(L / G);
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < N; x += kFusedThreads) {
+    const int nt = (s_cnt[x] + 127) / 128;
+    for (int i = 0; i < nt; ++i) tile_list[s_nt[x] + i] = make_int2(x, x * M + i * 128);
+  }
+}
+
 __global__ void __launch_bounds__(kFusedThreads)
 route_fused_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
                    int32_t* __restrict__ sel, float* __restrict__ psel,
@@ -522,76 +482,58 @@ route_fused_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
                    int32_t* __restrict__ counts, float* __restrict__ mean_prob,
                    int32_t* __restrict__ offsets, float* __restrict__ aux_out,
                    int32_t* __restrict__ bucket, int2* __restrict__ tile_list,
-                   int32_t* __restrict__ tile_count, int32_t* __restrict__ grid_ctr,
-                   int32_t* __restrict__ status, int64_t spin) {
+                   int32_t* __restrict__ tile_count, int32_t* __restrict__ cursor,
+                   int32_t* __restrict__ ticket) {
   extern __shared__ __align__(16) uint8_t dsmem[];
+  __shared__ int s_last;
   float* s_p = reinterpret_cast<float*>(dsmem);                         // [128][N]
   float* s_psum = s_p + kRouteBlock * N;                                // [128][G]
   unsigned char* s_hit = reinterpret_cast<unsigned char*>(s_psum + kRouteBlock * G);  // [128][N]
   uint8_t* scratch = dsmem + ((kRouteBlock * N * 4 + kRouteBlock * G * 4 + kRouteBlock * N + 15) / 16 * 16);
+  int* s_base = reinterpret_cast<int*>(scratch + ((kRouteBlock * N + 15) / 16 * 16));  // [N]
+  int* s_count = reinterpret_cast<int*>(scratch + fused_bucket_bytes(N));             // [N]
+  uint8_t* st = scratch + fused_bucket_bytes(N) + 4 * kMaxExperts;
   const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x)
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     fused_select(logits, blk, M, N, G, k, sel, psel, gates, wslot, part_counts, part_prob, s_p,
-                 s_hit, s_psum);
-  if (!grid_barrier(grid_ctr, gridDim.x, spin)) {
-    if (threadIdx.x == 0) atomicExch(status, kStatusTimeout);
-    return;
+                 s_hit, s_psum, s_count);
+    // claim this block's run of slots in every expert's bucket
+    if (threadIdx.x < N)
+      s_base[threadIdx.x] = threadIdx.x * M + atomicAdd(&cursor[threadIdx.x], s_count[threadIdx.x]);
+    __syncthreads();
+    fused_bucket(sel, nullptr, blk, M, N, G, k, bucket, s_hit, true, true, scratch);
   }
-  if (blockIdx.x == 0)
-    fused_scan(part_counts, part_prob, nblk, M, N, G, k, counts, mean_prob, offsets, aux_out,
-               tile_list, tile_count, scratch);
-  if (!grid_barrier(grid_ctr, 2 * gridDim.x, spin)) {
-    if (threadIdx.x == 0) atomicExch(status, kStatusTimeout);
-    return;
+  // the last CTA to get here finishes the statistics
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
   }
-  // a CTA that selected a single block still holds that block's ranks in shared memory
-  const bool single = nblk <= (int)gridDim.x;
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x)
-    fused_bucket(sel, part_counts, blk, M, N, G, k, bucket, s_hit, single, scratch);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  finalize_routing(part_prob, nblk, M, N, G, k, cursor, counts, mean_prob, offsets, aux_out,
+                   tile_list, tile_count, st);
+  if (threadIdx.x == 0) *ticket = 0;
 }
 
 int launch_route_fused(gqe_ctx* h, int M, float* aux_out, cudaStream_t st) {
   const int smem = fused_smem_bytes(h->N, h->G);
-  if (h->route_cap == 0) {
-    int per_sm = 0;
+  static bool configured = false;
+  if (!configured) {
+    // the largest size any shape can ask for, so that one setting serves every handle
     if (cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel, kFusedThreads,
-                                                      smem) != cudaSuccess ||
-        per_sm < 1)
+                             fused_smem_bytes(kMaxExperts, kMaxExperts)) != cudaSuccess)
       return -1;
-    h->route_cap = per_sm * h->num_sms;
+    configured = true;
   }
   const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
-  int grid = nblk < h->route_cap ? nblk : h->route_cap;
-  if (cudaMemsetAsync(h->ws.grid_sync, 0, 16, st) != cudaSuccess) return -1;
-  const float* logits = h->ws.logits;
-  int32_t* sel = h->ws.sel;
-  float* psel = h->ws.psel;
-  float* gates = h->ws.gates;
-  float* wslot = h->ws.w;
-  int32_t* pc = h->ws.part_counts;
-  float* pp = h->ws.part_prob;
-  int32_t* counts = h->ws.counts;
-  float* mp = h->ws.mean_prob;
-  int32_t* offs = h->ws.offsets;
-  int32_t* bucket = h->ws.bucket;
-  int2* tl = h->ws.tile_list;
-  int32_t* tc = h->ws.tile_count;
-  int32_t* gs = h->ws.grid_sync;
-  int32_t* status = h->ws.status;
-  // The grid barriers wait only for co-resident CTAs of this launch (the cooperative launch
-  // guarantees that they all run), so they use a fixed generous bound rather than the
-  // handle's spin limit: a test that shortens the other kernels' waits leaves the routing
-  // complete and consistent.
-  int64_t spin = (int64_t)1 << 26;
-  int N = h->N, G = h->G, k = h->k;
-  void* args[] = {&logits, &M, &N, &G, &k, &sel, &psel, &gates, &wslot, &pc, &pp, &counts,
-                  &mp, &offs, &aux_out, &bucket, &tl, &tc, &gs, &status, &spin};
-  if (cudaLaunchCooperativeKernel((const void*)route_fused_kernel, dim3(grid),
-                                  dim3(kFusedThreads), args, smem, st) != cudaSuccess)
-    return -1;
-  return 1;
+  const int grid = nblk < 4 * h->num_sms ? nblk : 4 * h->num_sms;
+  route_fused_kernel<<<grid, kFusedThreads, smem, st>>>(
+      h->ws.logits, M, h->N, h->G, h->k, h->ws.sel, h->ws.psel, h->ws.gates, h->ws.w,
+      h->ws.part_counts, h->ws.part_prob, h->ws.counts, h->ws.mean_prob, h->ws.offsets, aux_out,
+      h->ws.bucket, h->ws.tile_list, h->ws.tile_count, h->ws.cursor, h->ws.cursor + kMaxExperts);
+  return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
 int launch_route_select(gqe_ctx* h, int M, cudaStream_t st) {

@@ -104,10 +104,11 @@ __global__ void __launch_bounds__(256) dense_proj_kernel(const T* __restrict__ x
 template <typename T>
 __global__ void __launch_bounds__(256)
 qproj_kernel(const T* __restrict__ x, int M, int K, const T* __restrict__ Wq, int d_h, int E,
-             int k, const int32_t* __restrict__ offsets, const int32_t* __restrict__ bucket,
+             int k, const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
+             const int32_t* __restrict__ bucket,
              T* __restrict__ Q) {
   const int e = blockIdx.z;
-  const int beg = offsets[e], cnt = offsets[e + 1] - beg;
+  const int beg = offsets[e], cnt = counts[e];
   const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
   if (m0 >= cnt) return;
   float acc[4][4];
@@ -338,12 +339,12 @@ int launch_simt_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStr
   if (h->dtype == GQE_F32)
     qproj_kernel<float><<<grid, 256, 0, st>>>(
         static_cast<const float*>(x), M, h->dim, static_cast<const float*>(W_q), h->d_h, h->E,
-        h->k, h->ws.offsets, h->ws.bucket, static_cast<float*>(h->ws.Q));
+        h->k, h->ws.offsets, h->ws.counts, h->ws.bucket, static_cast<float*>(h->ws.Q));
   else
     qproj_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), M, h->dim,
         static_cast<const __nv_bfloat16*>(W_q), h->d_h, h->E, h->k, h->ws.offsets,
-        h->ws.bucket, static_cast<__nv_bfloat16*>(h->ws.Q));
+        h->ws.counts, h->ws.bucket, static_cast<__nv_bfloat16*>(h->ws.Q));
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

@@ -71,7 +71,8 @@ struct Params {
   const int32_t* bucket;                // entries (t << 3) | r
   const int2* tile_list;                // (expert, first bucket slot) per tile
   const int32_t* tile_count;            // number of tiles (device)
-  const int32_t* offsets;               // bucket offsets [N + 1]
+  const int32_t* offsets;               // bucket start of each expert [N]
+  const int32_t* counts;                // entries in each expert's bucket [N]
   __nv_bfloat16* Q;                     // query streams [S, M, d_h]
   int E, k, d_h;
   int32_t* status;
@@ -93,7 +94,7 @@ __device__ __forceinline__ TileInfo tile_info(const Params& P, int tile) {
     const int2 t = P.tile_list[tile];
     ti.p = t.x;
     ti.m0 = t.y;
-    const int end = P.offsets[t.x + 1];
+    const int end = P.offsets[t.x] + P.counts[t.x];
     ti.rows = min(BM, end - t.y);
     ti.n0 = 0;
     ti.n = P.prob[0].box_n;
@@ -204,7 +205,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       uint32_t g = 0;  // position in the CTA's stage sequence
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         const int2 t = P.tile_list[tile];
-        const int n = min(BM, P.offsets[t.x + 1] - t.y);
+        const int n = min(BM, P.offsets[t.x] + P.counts[t.x] - t.y);
         const uint32_t b_bytes = (uint32_t)P.prob[0].box_n * BK * 2;
         // source rows of this lane: r = 4 i + lane / 8 (rows past the tile's end repeat
         // its first row: computed, never stored)
@@ -528,6 +529,7 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStrea
   P.tile_list = h->ws.tile_list;
   P.tile_count = h->ws.tile_count;
   P.offsets = h->ws.offsets;
+  P.counts = h->ws.counts;
   P.Q = static_cast<__nv_bfloat16*>(h->ws.Q);
   P.E = h->E;
   P.k = h->k;
