@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_t16k", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default=None, choices=["gqe", "weighted_concat", "hard_concat"],
+                    help="output construction (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8192,
                     help="query rows in the oracle's bounded sample")
@@ -235,6 +237,8 @@ def bench_ours(args, rank, world, dist):
     from moe_query_head_b200 import gqe as G
 
     wl = W.WORKLOADS[args.workload]
+    if args.variant:
+        wl = wl.with_(variant=args.variant)
     inp = W.generate(wl)
     dev = _upload(inp, torch)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
@@ -399,6 +403,8 @@ def main():
         if rank != 0:
             return 0
         wl = W.WORKLOADS[args.workload]
+        if args.variant:
+            wl = wl.with_(variant=args.variant)
         inp = W.generate(wl)
         rows = max(16, min(args.cpu_rows, 256))
         for _ in range(args.warmup):
