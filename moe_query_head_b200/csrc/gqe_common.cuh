@@ -20,6 +20,32 @@ constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch. The forward's kernels are launched with it: a kernel may
+// begin (its set-up: barriers, TMEM, tensor-map prefetch) while the previous kernel on the
+// stream finishes, and waits for that kernel's completion and memory (pdl_wait) before it
+// touches global memory. pdl_allow_next lets the next kernel begin launching.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// ---------------------------------------------------------------------------------------
 // Element access helpers: every kernel computes in fp32; storage is float or bf16.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }

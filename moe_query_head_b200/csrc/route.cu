@@ -486,6 +486,8 @@ route_fused_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
                    int32_t* __restrict__ ticket) {
   extern __shared__ __align__(16) uint8_t dsmem[];
   __shared__ int s_last;
+  pdl_wait();  // the router logits are complete from here on
+  pdl_allow_next();
   float* s_p = reinterpret_cast<float*>(dsmem);                         // [128][N]
   float* s_psum = s_p + kRouteBlock * N;                                // [128][G]
   unsigned char* s_hit = reinterpret_cast<unsigned char*>(s_psum + kRouteBlock * G);  // [128][N]
@@ -529,11 +531,14 @@ int launch_route_fused(gqe_ctx* h, int M, float* aux_out, cudaStream_t st) {
   }
   const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
   const int grid = nblk < 4 * h->num_sms ? nblk : 4 * h->num_sms;
-  route_fused_kernel<<<grid, kFusedThreads, smem, st>>>(
-      h->ws.logits, M, h->N, h->G, h->k, h->ws.sel, h->ws.psel, h->ws.gates, h->ws.w,
-      h->ws.part_counts, h->ws.part_prob, h->ws.counts, h->ws.mean_prob, h->ws.offsets, aux_out,
-      h->ws.bucket, h->ws.tile_list, h->ws.tile_count, h->ws.cursor, h->ws.cursor + kMaxExperts);
-  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+  const float* logits = h->ws.logits;
+  return launch_pdl(route_fused_kernel, dim3(grid), dim3(kFusedThreads), smem, st, logits, M,
+                    h->N, h->G, h->k, h->ws.sel, h->ws.psel, h->ws.gates, h->ws.w,
+                    h->ws.part_counts, h->ws.part_prob, h->ws.counts, h->ws.mean_prob,
+                    h->ws.offsets, aux_out, h->ws.bucket, h->ws.tile_list, h->ws.tile_count,
+                    h->ws.cursor, h->ws.cursor + kMaxExperts) == cudaSuccess
+             ? 1
+             : -1;
 }
 
 int launch_route_select(gqe_ctx* h, int M, cudaStream_t st) {

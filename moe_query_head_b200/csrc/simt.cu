@@ -237,6 +237,8 @@ template <typename T>
 __global__ void slot_kernel(T* __restrict__ Z, const float* __restrict__ w, int M, int Sr,
                             int d_h, int Do) {
   constexpr int VEC = 16 / sizeof(T);
+  pdl_wait();  // Z and the slot weights are complete from here on
+  pdl_allow_next();
   const int per_tok = d_h / VEC;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)M * per_tok) return;
@@ -363,8 +365,11 @@ int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st) {
     slot_kernel<float><<<blocks, 256, 0, st>>>(static_cast<float*>(h->ws.Z), h->ws.w, M, Sr,
                                                h->d_h, Do);
   else
-    slot_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(h->ws.Z),
-                                                       h->ws.w, M, Sr, h->d_h, Do);
+    return launch_pdl(slot_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                      static_cast<__nv_bfloat16*>(h->ws.Z), static_cast<const float*>(h->ws.w),
+                      M, Sr, h->d_h, Do) == cudaSuccess
+               ? 1
+               : -1;
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

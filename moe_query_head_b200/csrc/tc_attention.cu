@@ -98,7 +98,8 @@ struct Params {
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
   int nq, items;
   float scale_log2;
-  int* next_item;  // global item counter (zero at launch); CTAs take items from it
+  int* next_item;  // [2] item counter and exit counter (zero at launch; the last CTA to
+                   // leave sets both back to zero)
   int32_t* status;
   int64_t spin;
 };
@@ -212,6 +213,8 @@ attn_kernel(const __grid_constant__ Params P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // Q, K, V and (weighted_concat) p_sel are complete from here on
+  pdl_allow_next();
 
   // MMA and softmax warps: the next item index from the ring (warp-collective); the slot
   // is released as soon as it has been read. -1 means no work is left.
@@ -600,6 +603,11 @@ attn_kernel(const __grid_constant__ Params P) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  // every CTA has taken its last item: the last one to leave resets the counters
+  if (threadIdx.x == 0 && atomicAdd(P.next_item + 1, 1) == (int)gridDim.x - 1) {
+    P.next_item[0] = 0;
+    P.next_item[1] = 0;
+  }
 }
 
 template <int DH>
@@ -643,9 +651,9 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
   const int slots = C::CTAS * h->num_sms;
   const int grid = P.items < slots ? P.items : slots;
   P.next_item = h->ws.attn_counter;
-  if (cudaMemsetAsync(h->ws.attn_counter, 0, sizeof(int), st) != cudaSuccess) return -1;
-  attn_kernel<DH><<<grid, THREADS, C::SMEM, st>>>(P);
-  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+  return launch_pdl(attn_kernel<DH>, dim3(grid), dim3(THREADS), C::SMEM, st, P) == cudaSuccess
+             ? 1
+             : -1;
 }
 
 }  // namespace

@@ -138,7 +138,6 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int total = GATHER ? *P.tile_count : P.total_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -165,6 +164,9 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int KB = (P.K + BK - 1) / BK;
+  pdl_wait();  // the previous kernel's outputs (x, the buckets, Z) are complete from here on
+  pdl_allow_next();
+  const int total = GATHER ? *P.tile_count : P.total_tiles;
 
   if (warp < L::NPROD) {
     // ------------------------------------------------------------------ producers
@@ -451,8 +453,10 @@ int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
       return -1;
     configured[GATHER] = true;
   }
-  tc_gemm_kernel<GATHER><<<grid, Lay<GATHER>::THREADS, SMEM_BYTES, st>>>(P);
-  return cudaGetLastError() == cudaSuccess ? 1 : -1;
+  return launch_pdl(tc_gemm_kernel<GATHER>, dim3(grid), dim3(Lay<GATHER>::THREADS), SMEM_BYTES,
+                    st, P) == cudaSuccess
+             ? 1
+             : -1;
 }
 
 Problem make_problem(int N, OutMap out) {
