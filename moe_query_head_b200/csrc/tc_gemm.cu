@@ -10,10 +10,11 @@
 //                     Overview: only the active query-head computation is reduced).
 //   output projection Z [M, D_o] times W_o [dim, D_o].
 //
-// One persistent kernel, one CTA per SM:
-//   producers  dense: one warp issuing TMA tile loads of A and B. Routed projection: four
+// One persistent kernel, two CTAs per SM (each CTA's pipeline hand-offs, fills and tail are
+// covered by the other CTA's work):
+//   producers  dense: one warp issuing TMA tile loads of A and B. Routed projection: three
 //              warps gathering A rows through registers into the 128-byte swizzled
-//              layout (each warp fills every fourth stage), B by TMA;
+//              layout (each warp fills every third stage), B by TMA;
 //   MMA warp   allocates TMEM; one lane issues tcgen05.mma (128 x BN x 16) and commits;
 //   4 warps    epilogue: tcgen05.ld of the fp32 accumulator, conversion, stores.
 // Shared-memory stages are guarded by full/empty mbarriers; two TMEM accumulators let the
@@ -34,11 +35,16 @@ using namespace tc;
 constexpr int BM = 128;        // tile rows = MMA M = TMEM lanes
 constexpr int BN = 128;        // widest tile (MMA N)
 constexpr int BK = 64;         // one 128-byte swizzle atom of bf16 along K
-constexpr int STAGES = 6;
+constexpr int STAGES = 3;
+constexpr int CTAS_PER_SM = 2;  // shared memory: 2 x ~98 KB; TMEM: 2 x 256 columns
 // Warp roles: producers, one MMA-issuing warp, four epilogue warps.
 template <bool GATHER>
 struct Lay {
-  static constexpr int NPROD = GATHER ? 4 : 1;
+  static constexpr int NPROD = GATHER ? 3 : 1;
+  // A producer warp waits only for the stage it fills next; with more producer warps than
+  // stages one of them could get two uses of a stage ahead of the MMA warp, and a parity
+  // wait cannot tell those phases apart.
+  static_assert(NPROD <= STAGES, "a producer warp could lap the stage ring");
   static constexpr int MMA = NPROD;
   static constexpr int EPI0 = NPROD + 1;
   static constexpr int THREADS = (NPROD + 5) * 32;
@@ -122,7 +128,7 @@ __device__ __forceinline__ void set_timeout(const Params& P, volatile int* abort
 }
 
 template <bool GATHER>
-__global__ void __launch_bounds__(Lay<GATHER>::THREADS, 1)
+__global__ void __launch_bounds__(Lay<GATHER>::THREADS, CTAS_PER_SM)
 tc_gemm_kernel(const __grid_constant__ Params P) {
   using L = Lay<GATHER>;
   extern __shared__ uint8_t smem_raw[];
@@ -196,7 +202,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
         }
       }
     } else {
-      // Four producer warps; warp p fills every fourth stage of the CTA's stage sequence.
+      // NPROD producer warps; warp p fills stages p, p + NPROD, ... of the CTA's stage sequence.
       // A rows are gathered by asynchronous 16-byte copies (cp.async, no registers, many
       // stages in flight): lane l moves chunk l % 8 of rows 4 i + l / 8 (eight lanes per
       // 128-byte row segment: coalesced reads, conflict-free writes into the
@@ -510,7 +516,7 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   P.total_tiles = P.m_tiles * P.tiles_per_m;
   P.status = h->ws.status;
   P.spin = spin_limit(h);
-  const int grid = P.total_tiles < h->num_sms ? P.total_tiles : h->num_sms;
+  const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
   return launch<false>(h, P, grid, st);
 }
 
@@ -541,7 +547,7 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStrea
   P.status = h->ws.status;
   P.spin = spin_limit(h);
   const int max_tiles = (int)(((int64_t)M * h->G * h->k + BM - 1) / BM) + h->N;
-  const int grid = max_tiles < h->num_sms ? max_tiles : h->num_sms;
+  const int grid = min(max_tiles, CTAS_PER_SM * h->num_sms);
   return launch<true>(h, P, grid, st);
 }
 
@@ -561,7 +567,7 @@ int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaS
   P.total_tiles = P.m_tiles * P.tiles_per_m;
   P.status = h->ws.status;
   P.spin = spin_limit(h);
-  const int grid = P.total_tiles < h->num_sms ? P.total_tiles : h->num_sms;
+  const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
   return launch<false>(h, P, grid, st);
 }
 
