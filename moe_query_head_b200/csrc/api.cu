@@ -66,8 +66,8 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.tile_count = (int32_t*)take(16);
   w.attn_counter = (int32_t*)take(16);
   w.cursor = (int32_t*)take((kMaxExperts + 4) * 4);
+  w.psum_fx = (unsigned long long*)take(kMaxExperts * 8);
   w.status = (int32_t*)take(16);
-  w.wcat = take((size_t)(N + (2 * G + 1) * d_h) * dim * esz);
   (void)dim;
   return off;
 }
@@ -220,9 +220,10 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   // bf16: tensor-core (tcgen05) kernels for the projections; fp32: CUDA-core kernels.
   const bool tc = h->dtype == GQE_BF16;
   bool ok = mark() &&
-            add(tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)
+            add(tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, aux_loss, st)
                    : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
-            add(launch_route_fused(h, M, aux_loss, st)) &&
+            // bf16: the routing usually runs in the dense projection's router tiles
+            add(tc && tc_dense_routes(h) ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
             add(tc ? launch_tc_qproj(h, x, M, W_q, st) : launch_simt_qproj(h, x, M, W_q, st)) &&
             add(tc ? launch_tc_attention(h, B, T, S, has_shared, variant, causal, Do, st)
                    : launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&

@@ -91,10 +91,11 @@ struct Workspace {
   int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* attn_counter = nullptr; // attention work-item counter
+  unsigned long long* psum_fx = nullptr;  // [kMaxExperts] probability sums in fixed point
+                                          // (dense-projection routing; zero between calls)
   int32_t* cursor = nullptr;       // [kMaxExperts] bucket cursors, then the routing ticket
                                    // (zero between calls)
   int32_t* status = nullptr;       // device status word
-  void* wcat = nullptr;            // concatenated [W_r; W_k; W_v; W_shared] (bf16 path)
   void* base = nullptr;            // the single allocation
   size_t bytes = 0;
 };
@@ -148,7 +149,9 @@ int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st);
 int launch_simt_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 // tcgen05 paths (bf16)
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, cudaStream_t st);
+                         const void* W_v, const void* W_shared, float* aux_out,
+                         cudaStream_t st);
+bool tc_dense_routes(const gqe_ctx* h);  // launch_tc_dense_proj also routes
 int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,

@@ -51,16 +51,36 @@ struct Lay {
 };
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int B_STAGE_BYTES = BN * BK * 2;
-constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256 +
-                           BM * 4 /*gathered row indices*/;
+// stages, 1024-byte alignment, barriers and flags, the routing statistics' scratch
+constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 + 256 +
+                           16 * (kMaxExperts + 8);
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_PROBLEMS = 4;
+constexpr int MAX_COL_TILES = 32;  // column tiles over all problems of one GEMM
 
 struct Problem {
   int N;        // output columns of this problem
   int n_tiles;  // ceil(N / BN)
   int box_n;    // rows of B per TMA box (<= BN, multiple of 16)
   OutMap out;
+};
+
+// Outputs of the routing done in the dense projection's router tiles (see route_rows).
+struct RouteOut {
+  float* logits_out;     // [M, N] problem 0's output (router logits, fp32)
+  int32_t* sel;          // [M, G, k]
+  float* psel;           // [M, G, k]
+  float* gates;          // [M, G, k]
+  float* wslot;          // [M, G, k]
+  unsigned long long* psum_fx;  // [kMaxExperts] probability sums, fixed point (zero between calls)
+  int32_t* cursor;       // [kMaxExperts] bucket cursors, then the CTA ticket (zero between calls)
+  int32_t* bucket;       // [N * M]
+  int32_t* counts;       // [N]
+  float* mean_prob;      // [N]
+  int32_t* offsets;      // [N + 1]
+  float* aux;            // [1] or null
+  int2* tile_list;
+  int32_t* tile_count;
 };
 
 struct Params {
@@ -70,8 +90,15 @@ struct Params {
   int nprob;
   int M, K;
   int m_tiles;
-  int tiles_per_m;                      // sum of n_tiles over problems
+  int tiles_per_m;                      // column tiles: sum of n_tiles over problems
   int total_tiles;                      // dense: m_tiles * tiles_per_m
+  // (problem, first column) of each column tile. Column-major (col_major): tile t covers
+  // column tile t / m_tiles of row tile t % m_tiles, so the CTAs' round-robin passes deal
+  // out the column tiles in this order (router tiles one per CTA, then the widest) instead
+  // of giving some CTAs only narrow tiles and others only full ones. Otherwise row-major:
+  // row tile t / tiles_per_m, column tile t % tiles_per_m (neighbouring CTAs share A rows).
+  int2 ctile[MAX_COL_TILES];
+  int col_major;
   // routed projection (gather mode)
   const __nv_bfloat16* x;               // A rows gathered from x [M, K]
   const int32_t* bucket;                // entries (t << 3) | r
@@ -80,6 +107,9 @@ struct Params {
   const int32_t* offsets;               // bucket start of each expert [N]
   const int32_t* counts;                // entries in each expert's bucket [N]
   __nv_bfloat16* Q;                     // query streams [S, M, d_h]
+  // dense projection with routing (the ROUTE instance): problem 0 = W_r
+  int G;
+  RouteOut ro;
   int E, k, d_h;
   int32_t* status;
   int64_t spin;
@@ -105,17 +135,20 @@ __device__ __forceinline__ TileInfo tile_info(const Params& P, int tile) {
     ti.n0 = 0;
     ti.n = P.prob[0].box_n;
   } else {
-    const int mt = tile / P.tiles_per_m;
-    int r = tile % P.tiles_per_m;
-    int p = 0;
-    while (r >= P.prob[p].n_tiles) {
-      r -= P.prob[p].n_tiles;
-      ++p;
+    int j, mt;
+    if (P.col_major) {
+      j = tile / P.m_tiles;
+      mt = tile - j * P.m_tiles;
+    } else {
+      mt = tile / P.tiles_per_m;
+      j = tile - mt * P.tiles_per_m;
     }
+    const int2 ct = P.ctile[j];
+    const int p = ct.x;
     ti.p = p;
     ti.m0 = mt * BM;
     ti.rows = min(BM, P.M - ti.m0);
-    ti.n0 = r * BN;
+    ti.n0 = ct.y;
     const int rem = P.prob[p].N - ti.n0;
     ti.n = min(BN, (rem + 15) / 16 * 16);
   }
@@ -127,7 +160,222 @@ __device__ __forceinline__ void set_timeout(const Params& P, volatile int* abort
   atomicExch(P.status, kStatusTimeout);
 }
 
-template <bool GATHER>
+// Fixed-point scale of the per-expert probability sums (integer additions do not depend on
+// their order, so the sums are the same whatever order the warps add them in).
+constexpr double kProbFix = 4294967296.0;  // 2^32
+
+// Routing of a router tile's rows, in the dense projection's epilogue ("GQE: Grouped Query
+// Experts" README, Algorithm Overview: N experts in G groups, the top k of each group by
+// router logit, ties to the lower index; softmax over each group's experts; gist.science
+// summary, Load Balancing). One thread per token (its TMEM lane), N and E = N / G fixed at
+// compile time so every index is static and the logits never leave registers:
+//   - the N fp32 logits come from TMEM; the accumulator is released; the row is stored;
+//   - per group: the top k (k passes of an argmax, ties to the lower index), the softmax
+//     p, the group's selected mass; sel (ascending expert index), p_sel, the gates
+//     p_sel / (group's selected mass) and the slot weights p_sel / (all G k selections);
+//   - per expert, over the warp's 32 tokens: the selection count (a ballot) and the
+//     probability sum (a butterfly), which lane e adds to the expert's totals: its bucket
+//     cursor (the atomic returns the warp's first slot) and, in fixed point, its
+//     probability sum;
+//   - the bucket entries (token << 3) | rank, in lane order within the warp's run.
+// The only memory round trip on this path is that atomic.
+template <int N, int E>
+__device__ void route_rows(const Params& P, uint32_t t_row, int t, bool valid, int lane,
+                           uint64_t* acc_empty) {
+  constexpr int G = N / E;
+  constexpr unsigned all = 0xffffffffu;
+  const RouteOut& R = P.ro;
+  const int k = P.k;
+  float lg[N];
+#pragma unroll
+  for (int c0 = 0; c0 < N; c0 += 16) {
+    uint32_t r[16];
+    tmem_ld16_wait(t_row + c0, r);
+#pragma unroll
+    for (int x = 0; x < 16; ++x)
+      if (c0 + x < N) lg[c0 + x] = __uint_as_float(r[x]);
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(acc_empty);
+  if (valid) {
+    float* d = R.logits_out + (int64_t)t * N;
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+      for (int c = 0; c < N; c += 4)
+        *reinterpret_cast<float4*>(d + c) = make_float4(lg[c], lg[c + 1], lg[c + 2], lg[c + 3]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < N; ++c) d[c] = lg[c];
+    }
+  }
+  // selections and probabilities
+  uint32_t hit = 0;  // bit e: expert e selected
+  float p[N];
+  float psum[G];
+  float p_tot = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float* l = lg + g * E;
+    uint32_t taken = 0;
+    for (int r = 0; r < k; ++r) {
+      int best = 0;
+      float bv = -INFINITY;
+      bool any = false;
+#pragma unroll
+      for (int j = 0; j < E; ++j) {
+        const bool ok = !(taken >> j & 1u) && (!any || l[j] > bv);
+        best = ok ? j : best;
+        bv = ok ? l[j] : bv;
+        any = any || !(taken >> j & 1u);
+      }
+      taken |= 1u << best;
+    }
+    float mx = l[0];
+#pragma unroll
+    for (int j = 1; j < E; ++j) mx = fmaxf(mx, l[j]);
+    float den = 0.f;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      p[g * E + j] = expf(l[j] - mx);
+      den += p[g * E + j];
+    }
+    const float inv = 1.f / den;
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      p[g * E + j] *= inv;
+      if (taken >> j & 1u) s += p[g * E + j];
+    }
+    psum[g] = s;
+    p_tot += s;
+    hit |= (E == 32 ? taken : (taken & ((1u << (E & 31)) - 1u))) << (g * E);
+  }
+  if (!valid) hit = 0;
+  if (valid) {
+    const float winv = 1.f / p_tot;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float ginv = 1.f / psum[g];
+      int r = 0;
+#pragma unroll
+      for (int j = 0; j < E; ++j) {
+        if (!(hit >> (g * E + j) & 1u)) continue;
+        const int64_t o = (int64_t)t * G * k + g * k + r;
+        R.sel[o] = j;
+        R.psel[o] = p[g * E + j];
+        R.gates[o] = p[g * E + j] * ginv;
+        R.wslot[o] = p[g * E + j] * winv;
+        ++r;
+      }
+    }
+  }
+  // per expert over the warp: counts and probability sums; lane e keeps expert e's
+  uint32_t bal[N];
+  int my_cnt = 0;
+  float my_sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    bal[e] = __ballot_sync(all, hit >> e & 1u);
+    float s = valid ? p[e] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(all, s, o);
+    if (lane == e) {
+      my_cnt = __popc(bal[e]);
+      my_sum = s;
+    }
+  }
+  int my_base = 0;
+  if (lane < N) {
+    if (my_cnt) my_base = atomicAdd(&R.cursor[lane], my_cnt);
+    atomicAdd(&R.psum_fx[lane], (unsigned long long)__double2ll_rn((double)my_sum * kProbFix));
+  }
+  const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const int base = __shfl_sync(all, my_base, e);
+    if (hit >> e & 1u) {
+      const int g0 = (e / E) * E;
+      const uint32_t grp_below = hit & ((1u << e) - 1u) & ~((1u << g0) - 1u);
+      const int slot = base + __popc(bal[e] & below);
+      if (slot < P.M) R.bucket[(int64_t)e * P.M + slot] = (t << 3) | __popc(grp_below);
+    }
+  }
+}
+
+template <int N>
+__device__ void route_rows_e(const Params& P, uint32_t t_row, int t, bool valid, int lane,
+                             uint64_t* bar) {
+  switch (N / P.G) {
+    case 1: route_rows<N, 1>(P, t_row, t, valid, lane, bar); break;
+    case 2: if constexpr (N >= 2) route_rows<N, (N >= 2 ? 2 : 1)>(P, t_row, t, valid, lane, bar); break;
+    case 4: if constexpr (N >= 4) route_rows<N, (N >= 4 ? 4 : 1)>(P, t_row, t, valid, lane, bar); break;
+    case 8: if constexpr (N >= 8) route_rows<N, (N >= 8 ? 8 : 1)>(P, t_row, t, valid, lane, bar); break;
+    case 16: if constexpr (N >= 16) route_rows<N, (N >= 16 ? 16 : 1)>(P, t_row, t, valid, lane, bar); break;
+    default: if constexpr (N >= 32) route_rows<N, (N >= 32 ? 32 : 1)>(P, t_row, t, valid, lane, bar); break;
+  }
+}
+
+__device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool valid, int lane,
+                               uint64_t* bar) {
+  switch (P.prob[0].N) {
+    case 1: route_rows_e<1>(P, t_row, t, valid, lane, bar); break;
+    case 2: route_rows_e<2>(P, t_row, t, valid, lane, bar); break;
+    case 4: route_rows_e<4>(P, t_row, t, valid, lane, bar); break;
+    case 8: route_rows_e<8>(P, t_row, t, valid, lane, bar); break;
+    case 16: route_rows_e<16>(P, t_row, t, valid, lane, bar); break;
+    default: route_rows_e<32>(P, t_row, t, valid, lane, bar); break;
+  }
+}
+
+// The last CTA's part once every router tile is done ("GQE" README, Algorithm Overview; the
+// Switch-style load-balancing loss): counts (the cursors), mean_prob, offsets (e M), the
+// loss L = (1/G) sum_e E f_e Pbar_e with f = count / (M k), Pbar = prob_sum / M, and the
+// routed-projection tiles (each expert's bucket cut into runs of 128 slots); then the
+// cursors and sums are zeroed for the next call.
+__device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_term) {
+  const RouteOut& R = P.ro;
+  const int N = P.prob[0].N, G = P.G, k = P.k, M = P.M, E = N / G;
+  const int tid = threadIdx.x;
+  if (tid < N) {
+    const int c = __ldcg(R.cursor + tid);
+    const double ps = (double)__ldcg(reinterpret_cast<const long long*>(R.psum_fx) + tid) / kProbFix;
+    R.counts[tid] = c;
+    R.offsets[tid] = tid * M;
+    R.mean_prob[tid] = (float)(ps / M);
+    s_term[tid] = (double)E * ((double)c / ((double)M * k)) * (ps / M);
+    s_nt[tid] = (c + 127) / 128;
+    R.cursor[tid] = 0;
+    R.psum_fx[tid] = 0ull;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nt = 0;
+    for (int x = 0; x < N; ++x) {
+      const int n = s_nt[x];
+      s_nt[x] = nt;
+      nt += n;
+    }
+    s_nt[N] = nt;
+    R.offsets[N] = N * M;
+    *R.tile_count = nt;
+    if (R.aux) {
+      double L = 0.0;
+      for (int x = 0; x < N; ++x) L += s_term[x];
+      R.aux[0] = (float)(L / G);
+    }
+  }
+  __syncthreads();
+  // tile i of expert x: (x, x M + 128 i); all threads stride over the list
+  for (int x = 0; x < N; ++x) {
+    const int first = s_nt[x], n = s_nt[x + 1] - first;
+    for (int i = tid; i < n; i += blockDim.x) R.tile_list[first + i] = make_int2(x, x * M + i * 128);
+  }
+}
+
+// ROUTE: the dense projection whose router tiles (problem 0) route (route_rows); a separate
+// instance, so the plain GEMMs carry none of that code.
+template <bool GATHER, bool ROUTE>
 __global__ void __launch_bounds__(Lay<GATHER>::THREADS, CTAS_PER_SM)
 tc_gemm_kernel(const __grid_constant__ Params P) {
   using L = Lay<GATHER>;
@@ -142,6 +390,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  uint8_t* scratch = reinterpret_cast<uint8_t*>(acc_empty + 2) + 16;  // routing statistics
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -362,6 +611,10 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
             *reinterpret_cast<uint4*>(dst + c0 + 8) = v1;
           }
         }
+      } else if (ROUTE && ti.p == 0) {
+        // router tile: the logits stay in registers for the routing, which also releases
+        // the accumulator and stores the logits
+        route_rows_any(P, t_row, ti.m0 + row, valid, lane, &acc_empty[acc]);
       } else {
         const Problem& pr = P.prob[ti.p];
         const OutMap& o = pr.out;
@@ -403,9 +656,11 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (!(ROUTE && ti.p == 0)) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
     }
   }
   tc_fence_before();
@@ -413,6 +668,24 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   if (warp == L::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if constexpr (ROUTE) {
+    {
+      // the last CTA to finish forms the routing statistics and the routed-projection tiles
+      __shared__ int s_last;
+      int32_t* ticket = P.ro.cursor + kMaxExperts;
+      if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        finalize_dense_routing(P, reinterpret_cast<int*>(scratch),
+                               reinterpret_cast<double*>(scratch + 8 * (kMaxExperts + 8)));
+        if (threadIdx.x == 0) *ticket = 0;
+      }
+    }
   }
 }
 
@@ -450,17 +723,17 @@ bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATHER>
+template <bool GATHER, bool ROUTE = false>
 int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
-  static bool configured[2] = {false, false};
-  if (!configured[GATHER]) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
+  static bool configured = false;  // one per instance
+  if (!configured) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER, ROUTE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
       return -1;
-    configured[GATHER] = true;
+    configured = true;
   }
-  return launch_pdl(tc_gemm_kernel<GATHER>, dim3(grid), dim3(Lay<GATHER>::THREADS), SMEM_BYTES,
-                    st, P) == cudaSuccess
+  return launch_pdl(tc_gemm_kernel<GATHER, ROUTE>, dim3(grid), dim3(Lay<GATHER>::THREADS),
+                    SMEM_BYTES, st, P) == cudaSuccess
              ? 1
              : -1;
 }
@@ -474,6 +747,30 @@ Problem make_problem(int N, OutMap out) {
   return p;
 }
 
+// Column tiles of all problems, widest first (stable: problem order within a width). With
+// `prob0_first` problem 0's tiles lead instead (the router tiles, whose epilogue routes:
+// that work then overlaps the wide tiles' products rather than trailing them).
+bool set_col_tiles(Params& P, bool prob0_first) {
+  int n = 0;
+  auto width = [&](int p, int t) {
+    const int rem = P.prob[p].N - t * BN;
+    return rem >= BN ? BN : (rem + 15) / 16 * 16;
+  };
+  if (prob0_first)
+    for (int t = 0; t < P.prob[0].n_tiles && n < MAX_COL_TILES; ++t)
+      P.ctile[n++] = make_int2(0, t * BN);
+  for (int w = BN; w >= 16; w -= 16)
+    for (int p = prob0_first ? 1 : 0; p < P.nprob; ++p)
+      for (int t = 0; t < P.prob[p].n_tiles; ++t) {
+        if (width(p, t) != w) continue;
+        if (n == MAX_COL_TILES) return false;
+        P.ctile[n++] = make_int2(p, t * BN);
+      }
+  P.tiles_per_m = n;
+  P.total_tiles = P.m_tiles * n;
+  return true;
+}
+
 int64_t spin_limit(const gqe_ctx* h) { return h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22; }
 
 }  // namespace
@@ -484,8 +781,15 @@ bool tmap_bf16_2d_ext(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
   return tmap_bf16_2d(m, ptr, cols, rows, ld, box_cols, box_rows, sw);
 }
 
+// The dense projection routes (see route_rows) for N a power of two up to 32.
+bool tc_dense_routes(const gqe_ctx* h) { return h->N <= 32 && (h->N & (h->N - 1)) == 0; }
+
+// Also routes when tc_dense_routes(h): the router tiles' epilogue selects the experts and
+// fills the buckets, and the last CTA forms the statistics, the aux loss (if aux_out) and
+// the routed-projection tiles.
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, cudaStream_t st) {
+                         const void* W_v, const void* W_shared, float* aux_out,
+                         cudaStream_t st) {
   const int d_h = h->d_h, G = h->G, dim = h->dim;
   const int S = G * h->k + (W_shared ? 1 : 0);
   Params P;
@@ -511,13 +815,19 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   P.M = M;
   P.K = dim;
   P.m_tiles = (M + BM - 1) / BM;
-  P.tiles_per_m = 0;
-  for (int i = 0; i < np; ++i) P.tiles_per_m += P.prob[i].n_tiles;
-  P.total_tiles = P.m_tiles * P.tiles_per_m;
+  const bool route = tc_dense_routes(h);
+  if (!set_col_tiles(P, route)) return -1;
+  P.col_major = 1;
   P.status = h->ws.status;
   P.spin = spin_limit(h);
+  P.G = G;
+  P.k = h->k;
+  const Workspace& w = h->ws;
+  P.ro = RouteOut{w.logits,  w.sel,    w.psel,   w.gates,     w.w,       w.psum_fx,
+                  w.cursor,  w.bucket, w.counts, w.mean_prob, w.offsets, aux_out,
+                  w.tile_list, w.tile_count};
   const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
-  return launch<false>(h, P, grid, st);
+  return route ? launch<false, true>(h, P, grid, st) : launch<false>(h, P, grid, st);
 }
 
 // The tile list (expert, first bucket slot) and its length come from the routing stage.
@@ -563,8 +873,7 @@ int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaS
   P.M = M;
   P.K = Do;
   P.m_tiles = (M + BM - 1) / BM;
-  P.tiles_per_m = P.prob[0].n_tiles;
-  P.total_tiles = P.m_tiles * P.tiles_per_m;
+  if (!set_col_tiles(P, false)) return -1;
   P.status = h->ws.status;
   P.spin = spin_limit(h);
   const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
