@@ -64,6 +64,11 @@ SMALL = {
     "large_small": dict(base="large_skew", B=1, T=260, skew=None),
     "tiny_f32_batch": dict(base="tiny_f32", B=3, T=77),
     "one_token": dict(base="main_b8_t2048", B=3, T=1),
+    # routing shapes: experts per group not a power of two (the separate routing kernel),
+    # one group of 32 (k = 2 of 32 in one warp-wide group), one expert per group
+    "experts_3_per_group": dict(base="main_b8_t2048", B=1, T=200, N=12, G=4, k=1),
+    "one_group_of_32": dict(base="main_b8_t2048", B=1, T=200, N=32, G=1, k=2),
+    "one_expert_per_group": dict(base="main_b8_t2048", B=1, T=200, N=8, G=8, k=1),
 }
 
 
