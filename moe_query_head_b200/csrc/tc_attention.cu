@@ -24,9 +24,9 @@
 //              maximum grows by more than 2^8 (rare after the first tiles). At the end of an
 //              item the same warps normalise O by the row sum, apply the weighted_concat
 //              scale if any, and store the row into its block of Z.
-// P has TMEM columns of its own. S runs a tile ahead of the softmax warps: S(j+2) is issued
-// as soon as they hold S(j+1) in registers, before P(j) V, which they need only before they
-// write P(j+1). For head dims up to 48 the row sums come from the tensor core (a chunk of
+// P has TMEM columns of its own. S runs a tile ahead of the softmax warps: once P(j) is in
+// TMEM the MMA warp issues P(j) V at once (the softmax warps wait for it before they write
+// P(j+1)), then S(j+2) as soon as they hold S(j+1) in registers. For head dims up to 48 the row sums come from the tensor core (a chunk of
 // ones after every V tile). Head dims above 64 run one CTA per SM with 512 TMEM columns.
 #include <cudaTypedefs.h>
 
@@ -350,10 +350,10 @@ attn_kernel(const __grid_constant__ Params P) {
     uint32_t n_sf = 0, n_p = 0, n_o = 0;  // uses of s_free / p_ready / o_full
     bool ok = true;
 
-    // Order of issue per item: S(0), S(1); then for every tile j, once P(j) is ready,
-    // S(j+2) (as soon as the softmax warps hold S(j+1) in registers) and only then P(j) V.
-    // S therefore always runs a tile ahead of the softmax warps, and the products of P(j)
-    // V, which they need only before they write P(j+1), never delay the next S.
+    // Order of issue per item: S(0), S(1); then for every tile j, once P(j) is ready, P(j) V
+    // and then S(j+2) (as soon as the softmax warps hold S(j+1) in registers). P(j) V is
+    // queued behind nothing the softmax warps do not need first, and S(j+2) is still a whole
+    // tile ahead of its use.
     // S = Q K^T for the next K tile; its stage is released when the product is done.
     auto issue_s = [&](bool last_s) -> bool {
       if (!warp_wait(&k_full[kst], k_phase, P, abort_flag)) return false;
@@ -395,12 +395,6 @@ attn_kernel(const __grid_constant__ Params P) {
       for (int j = 0; j < nk; ++j) {
         if (!warp_wait(p_ready, n_p & 1, P, abort_flag)) { ok = false; break; }
         ++n_p;
-        if (j + 2 < nk) {
-          // the softmax warps take S(j+1) into registers right after P(j)
-          if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) { ok = false; break; }
-          ++n_sf;
-          if (!issue_s(j + 3 == nk)) { ok = false; break; }  // S(j+2)
-        }
         if (j == 0 && n_o > 0 && !warp_wait(o_free, (n_o - 1) & 1, P, abort_flag)) {
           ok = false;
           break;
@@ -422,6 +416,12 @@ attn_kernel(const __grid_constant__ Params P) {
           mma_commit(&v_empty[vst]);
         }
         __syncwarp();
+        if (j + 2 < nk) {
+          // then S(j+2), once the softmax warps hold S(j+1) in registers
+          if (!warp_wait(s_free, n_sf & 1, P, abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!issue_s(j + 3 == nk)) { ok = false; break; }  // S(j+2)
+        }
         if (last) ++n_o;
         if (++vst == C::V_STAGES) {
           vst = 0;
