@@ -478,50 +478,92 @@ attn_kernel(const __grid_constant__ Params P) {
           for (int c = 0; c < TK; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
         }
-        // row maximum: eight independent chains of three-input max, then a tree
-        float mp[8];
+        // Row maximum in two halves of 64 columns: the exponentials of the first half need
+        // only its own maximum (and the running reference), so the second half's maximum is
+        // formed while they run. A reference moves only when a maximum passes it by more
+        // than the threshold; if the second half's does, the first half's P is rescaled
+        // (rare after a row's first tiles).
         static_assert(TK == 128, "the row-maximum schedule covers 128 columns");
+        float mp[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) mp[x] = fmax3(s[x], s[8 + x], s[16 + x]);        // 0..23
 #pragma unroll
-        for (int c = 24; c < 120; c += 16)                                          // 24..119
+        for (int c = 24; c < 56; c += 16)                                           // 24..55
 #pragma unroll
           for (int x = 0; x < 8; ++x) mp[x] = fmax3(mp[x], s[c + x], s[c + 8 + x]);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) mp[x] = fmaxf(mp[x], s[120 + x]);               // 120..127
-        const float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]),
-                               fmax3(fmax3(mp[3], mp[4], mp[5]), mp[6], mp[7]));
-        float m_new = mx * cs;
-        if (m_new == -INFINITY) m_new = 0.f;  // a row with every key masked
-        bool need = false;
-        float alpha = 1.f;
-        if (j == 0) {
-          m_used = m_new;
-        } else if (m_new > m_used + kRescaleThreshold) {
-          need = true;
-          alpha = fast_exp2(m_used - m_new);
-          m_used = m_new;
+        for (int x = 0; x < 8; ++x) mp[x] = fmaxf(mp[x], s[56 + x]);                // 56..63
+        const float m_old = m_used;
+        {
+          const float m_a = fmaxf(fmax3(mp[0], mp[1], mp[2]),
+                                  fmax3(fmax3(mp[3], mp[4], mp[5]), mp[6], mp[7])) * cs;
+          if (j == 0)
+            m_used = m_a == -INFINITY ? 0.f : m_a;  // a half with every key masked
+          else if (m_a > m_used + kRescaleThreshold)
+            m_used = m_a;
         }
         // p = exp2(s * scale - m) with a packed FMA for the argument; most pairs on MUFU,
         // kFmaPairsOf8 of every 8 on the FMA-pipe polynomial. P is kept in registers as
         // bf16 pairs until the whole tile is done.
         const float2 cs2 = make_float2(cs, cs);
-        const float2 nm2 = make_float2(-m_used, -m_used);
         uint32_t pk[TK / 2];
-        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
+        float2 lsa[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 lsb[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        {
+          const float2 nm2 = make_float2(-m_used, -m_used);
 #pragma unroll
-        for (int x = 0; x < TK / 2; ++x) {
-          const float2 t = fma2(make_float2(s[2 * x], s[2 * x + 1]), cs2, nm2);
-          const float2 p = (x & 7) >= 8 - kFmaPairsOf8
-                               ? exp2_fma2(t)
-                               : make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          if constexpr (!C::SUM_MMA) lsum[x & 3] = add2(lsum[x & 3], p);
-          pk[x] = pack_bf16x2(p.x, p.y);
+          for (int x = 0; x < TK / 4; ++x) {
+            const float2 t = fma2(make_float2(s[2 * x], s[2 * x + 1]), cs2, nm2);
+            const float2 p = (x & 7) >= 8 - kFmaPairsOf8
+                                 ? exp2_fma2(t)
+                                 : make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            if constexpr (!C::SUM_MMA) lsa[x & 1] = add2(lsa[x & 1], p);
+            pk[x] = pack_bf16x2(p.x, p.y);
+          }
         }
+        // second half's maximum
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mp[x] = fmax3(s[64 + x], s[72 + x], s[80 + x]);  // 64..87
+#pragma unroll
+        for (int c = 88; c < 120; c += 16)                                          // 88..119
+#pragma unroll
+          for (int x = 0; x < 8; ++x) mp[x] = fmax3(mp[x], s[c + x], s[c + 8 + x]);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mp[x] = fmaxf(mp[x], s[120 + x]);               // 120..127
+        {
+          const float m_b = fmaxf(fmax3(mp[0], mp[1], mp[2]),
+                                  fmax3(fmax3(mp[3], mp[4], mp[5]), mp[6], mp[7])) * cs;
+          if (m_b > m_used + kRescaleThreshold) {
+            const float a2 = fast_exp2(m_used - m_b);
+#pragma unroll
+            for (int x = 0; x < TK / 4; ++x)
+              pk[x] = pack_bf16x2(__uint_as_float(pk[x] << 16) * a2,
+                                  __uint_as_float(pk[x] & 0xffff0000u) * a2);
+            if constexpr (!C::SUM_MMA) {
+              lsa[0] = mul2(lsa[0], make_float2(a2, a2));
+              lsa[1] = mul2(lsa[1], make_float2(a2, a2));
+            }
+            m_used = m_b;
+          }
+        }
+        {
+          const float2 nm2 = make_float2(-m_used, -m_used);
+#pragma unroll
+          for (int x = TK / 4; x < TK / 2; ++x) {
+            const float2 t = fma2(make_float2(s[2 * x], s[2 * x + 1]), cs2, nm2);
+            const float2 p = (x & 7) >= 8 - kFmaPairsOf8
+                                 ? exp2_fma2(t)
+                                 : make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            if constexpr (!C::SUM_MMA) lsb[x & 1] = add2(lsb[x & 1], p);
+            pk[x] = pack_bf16x2(p.x, p.y);
+          }
+        }
+        // O is rescaled when this tile moved the reference (never on a row's first tile)
+        const bool need = j > 0 && m_used != m_old;
+        const float alpha = need ? fast_exp2(m_old - m_used) : 1.f;
         if constexpr (!C::SUM_MMA) {
-          const float2 a = add2(add2(lsum[0], lsum[1]), add2(lsum[2], lsum[3]));
-          l = l * alpha + (a.x + a.y);  // alpha = 1 unless this row's maximum moved on
+          const float2 a = add2(add2(lsa[0], lsa[1]), add2(lsb[0], lsb[1]));
+          l = l * alpha + (a.x + a.y);
         }
         // S(j) was issued without waiting for P(j-1) V, and the exponentials above did not
         // need it either: only now wait for that product before overwriting P or
