@@ -88,7 +88,7 @@ struct Workspace {
   int32_t* offsets = nullptr;      // [N + 1] bucket start of each expert (e M)
   int32_t* bucket = nullptr;       // [N * M] entries (token << 3) | rank; expert e's run of
                                    // counts[e] entries starts at e M
-  int2* tile_list = nullptr;       // routed-projection tiles (expert, first bucket slot)
+  int2* tile_list = nullptr;       // routed-projection tiles (expert | rows << 8, first slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* attn_counter = nullptr; // attention work-item counter
   unsigned long long* psum_fx = nullptr;  // [kMaxExperts] probability sums in fixed point

@@ -409,8 +409,8 @@ __device__ void fused_bucket(const int32_t* __restrict__ sel, const int32_t* __r
 // order (probabilities in double), so the result does not depend on scheduling. Writes
 // counts (the cursors' final values), mean_prob, offsets (e M), the Switch loss
 //   L = (1/G) sum_g E sum_j f_{g,j} Pbar_{g,j},  f = c / (M k),  Pbar = prob_sum / M,
-// and the routed-projection tiles (each expert's bucket cut into runs of 128 slots), then
-// zeroes the cursors.
+// and the routed-projection tiles (each expert's bucket cut into runs of 128 slots:
+// (expert | rows << 8, first slot)), then zeroes the cursors.
 __device__ void finalize_routing(const float* __restrict__ part_prob, int nblk, int M, int N,
                                  int G, int k, int32_t* __restrict__ cursor,
                                  int32_t* __restrict__ counts, float* __restrict__ mean_prob,
@@ -470,7 +470,8 @@ __device__ void finalize_routing(const float* __restrict__ part_prob, int nblk, 
   __syncthreads();
   for (int x = tid; x < N; x += kFusedThreads) {
     const int nt = (s_cnt[x] + 127) / 128;
-    for (int i = 0; i < nt; ++i) tile_list[s_nt[x] + i] = make_int2(x, x * M + i * 128);
+    for (int i = 0; i < nt; ++i)
+      tile_list[s_nt[x] + i] = make_int2(x | min(128, s_cnt[x] - 128 * i) << 8, x * M + i * 128);
   }
 }
 

@@ -35,25 +35,28 @@ using namespace tc;
 constexpr int BM = 128;        // tile rows = MMA M = TMEM lanes
 constexpr int BN = 128;        // widest tile (MMA N)
 constexpr int BK = 64;         // one 128-byte swizzle atom of bf16 along K
-constexpr int STAGES = 3;
 constexpr int CTAS_PER_SM = 2;  // shared memory: 2 x ~98 KB; TMEM: 2 x 256 columns
 // Warp roles: producers, one MMA-issuing warp, four epilogue warps.
 template <bool GATHER>
 struct Lay {
   static constexpr int NPROD = GATHER ? 3 : 1;
-  // A producer warp waits only for the stage it fills next; with more producer warps than
-  // stages one of them could get two uses of a stage ahead of the MMA warp, and a parity
-  // wait cannot tell those phases apart.
-  static_assert(NPROD <= STAGES, "a producer warp could lap the stage ring");
   static constexpr int MMA = NPROD;
   static constexpr int EPI0 = NPROD + 1;
   static constexpr int THREADS = (NPROD + 5) * 32;
 };
-constexpr int A_STAGE_BYTES = BM * BK * 2;
-constexpr int B_STAGE_BYTES = BN * BK * 2;
-// stages, 1024-byte alignment, barriers and flags, the routing statistics' scratch
-constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 + 256 +
-                           16 * (kMaxExperts + 8);
+// Shared-memory ring: B stages hold up to BN rows, or 64 for the routed projection of a head
+// dimension up to 64 (NARROW), whose smaller stages buy a fourth stage in the same space:
+// these GEMMs are bound by load latency times the bytes in flight.
+template <bool NARROW>
+struct Ring {
+  static constexpr int STAGES = NARROW ? 4 : 3;
+  static constexpr int B_ROWS = NARROW ? 64 : BN;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  // stages, 1024-byte alignment, barriers and flags, the routing statistics' scratch
+  static constexpr int SMEM =
+      STAGES * (A_BYTES + B_BYTES) + 1024 + 256 + 16 * (kMaxExperts + 8) + 4 * kMaxExperts;
+};
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_PROBLEMS = 4;
 constexpr int MAX_COL_TILES = 32;  // column tiles over all problems of one GEMM
@@ -102,7 +105,7 @@ struct Params {
   // routed projection (gather mode)
   const __nv_bfloat16* x;               // A rows gathered from x [M, K]
   const int32_t* bucket;                // entries (t << 3) | r
-  const int2* tile_list;                // (expert, first bucket slot) per tile
+  const int2* tile_list;                // (expert | rows << 8, first bucket slot) per tile
   const int32_t* tile_count;            // number of tiles (device)
   const int32_t* offsets;               // bucket start of each expert [N]
   const int32_t* counts;                // entries in each expert's bucket [N]
@@ -127,11 +130,10 @@ template <bool GATHER>
 __device__ __forceinline__ TileInfo tile_info(const Params& P, int tile) {
   TileInfo ti;
   if constexpr (GATHER) {
-    const int2 t = P.tile_list[tile];
-    ti.p = t.x;
+    const int2 t = P.tile_list[tile];  // (expert | rows << 8, first bucket slot)
+    ti.p = t.x & 255;
     ti.m0 = t.y;
-    const int end = P.offsets[t.x] + P.counts[t.x];
-    ti.rows = min(BM, end - t.y);
+    ti.rows = t.x >> 8;
     ti.n0 = 0;
     ti.n = P.prob[0].box_n;
   } else {
@@ -333,7 +335,7 @@ __device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool vali
 // loss L = (1/G) sum_e E f_e Pbar_e with f = count / (M k), Pbar = prob_sum / M, and the
 // routed-projection tiles (each expert's bucket cut into runs of 128 slots); then the
 // cursors and sums are zeroed for the next call.
-__device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_term) {
+__device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_term, int* s_cnt) {
   const RouteOut& R = P.ro;
   const int N = P.prob[0].N, G = P.G, k = P.k, M = P.M, E = N / G;
   const int tid = threadIdx.x;
@@ -345,6 +347,7 @@ __device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_ter
     R.mean_prob[tid] = (float)(ps / M);
     s_term[tid] = (double)E * ((double)c / ((double)M * k)) * (ps / M);
     s_nt[tid] = (c + 127) / 128;
+    s_cnt[tid] = c;
     R.cursor[tid] = 0;
     R.psum_fx[tid] = 0ull;
   }
@@ -366,19 +369,28 @@ __device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_ter
     }
   }
   __syncthreads();
-  // tile i of expert x: (x, x M + 128 i); all threads stride over the list
+  // tile i of expert x: (x | rows << 8, x M + 128 i); all threads stride over the list
   for (int x = 0; x < N; ++x) {
     const int first = s_nt[x], n = s_nt[x + 1] - first;
-    for (int i = tid; i < n; i += blockDim.x) R.tile_list[first + i] = make_int2(x, x * M + i * 128);
+    for (int i = tid; i < n; i += blockDim.x)
+      R.tile_list[first + i] = make_int2(x | min(128, s_cnt[x] - 128 * i) << 8, x * M + i * 128);
   }
 }
 
 // ROUTE: the dense projection whose router tiles (problem 0) route (route_rows); a separate
 // instance, so the plain GEMMs carry none of that code.
-template <bool GATHER, bool ROUTE>
+template <bool GATHER, bool ROUTE, bool NARROW>
 __global__ void __launch_bounds__(Lay<GATHER>::THREADS, CTAS_PER_SM)
 tc_gemm_kernel(const __grid_constant__ Params P) {
   using L = Lay<GATHER>;
+  using R = Ring<NARROW>;
+  constexpr int STAGES = R::STAGES;
+  constexpr int A_STAGE_BYTES = R::A_BYTES;
+  constexpr int B_STAGE_BYTES = R::B_BYTES;
+  // A producer warp waits only for the stage it fills next; with more producer warps than
+  // stages one of them could get two uses of a stage ahead of the MMA warp, and a parity
+  // wait cannot tell those phases apart.
+  static_assert(L::NPROD <= STAGES, "a producer warp could lap the stage ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -460,20 +472,42 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       const int pw = warp;
       const int c = lane & 7;
       uint32_t g = 0;  // position in the CTA's stage sequence
-      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const int2 t = P.tile_list[tile];
-        const int n = min(BM, P.offsets[t.x] + P.counts[t.x] - t.y);
-        const uint32_t b_bytes = (uint32_t)P.prob[0].box_n * BK * 2;
-        // source rows of this lane: r = 4 i + lane / 8 (rows past the tile's end repeat
-        // its first row: computed, never stored)
-        int src[BM / 4];
-        // (token indices are clamped to the call's rows: defence against a bucket that a
-        // failed routing pass left stale; a complete pass never needs it)
-        const int first = min(P.bucket[t.y] >> 3, P.M - 1);
+      // Index pipeline: the tile-list entry two tiles ahead and the bucket entries (source
+      // rows) of the next tile are loaded while this tile's rows stream, and only used a
+      // tile later, so no tile boundary waits for an index load.
+      const int stride = gridDim.x;
+      int tile = blockIdx.x;
+      int2 t = tile < total ? P.tile_list[tile] : make_int2(0, 0);
+      int2 t_nxt = tile + stride < total ? P.tile_list[tile + stride] : make_int2(0, 0);
+      // raw bucket entries of this lane's source rows r = 4 i + lane / 8 (rows past the
+      // tile's end repeat its first row: computed, never stored)
+      int raw[BM / 4], raw0;
+      auto load_rows = [&](int2 tt, int (&dst)[BM / 4], int& d0) {
+        const int n = tt.x >> 8;
+        d0 = P.bucket[tt.y];
 #pragma unroll
         for (int i = 0; i < BM / 4; ++i) {
           const int r = 4 * i + (lane >> 3);
-          src[i] = r < n ? min(P.bucket[t.y + r] >> 3, P.M - 1) : first;
+          dst[i] = r < n ? P.bucket[tt.y + r] : 0;
+        }
+      };
+      if (tile < total) load_rows(t, raw, raw0);
+      for (; tile < total && !*abort_flag; tile += stride) {
+        const int2 t_nn =
+            tile + 2 * stride < total ? P.tile_list[tile + 2 * stride] : make_int2(0, 0);
+        int nraw[BM / 4], nraw0 = 0;
+        if (tile + stride < total) load_rows(t_nxt, nraw, nraw0);
+        const int n = t.x >> 8;
+        const int e = t.x & 255;
+        const uint32_t b_bytes = (uint32_t)P.prob[0].box_n * BK * 2;
+        // (token indices are clamped to the call's rows: defence against a bucket that a
+        // failed routing pass left stale; a complete pass never needs it)
+        const int first = min(raw0 >> 3, P.M - 1);
+        int src[BM / 4];
+#pragma unroll
+        for (int i = 0; i < BM / 4; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          src[i] = r < n ? min(raw[i] >> 3, P.M - 1) : first;
         }
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++g) {
@@ -487,7 +521,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           }
           if (elect_one()) {
             mbar_arrive_expect_tx(&full[stage], b_bytes);
-            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, t.x * P.d_h,
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, e * P.d_h,
                         &full[stage]);
           }
           const uint32_t dst = smem_u32(sA + stage * A_STAGE_BYTES);
@@ -504,6 +538,11 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           cp_async_mbar_arrive_noinc(&full[stage]);
         }
         if (!ok) break;
+        t = t_nxt;
+        t_nxt = t_nn;
+        raw0 = nraw0;
+#pragma unroll
+        for (int i = 0; i < BM / 4; ++i) raw[i] = nraw[i];
       }
       // no copy of this warp may still be writing when the CTA leaves
       cp_async_wait<0>();
@@ -682,7 +721,8 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       if (s_last) {
         __threadfence();
         finalize_dense_routing(P, reinterpret_cast<int*>(scratch),
-                               reinterpret_cast<double*>(scratch + 8 * (kMaxExperts + 8)));
+                               reinterpret_cast<double*>(scratch + 8 * (kMaxExperts + 8)),
+                               reinterpret_cast<int*>(scratch + 16 * (kMaxExperts + 8)));
         if (threadIdx.x == 0) *ticket = 0;
       }
     }
@@ -723,17 +763,18 @@ bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATHER, bool ROUTE = false>
+template <bool GATHER, bool ROUTE = false, bool NARROW = false>
 int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
+  constexpr int smem = Ring<NARROW>::SMEM;
   static bool configured = false;  // one per instance
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER, ROUTE>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER, ROUTE, NARROW>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return -1;
     configured = true;
   }
-  return launch_pdl(tc_gemm_kernel<GATHER, ROUTE>, dim3(grid), dim3(Lay<GATHER>::THREADS),
-                    SMEM_BYTES, st, P) == cudaSuccess
+  return launch_pdl(tc_gemm_kernel<GATHER, ROUTE, NARROW>, dim3(grid),
+                    dim3(Lay<GATHER>::THREADS), smem, st, P) == cudaSuccess
              ? 1
              : -1;
 }
@@ -830,7 +871,7 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   return route ? launch<false, true>(h, P, grid, st) : launch<false>(h, P, grid, st);
 }
 
-// The tile list (expert, first bucket slot) and its length come from the routing stage.
+// The tile list (expert | rows << 8, first bucket slot) and its length come from the routing.
 int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st) {
   Params P;
   memset(&P, 0, sizeof(P));
@@ -858,7 +899,8 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStrea
   P.spin = spin_limit(h);
   const int max_tiles = (int)(((int64_t)M * h->G * h->k + BM - 1) / BM) + h->N;
   const int grid = min(max_tiles, CTAS_PER_SM * h->num_sms);
-  return launch<true>(h, P, grid, st);
+  return P.prob[0].box_n <= Ring<true>::B_ROWS ? launch<true, false, true>(h, P, grid, st)
+                                                : launch<true>(h, P, grid, st);
 }
 
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st) {
