@@ -66,7 +66,8 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.tile_count = (int32_t*)take(16);
   w.attn_counter = (int32_t*)take(16);
   w.cursor = (int32_t*)take((kMaxExperts + 4) * 4);
-  w.psum_fx = (unsigned long long*)take(kMaxExperts * 8);
+  w.rcur = (int32_t*)take(2 * kMaxExperts * 4);
+  w.rpsum = (unsigned long long*)take(2 * kMaxExperts * 8);
   w.status = (int32_t*)take(16);
   (void)dim;
   return off;
@@ -219,17 +220,25 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   // launches (the arguments are evaluated first), so event i precedes stage i.
   // bf16: tensor-core (tcgen05) kernels for the projections; fp32: CUDA-core kernels.
   const bool tc = h->dtype == GQE_BF16;
+  // bf16 with N a power of two up to 32: the routing runs in the dense projection's router
+  // tiles, and the routed projection schedules from its cursors (set `rs`, alternating)
+  const bool fused = tc && tc_dense_routes(h);
+  const int rs = h->route_set;
+  int dense = -1;
   bool ok = mark() &&
-            add(tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, aux_loss, st)
-                   : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
-            // bf16: the routing usually runs in the dense projection's router tiles
-            add(tc && tc_dense_routes(h) ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
-            add(tc ? launch_tc_qproj(h, x, M, W_q, st) : launch_simt_qproj(h, x, M, W_q, st)) &&
+            add(dense = tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, rs, st)
+                           : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
+            add(fused ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
+            add(tc ? launch_tc_qproj(h, x, M, W_q, fused ? rs : -1, aux_loss, st)
+                   : launch_simt_qproj(h, x, M, W_q, st)) &&
             add(tc ? launch_tc_attention(h, B, T, S, has_shared, variant, causal, Do, st)
                    : launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&
             add(launch_combine(h, M, variant, Do, st)) &&
             add(tc ? launch_tc_oproj(h, M, Do, W_o, out, st)
                    : launch_simt_oproj(h, M, Do, W_o, out, st));
+  // once the dense projection has run, this call's cursor set is in use and the other one
+  // cleared: the next call takes the other one
+  if (fused && dense >= 0) h->route_set ^= 1;
   h->last_M = M;
   h->last_S = S;
   h->last_Do = Do;

@@ -91,8 +91,10 @@ struct Workspace {
   int2* tile_list = nullptr;       // routed-projection tiles (expert | rows << 8, first slot)
   int32_t* tile_count = nullptr;   // number of routed-projection tiles
   int32_t* attn_counter = nullptr; // attention work-item counter
-  unsigned long long* psum_fx = nullptr;  // [kMaxExperts] probability sums in fixed point
-                                          // (dense-projection routing; zero between calls)
+  // dense-projection routing: two sets (alternate calls) of bucket cursors and
+  // fixed-point probability sums; a call's set is zero when it starts
+  int32_t* rcur = nullptr;                // [2, kMaxExperts]
+  unsigned long long* rpsum = nullptr;    // [2, kMaxExperts]
   int32_t* cursor = nullptr;       // [kMaxExperts] bucket cursors, then the routing ticket
                                    // (zero between calls)
   int32_t* status = nullptr;       // device status word
@@ -116,6 +118,7 @@ struct gqe_ctx {
   int n_stage_events = 0;
   // state of the last forward
   int last_M = 0, last_S = 0, last_Do = 0, last_launches = 0;
+  int route_set = 0;  // the dense-projection routing's cursor set for the next call
 };
 
 namespace gqe {
@@ -149,10 +152,11 @@ int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st);
 int launch_simt_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 // tcgen05 paths (bf16)
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, float* aux_out,
+                         const void* W_v, const void* W_shared, int route_set,
                          cudaStream_t st);
 bool tc_dense_routes(const gqe_ctx* h);  // launch_tc_dense_proj also routes
-int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st);
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route_set,
+                    float* aux_out, cudaStream_t st);
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,
                         int causal, int Do, cudaStream_t st);

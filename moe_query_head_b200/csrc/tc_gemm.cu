@@ -53,7 +53,7 @@ struct Ring {
   static constexpr int B_ROWS = NARROW ? 64 : BN;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
-  // stages, 1024-byte alignment, barriers and flags, the routing statistics' scratch
+  // stages, 1024-byte alignment, barriers and flags, the routed schedule's scratch
   static constexpr int SMEM =
       STAGES * (A_BYTES + B_BYTES) + 1024 + 256 + 16 * (kMaxExperts + 8) + 4 * kMaxExperts;
 };
@@ -68,21 +68,30 @@ struct Problem {
   OutMap out;
 };
 
-// Outputs of the routing done in the dense projection's router tiles (see route_rows).
+// Outputs of the routing done in the dense projection's router tiles (see route_rows). The
+// cursors and probability sums come in two sets used by alternate calls: this call's set
+// is zero when it starts (the previous call's dense projection cleared it), and this call
+// clears the other one, whose last reader (the previous call's routed projection) is done.
 struct RouteOut {
   float* logits_out;     // [M, N] problem 0's output (router logits, fp32)
   int32_t* sel;          // [M, G, k]
   float* psel;           // [M, G, k]
   float* gates;          // [M, G, k]
   float* wslot;          // [M, G, k]
-  unsigned long long* psum_fx;  // [kMaxExperts] probability sums, fixed point (zero between calls)
-  int32_t* cursor;       // [kMaxExperts] bucket cursors, then the CTA ticket (zero between calls)
+  unsigned long long* psum_fx;  // [kMaxExperts] probability sums, fixed point
+  int32_t* cursor;       // [kMaxExperts] bucket cursors
+  unsigned long long* clear_psum;  // the other set, zeroed here
+  int32_t* clear_cursor;
   int32_t* bucket;       // [N * M]
+};
+
+// Routing statistics written by the routed projection's CTA 0 when it schedules from the
+// cursors ("GQE" README, Algorithm Overview; the Switch-style load-balancing loss).
+struct StatsOut {
   int32_t* counts;       // [N]
   float* mean_prob;      // [N]
   int32_t* offsets;      // [N + 1]
   float* aux;            // [1] or null
-  int2* tile_list;
   int32_t* tile_count;
 };
 
@@ -107,8 +116,12 @@ struct Params {
   const int32_t* bucket;                // entries (t << 3) | r
   const int2* tile_list;                // (expert | rows << 8, first bucket slot) per tile
   const int32_t* tile_count;            // number of tiles (device)
-  const int32_t* offsets;               // bucket start of each expert [N]
-  const int32_t* counts;                // entries in each expert's bucket [N]
+  // scheduling from the dense projection's cursors instead of the tile list (rc non-null):
+  // expert e's bucket holds rc[e] entries; CTA 0 also writes the statistics
+  const int32_t* rc;
+  const unsigned long long* rpsum;      // probability sums, fixed point
+  int nexp;
+  StatsOut so;
   __nv_bfloat16* Q;                     // query streams [S, M, d_h]
   // dense projection with routing (the ROUTE instance): problem 0 = W_r
   int G;
@@ -126,11 +139,24 @@ struct TileInfo {
   int n;       // MMA N (multiple of 16)
 };
 
+// Routed-projection tile `tile` as (expert | rows << 8, first bucket slot): from the tile
+// list, or (scheduling from the cursors) from the per-expert counts s_cnt and first tiles
+// s_t0 [nexp + 1] in shared memory (experts in order; each bucket cut into runs of 128).
+__device__ __forceinline__ int2 tile_entry(const Params& P, const int* s_cnt, const int* s_t0,
+                                           int tile) {
+  if (P.rc == nullptr) return P.tile_list[tile];
+  int x = 0;
+  while (x + 1 < P.nexp && s_t0[x + 1] <= tile) ++x;
+  const int i = tile - s_t0[x];
+  return make_int2(x | min(BM, s_cnt[x] - BM * i) << 8, x * P.M + i * BM);
+}
+
 template <bool GATHER>
-__device__ __forceinline__ TileInfo tile_info(const Params& P, int tile) {
+__device__ __forceinline__ TileInfo tile_info(const Params& P, int tile, const int* s_cnt,
+                                              const int* s_t0) {
   TileInfo ti;
   if constexpr (GATHER) {
-    const int2 t = P.tile_list[tile];  // (expert | rows << 8, first bucket slot)
+    const int2 t = tile_entry(P, s_cnt, s_t0, tile);  // (expert | rows << 8, first slot)
     ti.p = t.x & 255;
     ti.m0 = t.y;
     ti.rows = t.x >> 8;
@@ -330,51 +356,47 @@ __device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool vali
   }
 }
 
-// The last CTA's part once every router tile is done ("GQE" README, Algorithm Overview; the
-// Switch-style load-balancing loss): counts (the cursors), mean_prob, offsets (e M), the
-// loss L = (1/G) sum_e E f_e Pbar_e with f = count / (M k), Pbar = prob_sum / M, and the
-// routed-projection tiles (each expert's bucket cut into runs of 128 slots); then the
-// cursors and sums are zeroed for the next call.
-__device__ void finalize_dense_routing(const Params& P, int* s_nt, double* s_term, int* s_cnt) {
-  const RouteOut& R = P.ro;
-  const int N = P.prob[0].N, G = P.G, k = P.k, M = P.M, E = N / G;
+// The routed projection's schedule from the dense projection's cursors, in every CTA
+// (block-wide, shared memory): s_cnt[e] = expert e's entries, s_t0[e] = its first tile
+// (each bucket cut into runs of 128 slots), s_t0[nexp] = the number of tiles. CTA 0 also
+// writes the routing statistics ("GQE" README, Algorithm Overview; the Switch-style
+// load-balancing loss): counts, mean_prob (fixed-point sum / M), offsets (e M) and
+//   L = (1/G) sum_e E f_e Pbar_e,  f = count / (M k),  Pbar = prob_sum / M.
+__device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0) {
+  const int N = P.nexp, M = P.M;
   const int tid = threadIdx.x;
-  if (tid < N) {
-    const int c = __ldcg(R.cursor + tid);
-    const double ps = (double)__ldcg(reinterpret_cast<const long long*>(R.psum_fx) + tid) / kProbFix;
-    R.counts[tid] = c;
-    R.offsets[tid] = tid * M;
-    R.mean_prob[tid] = (float)(ps / M);
-    s_term[tid] = (double)E * ((double)c / ((double)M * k)) * (ps / M);
-    s_nt[tid] = (c + 127) / 128;
-    s_cnt[tid] = c;
-    R.cursor[tid] = 0;
-    R.psum_fx[tid] = 0ull;
-  }
+  if (tid < N) s_cnt[tid] = __ldcg(P.rc + tid);
   __syncthreads();
   if (tid == 0) {
     int nt = 0;
     for (int x = 0; x < N; ++x) {
-      const int n = s_nt[x];
-      s_nt[x] = nt;
-      nt += n;
+      s_t0[x] = nt;
+      nt += (s_cnt[x] + BM - 1) / BM;
     }
-    s_nt[N] = nt;
-    R.offsets[N] = N * M;
-    *R.tile_count = nt;
-    if (R.aux) {
+    s_t0[N] = nt;
+  }
+  if (blockIdx.x == 0) {
+    const StatsOut& S = P.so;
+    const int G = N / P.E;
+    if (tid < N) {
+      const double ps = (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + tid) / kProbFix;
+      S.counts[tid] = s_cnt[tid];
+      S.offsets[tid] = tid * M;
+      S.mean_prob[tid] = (float)(ps / M);
+    }
+    if (tid == 0) {
+      S.offsets[N] = N * M;
       double L = 0.0;
-      for (int x = 0; x < N; ++x) L += s_term[x];
-      R.aux[0] = (float)(L / G);
+      for (int x = 0; x < N; ++x) {
+        const double ps =
+            (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + x) / kProbFix;
+        L += (double)P.E * ((double)s_cnt[x] / ((double)M * P.k)) * (ps / M);
+      }
+      if (S.aux) S.aux[0] = (float)(L / G);
     }
   }
   __syncthreads();
-  // tile i of expert x: (x | rows << 8, x M + 128 i); all threads stride over the list
-  for (int x = 0; x < N; ++x) {
-    const int first = s_nt[x], n = s_nt[x + 1] - first;
-    for (int i = tid; i < n; i += blockDim.x)
-      R.tile_list[first + i] = make_int2(x | min(128, s_cnt[x] - 128 * i) << 8, x * M + i * 128);
-  }
+  if (blockIdx.x == 0 && tid == 0) *P.so.tile_count = s_t0[N];
 }
 
 // ROUTE: the dense projection whose router tiles (problem 0) route (route_rows); a separate
@@ -402,7 +424,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  uint8_t* scratch = reinterpret_cast<uint8_t*>(acc_empty + 2) + 16;  // routing statistics
+  uint8_t* scratch = reinterpret_cast<uint8_t*>(acc_empty + 2) + 16;  // routed schedule
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -433,7 +455,24 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   const int KB = (P.K + BK - 1) / BK;
   pdl_wait();  // the previous kernel's outputs (x, the buckets, Z) are complete from here on
   pdl_allow_next();
-  const int total = GATHER ? *P.tile_count : P.total_tiles;
+  int* s_cnt = reinterpret_cast<int*>(scratch);         // [kMaxExperts] routed schedule
+  int* s_t0 = s_cnt + kMaxExperts;                      // [kMaxExperts + 1]
+  int total = P.total_tiles;
+  if constexpr (ROUTE) {
+    // this call's cursor set is zero; the other one (the previous call's) is cleared here
+    if (blockIdx.x == 0 && threadIdx.x < kMaxExperts) {
+      P.ro.clear_cursor[threadIdx.x] = 0;
+      P.ro.clear_psum[threadIdx.x] = 0ull;
+    }
+  }
+  if constexpr (GATHER) {
+    if (P.rc != nullptr) {
+      routed_schedule(P, s_cnt, s_t0);  // block-wide
+      total = s_t0[P.nexp];
+    } else {
+      total = *P.tile_count;
+    }
+  }
 
   if (warp < L::NPROD) {
     // ------------------------------------------------------------------ producers
@@ -442,7 +481,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const TileInfo ti = tile_info<false>(P, tile);
+        const TileInfo ti = tile_info<false>(P, tile, nullptr, nullptr);
         const uint32_t b_bytes = (uint32_t)P.prob[ti.p].box_n * BK * 2;
         for (int kb = 0; kb < KB; ++kb) {
           bool ok = mbar_wait(&empty[stage], phase ^ 1, P.spin);
@@ -477,8 +516,9 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       // tile later, so no tile boundary waits for an index load.
       const int stride = gridDim.x;
       int tile = blockIdx.x;
-      int2 t = tile < total ? P.tile_list[tile] : make_int2(0, 0);
-      int2 t_nxt = tile + stride < total ? P.tile_list[tile + stride] : make_int2(0, 0);
+      int2 t = tile < total ? tile_entry(P, s_cnt, s_t0, tile) : make_int2(0, 0);
+      int2 t_nxt = tile + stride < total ? tile_entry(P, s_cnt, s_t0, tile + stride)
+                                         : make_int2(0, 0);
       // raw bucket entries of this lane's source rows r = 4 i + lane / 8 (rows past the
       // tile's end repeat its first row: computed, never stored)
       int raw[BM / 4], raw0;
@@ -494,7 +534,8 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       if (tile < total) load_rows(t, raw, raw0);
       for (; tile < total && !*abort_flag; tile += stride) {
         const int2 t_nn =
-            tile + 2 * stride < total ? P.tile_list[tile + 2 * stride] : make_int2(0, 0);
+            tile + 2 * stride < total ? tile_entry(P, s_cnt, s_t0, tile + 2 * stride)
+                                      : make_int2(0, 0);
         int nraw[BM / 4], nraw0 = 0;
         if (tile + stride < total) load_rows(t_nxt, nraw, nraw0);
         const int n = t.x >> 8;
@@ -561,7 +602,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       if constexpr (GATHER) {
         n_mma = P.prob[0].box_n;
       } else {
-        n_mma = tile_info<false>(P, tile).n;
+        n_mma = tile_info<false>(P, tile, nullptr, nullptr).n;
       }
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -611,7 +652,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
     const int row = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
-      const TileInfo ti = tile_info<GATHER>(P, tile);
+      const TileInfo ti = tile_info<GATHER>(P, tile, s_cnt, s_t0);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       const bool valid = row < ti.rows;
@@ -707,25 +748,6 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   if (warp == L::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
-  }
-  if constexpr (ROUTE) {
-    {
-      // the last CTA to finish forms the routing statistics and the routed-projection tiles
-      __shared__ int s_last;
-      int32_t* ticket = P.ro.cursor + kMaxExperts;
-      if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
-      }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        finalize_dense_routing(P, reinterpret_cast<int*>(scratch),
-                               reinterpret_cast<double*>(scratch + 8 * (kMaxExperts + 8)),
-                               reinterpret_cast<int*>(scratch + 16 * (kMaxExperts + 8)));
-        if (threadIdx.x == 0) *ticket = 0;
-      }
-    }
   }
 }
 
@@ -829,7 +851,7 @@ bool tc_dense_routes(const gqe_ctx* h) { return h->N <= 32 && (h->N & (h->N - 1)
 // fills the buckets, and the last CTA forms the statistics, the aux loss (if aux_out) and
 // the routed-projection tiles.
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, float* aux_out,
+                         const void* W_v, const void* W_shared, int route_set,
                          cudaStream_t st) {
   const int d_h = h->d_h, G = h->G, dim = h->dim;
   const int S = G * h->k + (W_shared ? 1 : 0);
@@ -864,15 +886,19 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   P.G = G;
   P.k = h->k;
   const Workspace& w = h->ws;
-  P.ro = RouteOut{w.logits,  w.sel,    w.psel,   w.gates,     w.w,       w.psum_fx,
-                  w.cursor,  w.bucket, w.counts, w.mean_prob, w.offsets, aux_out,
-                  w.tile_list, w.tile_count};
+  const int cur = route_set & 1, other = cur ^ 1;
+  P.ro = RouteOut{w.logits, w.sel, w.psel, w.gates, w.w,
+                  w.rpsum + cur * kMaxExperts, w.rcur + cur * kMaxExperts,
+                  w.rpsum + other * kMaxExperts, w.rcur + other * kMaxExperts, w.bucket};
   const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
   return route ? launch<false, true>(h, P, grid, st) : launch<false>(h, P, grid, st);
 }
 
 // The tile list (expert | rows << 8, first bucket slot) and its length come from the routing.
-int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStream_t st) {
+// route_set >= 0: schedule from the dense projection's cursor set route_set and write the
+// routing statistics (aux_out if non-null); otherwise from the routing kernel's tile list.
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route_set,
+                    float* aux_out, cudaStream_t st) {
   Params P;
   memset(&P, 0, sizeof(P));
   // A: rows of x gathered four at a time (box one row high, 128 bytes wide)
@@ -889,8 +915,12 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, cudaStrea
   P.bucket = h->ws.bucket;
   P.tile_list = h->ws.tile_list;
   P.tile_count = h->ws.tile_count;
-  P.offsets = h->ws.offsets;
-  P.counts = h->ws.counts;
+  if (route_set >= 0) {
+    P.rc = h->ws.rcur + (route_set & 1) * kMaxExperts;
+    P.rpsum = h->ws.rpsum + (route_set & 1) * kMaxExperts;
+    P.so = StatsOut{h->ws.counts, h->ws.mean_prob, h->ws.offsets, aux_out, h->ws.tile_count};
+  }
+  P.nexp = h->N;
   P.Q = static_cast<__nv_bfloat16*>(h->ws.Q);
   P.E = h->E;
   P.k = h->k;
