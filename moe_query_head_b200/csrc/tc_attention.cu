@@ -39,6 +39,9 @@ namespace gqe {
 bool tmap_bf16_2d_ext(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
                       uint64_t ld, uint32_t box_cols, uint32_t box_rows,
                       CUtensorMapSwizzle sw);
+bool tmap_bf16_chunked(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                       uint64_t ld, uint32_t chunk_cols, uint32_t box_rows,
+                       CUtensorMapSwizzle sw);
 
 namespace {
 
@@ -97,6 +100,7 @@ struct Params {
   const float* psel;
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
   int nq, items;
+  int chunked;  // 1: tm_q / tm_k / tm_v are 3D chunked maps, one copy per tile
   float scale_log2;
   int* next_item;  // [2] item counter and exit counter (zero at launch; the last CTA to
                    // leave sets both back to zero)
@@ -269,9 +273,13 @@ attn_kernel(const __grid_constant__ Params P) {
         q_phase ^= 1;
         mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
         const int qrow = it.s * P.M + it.b * P.T + it.qt * TQ;
+        if (C::NC > 1 && P.chunked) {
+          tma_load_3d(sQ, &P.tm_q, 0, qrow, 0, q_full);
+        } else {
 #pragma unroll
-        for (int c = 0; c < C::NC; ++c)
-          tma_load_2d(sQ + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow, q_full);
+          for (int c = 0; c < C::NC; ++c)
+            tma_load_2d(sQ + c * C::CHUNK_BYTES, &P.tm_q, c * C::CW, qrow, q_full);
+        }
         const int kvh = it.s < P.Sr ? it.s / P.k : 0;
         const int krow0 = kvh * P.M + it.b * P.T;
         for (int j = 0; j < it.nkv; ++j) {
@@ -281,10 +289,14 @@ attn_kernel(const __grid_constant__ Params P) {
             break;
           }
           mbar_arrive_expect_tx(&k_full[kst], C::TILE_BYTES);
+          if (C::NC > 1 && P.chunked) {
+            tma_load_3d(sK + kst * C::TILE_BYTES, &P.tm_k, 0, krow0 + j * TK, 0, &k_full[kst]);
+          } else {
 #pragma unroll
-          for (int c = 0; c < C::NC; ++c)
-            tma_load_2d(sK + kst * C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW,
-                        krow0 + j * TK, &k_full[kst]);
+            for (int c = 0; c < C::NC; ++c)
+              tma_load_2d(sK + kst * C::TILE_BYTES + c * C::CHUNK_BYTES, &P.tm_k, c * C::CW,
+                          krow0 + j * TK, &k_full[kst]);
+          }
           if (++kst == C::K_STAGES) {
             kst = 0;
             k_phase ^= 1;
@@ -322,10 +334,14 @@ attn_kernel(const __grid_constant__ Params P) {
             break;
           }
           mbar_arrive_expect_tx(&v_full[vst], C::TILE_BYTES);
+          if (C::NC > 1 && P.chunked) {
+            tma_load_3d(sV + vst * C::V_BYTES, &P.tm_v, 0, krow0 + j * TK, 0, &v_full[vst]);
+          } else {
 #pragma unroll
-          for (int c = 0; c < C::NC; ++c)
-            tma_load_2d(sV + vst * C::V_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW,
-                        krow0 + j * TK, &v_full[vst]);
+            for (int c = 0; c < C::NC; ++c)
+              tma_load_2d(sV + vst * C::V_BYTES + c * C::CHUNK_BYTES, &P.tm_v, c * C::CW,
+                          krow0 + j * TK, &v_full[vst]);
+          }
           if (++vst == C::V_STAGES) {
             vst = 0;
             v_phase ^= 1;
@@ -669,9 +685,15 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
   const CUtensorMapSwizzle sw = C::CW == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : C::CW == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                               : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, TQ, sw) ||
-      !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw) ||
-      !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw))
+  // One copy per tile where the driver accepts the chunked 3D maps, else one per chunk.
+  P.chunked = C::NC > 1 &&
+              tmap_bf16_chunked(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, TQ, sw) &&
+              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw) &&
+              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw);
+  if (!P.chunked &&
+      (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, TQ, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw)))
     return -1;
   P.Z = static_cast<__nv_bfloat16*>(h->ws.Z);
   P.psel = h->ws.psel;

@@ -844,6 +844,25 @@ bool tmap_bf16_2d_ext(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
   return tmap_bf16_2d(m, ptr, cols, rows, ld, box_cols, box_rows, sw);
 }
 
+// A row-major [rows, cols] bf16 matrix seen as chunks of `chunk_cols` columns: dimensions
+// (column within the chunk, row, chunk), so one box of (chunk_cols, box_rows, cols /
+// chunk_cols) lands in shared memory chunk after chunk, each chunk box_rows x chunk_cols --
+// the layout the per-chunk 2D boxes produce, in one copy. Returns false if the driver does
+// not accept the map (the caller then issues one 2D box per chunk).
+bool tmap_bf16_chunked(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                       uint64_t ld, uint32_t chunk_cols, uint32_t box_rows,
+                       CUtensorMapSwizzle sw) {
+  if (!encoder() || cols % chunk_cols != 0) return false;
+  cuuint64_t dims[3] = {chunk_cols, rows, cols / chunk_cols};
+  cuuint64_t strides[2] = {ld * 2, (cuuint64_t)chunk_cols * 2};
+  cuuint32_t box[3] = {chunk_cols, box_rows, (cuuint32_t)(cols / chunk_cols)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The dense projection routes (see route_rows) for N a power of two up to 32.
 bool tc_dense_routes(const gqe_ctx* h) { return h->N <= 32 && (h->N & (h->N - 1)) == 0; }
 
