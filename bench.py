@@ -66,20 +66,30 @@ def parse_args():
     return a
 
 
+ATTENTION_SOURCES = ("tc_attention.cu", "exp2_fma.cuh", "tc_ptx.cuh", "gqe_common.cuh")
+
+
+def attention_source_sha() -> str:
+    """sha256 over the attention kernel's translation unit and the headers it includes."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTENTION_SOURCES:
+        with open(os.path.join(ROOT, "moe_query_head_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def attention_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu capture, if that capture was
-    taken on this workload and on the current attention source; else None."""
-    import hashlib
+    taken on this workload and on the current attention sources; else None."""
     rec_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
-    src = os.path.join(ROOT, "moe_query_head_b200", "csrc", "tc_attention.cu")
     try:
         with open(rec_path) as f:
             rec = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
+        sha = attention_source_sha()
     except OSError:
         return None
-    if rec.get("source_sha256") != sha or rec.get("workload") != workload:
+    if rec.get("sources_sha256") != sha or rec.get("workload") != workload:
         return None
     return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
 

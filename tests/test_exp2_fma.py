@@ -1,17 +1,18 @@
 """The FMA-pipe exp2 the attention softmax uses for part of its exponentials.
 
-CPU: the algorithm (round-to-nearest range reduction with the 1.5 * 2^23 add, the degree-3
+CPU: the algorithm (round-to-nearest range reduction with the 1.5 * 2^23 add, the degree-2
 polynomial in fp32 Horner form, exponent-field scaling) emulated in numpy float32 against
-float64 exp2: maximum relative error below 8e-5 on [-125, 9], finite and non-negative for
--inf and very negative inputs.
+float64 exp2: maximum relative error below 2e-3 on [-125, 9] (the polynomial's minimax error
+on [-1/2, 1/2] is 1.89e-3; P is rounded to bf16, 1.95e-3, right after), finite and
+non-negative for -inf and very negative inputs.
 GPU: the library's own implementation (gqe_exp2_fma) against CUDA's exp2f (torch.exp2).
 """
 import numpy as np
 import pytest
 import torch
 
-COEF = (0.99992812, 0.69326097, 0.24261054, 0.05517132)
-BOUND = 8e-5
+COEF = (1.00047162, 0.70411982, 0.23876238)
+BOUND = 2e-3
 
 
 def emulate(x):
@@ -21,8 +22,8 @@ def emulate(x):
     n = (j - M).astype(np.float32)
     f = (x - n).astype(np.float32)
     c = [np.float32(v) for v in COEF]
-    p = np.float32(c[3])
-    for k in (2, 1, 0):
+    p = np.float32(c[-1])
+    for k in range(len(c) - 2, -1, -1):
         p = (p * f + c[k]).astype(np.float32)
     bits = (p.view(np.uint32).astype(np.uint64)
             + (j.view(np.uint32).astype(np.uint64) << np.uint64(23))) & np.uint64(0xFFFFFFFF)
@@ -57,4 +58,4 @@ def test_library_exp2_matches_cuda_exp2f():
     rel = (out[:-3].double() / ref - 1).abs().max().item()
     assert rel < BOUND, rel
     tail = out[-3:].cpu()
-    assert torch.isfinite(tail).all() and (tail[:2] < 3e-38).all() and tail[2].item() == pytest.approx(1.0, rel=1e-4)
+    assert torch.isfinite(tail).all() and (tail[:2] < 3e-38).all() and tail[2].item() == pytest.approx(1.0, rel=BOUND)
