@@ -356,3 +356,65 @@ def forward_rows(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v
     return dict(y=y, Z=Z, O=O, sel=sel, gates=rt.gates[rows], w=rt.w[rows],
                 p_sel=rt.p_sel[rows], counts=rt.counts, prob_sum=rt.prob_sum, aux=aux,
                 routing=rt)
+
+
+# ----------------------------------------------------------------------------------------
+# Decode step with a KV cache ([README] Algorithm Overview: the KV heads stay dense and
+# unchanged, so the cache is GQA's; routing and the sparse query heads apply to each new
+# token).
+# ----------------------------------------------------------------------------------------
+
+@dataclass
+class DecodeResult:
+    routing: Routing
+    K_new: np.ndarray      # [G, B, d_h]: the new tokens' keys (written into the cache)
+    V_new: np.ndarray      # [G, B, d_h]
+    K_cache: np.ndarray    # [G, B, L_max, d_h] after the step
+    V_cache: np.ndarray
+    Q: np.ndarray          # [S, B, d_h]
+    O: np.ndarray          # [S, B, d_h]
+    Z: np.ndarray          # [B, D_o]
+    y: np.ndarray          # [B, d]
+    aux: float
+
+
+def decode(layer: Layer, x: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray, lengths,
+           W_r, W_q, W_k, W_v, W_shared, W_o) -> DecodeResult:
+    """One generation step for B sequences (float64 arrays).
+
+    x [B, dim] holds each sequence's next token, at position lengths[b]; K_cache / V_cache
+    [G, B, L_max, d_h] hold the keys and values of positions 0 .. lengths[b]-1. The new
+    token's K and V are written at position lengths[b] of copies of the caches (the inputs
+    are not modified), and its output is the causal attention over positions
+    0 .. lengths[b], i.e. row lengths[b] of the prefill forward over the whole sequence.
+    """
+    if not layer.causal:
+        raise ValueError("a decode step is causal")
+    B = x.shape[0]
+    G, k, d_h = layer.G, layer.k, layer.d_h
+    L_max = K_cache.shape[2]
+    lengths = np.asarray(lengths, dtype=np.int64)
+    if lengths.shape != (B,) or np.any(lengths < 0) or np.any(lengths >= L_max):
+        raise ValueError("every position must lie inside the cache")
+    rt = route(x, W_r, G, k)
+    K_new, V_new = kv_projection(x, W_k, W_v, G, d_h)
+    Kc = K_cache.copy()
+    Vc = V_cache.copy()
+    for b in range(B):
+        Kc[:, b, lengths[b]] = K_new[:, b]
+        Vc[:, b, lengths[b]] = V_new[:, b]
+    Q = routed_queries(x, W_q, rt.sel, G, layer.E, d_h)
+    if layer.shared:
+        Q = np.concatenate([Q, shared_query(x, W_shared)[None]], axis=0)
+    S = Q.shape[0]
+    O = np.empty((S, B, d_h))
+    for s in range(S):
+        h = stream_kv_head(s, k, G)
+        for b in range(B):
+            n = lengths[b] + 1  # the cached positions and the new one
+            O[s, b] = attention_rows(Q[s, b][None], np.array([lengths[b]]), Kc[h, b, :n],
+                                     Vc[h, b, :n], True)[0]
+    Z = combine(O, rt, layer)
+    y = output_projection(Z, W_o)
+    aux = aux_loss(rt.counts, rt.prob_sum, B, G, k)
+    return DecodeResult(rt, K_new, V_new, Kc, Vc, Q, O, Z, y, aux)
