@@ -45,6 +45,8 @@ if ROOT not in sys.path:
 from moe_query_head_b200 import workloads as W  # noqa: E402
 
 METRIC = "GQE prefill tokens/s @1 B200; % bf16 tensor peak (active FLOPs); speedup vs k=E"
+DECODE_METRIC = "GQE decode tokens/s @1 B200 (one new token per sequence over its KV cache)"
+DECODE_BASE = "main_b8_t2048"  # the paper's layer shapes: dim 768, N 16, G 8, k 1, d_h 48
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
@@ -59,6 +61,11 @@ def parse_args():
     ap.add_argument("--variant", default=None, choices=["gqe", "weighted_concat", "hard_concat"],
                     help="output construction (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"],
+                    help="prefill (default, the headline) or one decode step with a KV cache")
+    ap.add_argument("--decode-batch", type=int, default=64, help="decode: sequences per step")
+    ap.add_argument("--decode-len", type=int, default=8192,
+                    help="decode: tokens already cached per sequence")
     ap.add_argument("--cpu-rows", type=int, default=8192,
                     help="query rows in the oracle's bounded sample")
     a = ap.parse_args()
@@ -448,11 +455,203 @@ def bench_ours(args, rank, world, dist):
     return res, inp
 
 
+# ----------------------------------------------------------------------------------------
+# Decode mode: one gqe_decode step (one new token per sequence over its KV cache).
+# ----------------------------------------------------------------------------------------
+
+def decode_workload(args):
+    wl = W.WORKLOADS[DECODE_BASE].with_(B=args.decode_batch, T=1)
+    if args.variant:
+        wl = wl.with_(variant=args.variant)
+    return wl
+
+
+def oracle_decode_sample(wl, L: int, n_seq: int) -> dict:
+    """The float64 oracle's decode step on n_seq sequences with L cached tokens each (the
+    same layer and cache length as the GPU run; seeded host inputs)."""
+    from oracle import gqe_oracle as go
+    sub = wl.with_(B=n_seq)
+    d = W.generate_decode(sub, [L] * n_seq, L + 1)
+    inp = d.inp
+    layer = go.Layer(wl.dim, wl.N, wl.G, wl.k, wl.d_h, shared=wl.shared, variant=wl.variant)
+    args64 = [inp.f64(n) for n in ("W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")]
+    kc, vc, x = d.k_cache.astype(np.float64), d.v_cache.astype(np.float64), inp.f64("x")
+    t0 = time.perf_counter()
+    go.decode(layer, x, kc, vc, d.lengths, *args64)
+    dt = time.perf_counter() - t0
+    return {"seconds": dt, "tokens_per_s": n_seq / dt,
+            "sample": f"{n_seq} sequences of the decode workload ({L} cached tokens each), "
+                      f"float64 numpy oracle; tokens/s of that sample"}
+
+
+def bench_decode(args, rank, world, dist):
+    import torch
+    from moe_query_head_b200 import gqe as G
+
+    wl = decode_workload(args)
+    B, L = args.decode_batch, args.decode_len
+    L_max = L + 64
+    inp = W.generate(wl)  # the B new tokens and the layer's weights
+    dev = _upload(inp, torch)
+    variant = W.VARIANT_IDS[wl.variant]
+    W_s = dev["W_shared"] if wl.shared else None
+    # caches: seeded normal values with the spread of a projected K/V element (bf16, on the
+    # device; together larger than L2, so no flush is needed between steps)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(wl.seed + 2000)
+    sd = (wl.w_std if wl.w_std is not None else (1.0 / wl.dim) ** 0.5) * wl.dim ** 0.5
+    shape = (wl.G, B, L_max, wl.d_h)
+    kc = torch.randn(shape, generator=gen, device="cuda", dtype=torch.bfloat16).mul_(sd)
+    vc = torch.randn(shape, generator=gen, device="cuda", dtype=torch.bfloat16).mul_(sd)
+    lengths = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    h = G.gqe_create(wl.dim, wl.N, wl.G, wl.k, wl.d_h, G.GQE_BF16, B)
+    out = torch.empty((B, wl.dim), dtype=torch.bfloat16, device="cuda")
+    aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+    kE = wl.all_active()
+    hE = G.gqe_create(wl.dim, wl.N, wl.G, kE.k, wl.d_h, G.GQE_BF16, B)
+    W_oE = (torch.randn((wl.dim, kE.D_o), generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+    outE = torch.empty_like(out)
+
+    def step(handle, k, W_o, o, x=None, stream=None):
+        G.gqe_decode(handle, dev["x"] if x is None else x, B, kc, vc, L_max, lengths,
+                     dev["W_r"], dev["W_q"], dev["W_k"], dev["W_v"], W_s, W_o, wl.N, wl.G, k,
+                     wl.d_h, variant, o, aux, stream=stream)
+
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(G.GQE_NUM_STAGES + 1)]
+    for e in stage_ev:
+        e.record()
+    torch.cuda.synchronize()
+
+    def timed(fn, steps, stages=None):
+        s_ev = torch.cuda.Event(enable_timing=True)
+        e_ev = torch.cuda.Event(enable_timing=True)
+        total = 0.0
+        st_tot = np.zeros(G.GQE_NUM_STAGES)
+        for _ in range(steps):
+            s_ev.record()
+            fn()
+            e_ev.record()
+            torch.cuda.synchronize()
+            total += s_ev.elapsed_time(e_ev)
+            if stages:
+                for i in range(G.GQE_NUM_STAGES):
+                    st_tot[i] += stages[i].elapsed_time(stages[i + 1])
+        return total, st_tot
+
+    gpu_id = torch.cuda.get_device_properties(0).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    for _ in range(args.warmup):
+        step(h, wl.k, dev["W_o"], out)
+        step(hE, kE.k, W_oE, outE)
+    torch.cuda.synchronize()
+    st = G.gqe_check_device_status(h)
+    if st != G.GQE_OK:
+        raise RuntimeError("device status after warm-up: " + G.status_str(st))
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms, _ = timed(lambda: step(h, wl.k, dev["W_o"], out), args.steps)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = G.gqe_kernel_launches(h)
+    G.gqe_set_stage_events(h, stage_ev)
+    _, stage_ms = timed(lambda: step(h, wl.k, dev["W_o"], out), args.steps, stage_ev)
+    G.gqe_set_stage_events(h, None)
+    totalE_ms, _ = timed(lambda: step(hE, kE.k, W_oE, outE), args.steps)
+    # end to end through the API: each step copies its tokens in from pinned host memory
+    # and its output and aux loss back out, on the same stream
+    x_host = dev["x"].cpu().pin_memory()
+    y_host = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(dev["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        step(h, wl.k, dev["W_o"], out, x=x_dev)
+        y_host.copy_(out, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+
+    e2e_ms, _ = timed(e2e_step, args.steps)
+    clocks = sampler.stop()
+    st = G.gqe_check_device_status(h)
+    if st != G.GQE_OK:
+        raise RuntimeError("device status after timing: " + G.status_str(st))
+    att_i = [G.gqe_stage_name(i) for i in range(G.GQE_NUM_STAGES)].index("attention")
+    att_tot = float(stage_ms[att_i])
+    if dist:
+        total_ms, totalE_ms, e2e_ms, att_tot = reduce_max_over_ranks(
+            [total_ms, totalE_ms, e2e_ms, att_tot], dist, "cuda")
+    peaks, peak_src = load_peaks()
+    ms = total_ms / args.steps
+    # algorithmic bytes of the cache attention: every cached K and V row read once, the new
+    # rows read from the workspace and written into the caches
+    kv_bytes = B * wl.G * (L + 1) * wl.d_h * 2 * 2 + B * wl.G * wl.d_h * 2 * 2
+    att_ms = att_tot / args.steps
+    gbs = kv_bytes / (att_ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    res = {
+        "metric": DECODE_METRIC, "value": B * world / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal tokens, caches and random-init weights of the layer "
+                "shapes)",
+        "config": {"workload": f"decode_b{B}_l{L}", "dim": wl.dim, "N": wl.N, "G": wl.G,
+                   "k": wl.k, "d_h": wl.d_h, "B": B, "cache_len": L, "L_max": L_max,
+                   "variant": wl.variant, "shared": wl.shared,
+                   "l2": f"caches ({2 * kc.numel() * 2 / 2**30:.2f} GiB) larger than L2; "
+                         f"no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "speedup_vs_kE": (totalE_ms / args.steps) / ms,
+        "kE_tokens_per_s": B * world / (totalE_ms / args.steps / 1e3),
+        "stages_ms": {G.gqe_stage_name(i): float(stage_ms[i] / args.steps)
+                      for i in range(G.GQE_NUM_STAGES)},
+        "roofline": {"kernel": "decode attention (cache read, merge)", "bound": "hbm",
+                     "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "algorithmic_bytes": kv_bytes},
+        "e2e": {"value": B * world / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2 + 4)},
+        "gpu_launches": int(launches * args.steps),
+        "clocks": clocks,
+    }
+    G.gqe_destroy(h)
+    G.gqe_destroy(hE)
+    return res, wl
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference" and args.mode == "decode":
+        if rank != 0:
+            return 0
+        wl = decode_workload(args)
+        n_seq = 4
+        for _ in range(args.warmup):
+            oracle_decode_sample(wl, args.decode_len, n_seq)
+        samples = [oracle_decode_sample(wl, args.decode_len, n_seq) for _ in range(args.steps)]
+        value = sum(s["tokens_per_s"] for s in samples) / len(samples)
+        res = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "tokens/s",
+               "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": args.decode_batch / value * 1e3, "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": f"decode_b{args.decode_batch}_l{args.decode_len}",
+                          "dim": wl.dim, "N": wl.N, "G": wl.G, "k": wl.k, "d_h": wl.d_h,
+                          "B": args.decode_batch, "cache_len": args.decode_len,
+                          "variant": wl.variant},
+               "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": samples[0]["sample"]},
+               "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return 0
 
     if args.impl == "reference":
         if rank != 0:
@@ -491,6 +690,19 @@ def main():
         dist = td
     else:
         torch.cuda.set_device(0)
+    if args.mode == "decode":
+        res, wl = bench_decode(args, rank, world, dist)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                s = oracle_decode_sample(wl, args.decode_len, 4)
+                res["cpu_baseline"] = {"value": s["tokens_per_s"], "unit": "tokens/s",
+                                       "cores": blas_threads(), "kind": "oracle",
+                                       "sample": s["sample"], "seconds": s["seconds"]}
+            print(json.dumps(res))
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
     res, inp = bench_ours(args, rank, world, dist)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:

@@ -116,6 +116,37 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
                        void* out, float* aux_loss, void* stream);
 
 /*
+ * gqe_decode — one generation step with a KV cache: for each of B sequences, its next token
+ * at position lengths[b]. GQE keeps the KV heads dense and unchanged (README, Algorithm
+ * Overview), so the cache is GQA's; the new token is routed, its selected query heads and the
+ * shared head are projected, and each attends over positions 0 .. lengths[b] of its KV head.
+ * The result equals row lengths[b] of gqe_forward (causal) over the whole sequence.
+ *
+ *   x         [B, dim]               the new tokens.
+ *   k_cache,  [G, B, L_max, d_h]     caller-owned caches in the handle's dtype; rows
+ *   v_cache                          0 .. lengths[b]-1 of (g, b) hold K / V of those positions.
+ *                                    The step writes the new token's K / V at row lengths[b]
+ *                                    and reads no row after it; no other row is written.
+ *   L_max     rows per (group, sequence) in the caches, >= 1.
+ *   lengths   [B] int32, DEVICE      positions of the new tokens, 0 <= lengths[b] < L_max.
+ *                                    Not modified: the caller advances them after the step.
+ *   W_*, N, G, k, d_h, variant, out [B, dim], aux_loss, stream: as gqe_forward (the aux loss
+ *                                    is the Switch loss over the B new tokens).
+ *
+ * bf16 handles only (GQE_ERR_UNSUPPORTED for fp32, or for B > 65535). Requires
+ * B <= max_tokens (GQE_ERR_WORKSPACE). Allocates nothing and does not synchronise; the routing and tensors
+ * of the step are available through gqe_get_routing / gqe_get_tensor (M = B). A position
+ * outside [0, L_max) cannot be checked on the host: the step then reads and writes nothing
+ * for that sequence, leaves its output undefined, and the next gqe_check_device_status
+ * returns GQE_ERR_INVALID_ARG. Other errors as gqe_forward.
+ */
+gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v_cache,
+                      int L_max, const int32_t* lengths, const void* W_r, const void* W_q,
+                      const void* W_k, const void* W_v, const void* W_shared, const void* W_o,
+                      int N, int G, int k, int d_h, int variant, void* out, float* aux_loss,
+                      void* stream);
+
+/*
  * gqe_get_routing — copy the routing of the last gqe_forward on this handle.
  *   sel        [M, G, k] int32   selected expert index j within the group, ascending.
  *   gates      [M, G, k] float   p renormalised within the group (sums to 1 per group).
@@ -136,8 +167,8 @@ gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void
 /*
  * gqe_check_device_status — synchronise `stream`, then read and clear the handle's device
  * status word. Returns GQE_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
- * check (its output is then invalid), GQE_ERR_CUDA if the stream reports an error, else
- * GQE_OK.
+ * check (its output is then invalid), GQE_ERR_INVALID_ARG if a gqe_decode met a position
+ * outside its cache, GQE_ERR_CUDA if the stream reports an error, else GQE_OK.
  */
 gqe_status gqe_check_device_status(gqe_handle h, void* stream);
 

@@ -68,6 +68,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.cursor = (int32_t*)take((kMaxExperts + 4) * 4);
   w.rcur = (int32_t*)take(2 * kMaxExperts * 4);
   w.rpsum = (unsigned long long*)take(2 * kMaxExperts * 8);
+  w.dec_part = (float*)take((size_t)kDecodeSlots * (k + 1) * (d_h + 2) * 4);
   w.status = (int32_t*)take(16);
   (void)dim;
   return off;
@@ -246,6 +247,67 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   return ok ? GQE_OK : GQE_ERR_CUDA;
 }
 
+gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v_cache,
+                      int L_max, const int32_t* lengths, const void* W_r, const void* W_q,
+                      const void* W_k, const void* W_v, const void* W_shared, const void* W_o,
+                      int N, int G, int k, int d_h, int variant, void* out, float* aux_loss,
+                      void* stream) {
+  if (!h) return GQE_ERR_INVALID_ARG;
+  if (N != h->N || G != h->G || k != h->k || d_h != h->d_h) return GQE_ERR_INVALID_ARG;
+  if (B < 1 || L_max < 1) return GQE_ERR_INVALID_ARG;
+  if (variant < GQE_VARIANT_GQE || variant > GQE_VARIANT_HARD_CONCAT) return GQE_ERR_INVALID_ARG;
+  if (!x || !W_r || !W_q || !W_k || !W_v || !W_o || !out || !k_cache || !v_cache || !lengths)
+    return GQE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_r, W_q, W_k, W_v, W_o, out, k_cache, v_cache};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GQE_ERR_INVALID_ARG;
+  if (W_shared && !aligned16(W_shared)) return GQE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lengths) & 3u) return GQE_ERR_INVALID_ARG;
+  if (aux_loss && (reinterpret_cast<uintptr_t>(aux_loss) & 3u)) return GQE_ERR_INVALID_ARG;
+  if (h->dtype != GQE_BF16) return GQE_ERR_UNSUPPORTED;
+  if (B > 65535) return GQE_ERR_UNSUPPORTED;  // one grid row per sequence
+  if (B > h->max_tokens) return GQE_ERR_WORKSPACE;
+  const int M = B;
+  const int has_shared = W_shared != nullptr;
+  const int S = G * k + has_shared;
+  const int Do = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  int launches = 0;
+  int stage = 0;
+  auto add = [&](int n) -> bool {
+    if (h->n_stage_events) cudaEventRecord(h->stage_events[stage], st);
+    ++stage;
+    if (n < 0) return false;
+    launches += n;
+    return true;
+  };
+  auto mark = [&]() {
+    if (h->n_stage_events) cudaEventRecord(h->stage_events[stage], st);
+    ++stage;
+    return true;
+  };
+  // the forward's stages on the B new tokens, with the cache attention in place of the
+  // prefill attention
+  const bool fused = tc_dense_routes(h);
+  const int rs = h->route_set;
+  int dense = -1;
+  bool ok = mark() &&
+            add(dense = launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, rs, st)) &&
+            add(fused ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
+            add(launch_tc_qproj(h, x, M, W_q, fused ? rs : -1, aux_loss, st)) &&
+            add(launch_tc_decode_attention(h, B, S, has_shared, variant, Do, k_cache, v_cache,
+                                           L_max, lengths, st)) &&
+            add(launch_combine(h, M, variant, Do, st)) &&
+            add(launch_tc_oproj(h, M, Do, W_o, out, st));
+  if (fused && dense >= 0) h->route_set ^= 1;
+  h->last_M = M;
+  h->last_S = S;
+  h->last_Do = Do;
+  h->last_launches = launches;
+  return ok ? GQE_OK : GQE_ERR_CUDA;
+}
+
 gqe_status gqe_get_routing(gqe_handle h, int32_t* sel, float* gates, int32_t* counts,
                            float* mean_prob, void* stream) {
   if (!h || h->last_M == 0) return GQE_ERR_INVALID_ARG;
@@ -295,7 +357,7 @@ gqe_status gqe_check_device_status(gqe_handle h, void* stream) {
   if (cudaMemcpy(&v, h->ws.status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return GQE_ERR_CUDA;
   if (v != kStatusOk) {
     cudaMemset(h->ws.status, 0, 4);
-    return GQE_ERR_TIMEOUT;
+    return v == kStatusBadInput ? GQE_ERR_INVALID_ARG : GQE_ERR_TIMEOUT;
   }
   return GQE_OK;
 }

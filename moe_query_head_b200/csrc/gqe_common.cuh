@@ -18,6 +18,12 @@ constexpr int kMaxTopK = 8;
 // Device status word values (written by kernels whose bounded waits give up).
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadInput = 2;  // a decode position outside its cache
+
+// Partial-result slots of the decode attention: (sequence, group, key chunk) triples whose
+// (m, l, O) are merged by a second kernel. Bounded independently of the cache length (the
+// chunks grow with it), so the handle's workspace holds them.
+constexpr int kDecodeSlots = 1024;
 
 // ---------------------------------------------------------------------------------------
 // Programmatic dependent launch. The forward's kernels are launched with it: a kernel may
@@ -97,6 +103,7 @@ struct Workspace {
   unsigned long long* rpsum = nullptr;    // [2, kMaxExperts]
   int32_t* cursor = nullptr;       // [kMaxExperts] bucket cursors, then the routing ticket
                                    // (zero between calls)
+  float* dec_part = nullptr;       // [kDecodeSlots, k + 1, d_h + 2] decode partial (m, l, O)
   int32_t* status = nullptr;       // device status word
   void* base = nullptr;            // the single allocation
   size_t bytes = 0;
@@ -160,5 +167,11 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,
                         int causal, int Do, cudaStream_t st);
+// Decode step: attention of one new token per sequence over its KV cache, and the append of
+// the new token's K/V (decode.cu). bf16 handles.
+int launch_tc_decode_attention(gqe_ctx* h, int B, int S, int has_shared, int variant, int Do,
+                               void* k_cache, void* v_cache, int L_max, const int32_t* lengths,
+                               cudaStream_t st);
+int decode_chunks(const gqe_ctx* h, int B, int L_max);
 
 }  // namespace gqe

@@ -23,7 +23,8 @@ TENSORS = {"K": 0, "V": 1, "Q": 2, "Z": 3, "PSEL": 4, "W": 5, "LOGITS": 6}
 EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
-            "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma", "gqe_selftest_timeout")
+            "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma", "gqe_selftest_timeout",
+            "gqe_decode")
 GQE_NUM_STAGES = 6
 
 
@@ -44,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.gqe_create.restype = I
     lib.gqe_forward.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
     lib.gqe_forward.restype = I
+    lib.gqe_decode.argtypes = [P, P, I, P, P, I, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P]
+    lib.gqe_decode.restype = I
     lib.gqe_get_routing.argtypes = [P, P, P, P, P, P]
     lib.gqe_get_routing.restype = I
     lib.gqe_get_tensor.argtypes = [P, I, P, SZ, P]
@@ -109,6 +112,16 @@ def gqe_forward(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, var
     _check(lib.gqe_forward(h, _ptr(x), B, T, _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v),
                            _ptr(W_shared), _ptr(W_o), N, G, k, d_h, variant, causal, _ptr(out),
                            _ptr(aux_loss), _stream(stream)), "gqe_forward")
+
+
+def gqe_decode(h, x, B, k_cache, v_cache, L_max, lengths, W_r, W_q, W_k, W_v, W_shared, W_o,
+               N, G, k, d_h, variant, out, aux_loss=None, stream=None) -> None:
+    """One generation step with a KV cache (see include/gqe.h); lengths is an int32 device
+    tensor and is not modified."""
+    _check(lib.gqe_decode(h, _ptr(x), B, _ptr(k_cache), _ptr(v_cache), L_max, _ptr(lengths),
+                          _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(W_shared), _ptr(W_o),
+                          N, G, k, d_h, variant, _ptr(out), _ptr(aux_loss), _stream(stream)),
+           "gqe_decode")
 
 
 def gqe_get_routing(h, sel=None, gates=None, counts=None, mean_prob=None, stream=None) -> None:

@@ -255,6 +255,42 @@ def generate(wl: Workload) -> Inputs:
     return Inputs(wl, x, W_r, W_q, W_k, W_v, W_s if wl.shared else None, W_o, report)
 
 
+@dataclass
+class DecodeInputs:
+    """One decode step's inputs: `inp` holds the B new tokens (x [B, dim], one per
+    sequence, margin filter applied) and the layer's weights; the caches hold values exact
+    in bf16 (float32 containers)."""
+
+    inp: Inputs
+    k_cache: np.ndarray    # [G, B, L_max, d_h]
+    v_cache: np.ndarray
+    lengths: np.ndarray    # [B] int32: the new tokens' positions
+
+    def raw_cache(self, name: str) -> np.ndarray:
+        return f32_to_bf16_bits(getattr(self, name))
+
+
+def generate_decode(wl: Workload, lengths, L_max: int) -> DecodeInputs:
+    """A decode step on the workload's layer: B = len(lengths) sequences, each with one new
+    token (drawn as generate(wl with B, T = 1) draws its x and weights) at position
+    lengths[b] < L_max. Cache entries are N(0, s^2) with s the standard deviation of a
+    projected K/V element under the workload's weights (sqrt(dim) * weight std, x ~ N(0, 1)),
+    from PCG64([seed, 2]); rows at and after each position are drawn too (the step must not
+    read them)."""
+    lengths = np.asarray(lengths, dtype=np.int32)
+    B = lengths.size
+    if lengths.min() < 0 or lengths.max() >= L_max:
+        raise ValueError("every position must lie inside the cache")
+    inp = generate(wl.with_(B=B, T=1))
+    std = wl.w_std if wl.w_std is not None else (1.0 / wl.dim) ** 0.5
+    s = std * wl.dim ** 0.5
+    rng = np.random.Generator(np.random.PCG64([wl.seed, 2]))
+    shape = (wl.G, B, L_max, wl.d_h)
+    k_cache = quantize(rng.standard_normal(shape, dtype=np.float32) * s, "bf16")
+    v_cache = quantize(rng.standard_normal(shape, dtype=np.float32) * s, "bf16")
+    return DecodeInputs(inp, k_cache, v_cache, lengths)
+
+
 @lru_cache(maxsize=4)
 def cached(name: str, **overrides) -> Inputs:
     wl = WORKLOADS[name]
