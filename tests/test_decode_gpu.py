@@ -5,9 +5,10 @@ written at its position (equal to the step's own projection, and to the oracle's
 rounding) and every other cache row left bit-identical.
 
 Cases cover both ways the attention runs (one CTA per sequence and group writing Z
-directly, and split key chunks merged by a second kernel), ragged positions (0, tile edges,
-long), the three variants, head dims 48 / 64 / 128, a layer without the shared head, and the
-consistency of a decode step with the GPU prefill row at the same position."""
+directly when there are at least four such pairs per SM, and split key chunks merged by a
+second kernel), ragged positions (0, tile edges, long), the three variants, head dims
+48 / 64 / 128, a layer without the shared head, and the consistency of a decode step with
+the GPU prefill row at the same position."""
 import numpy as np
 import pytest
 import torch
@@ -110,10 +111,13 @@ WIDE = W.WORKLOADS["wide_k2"]
 LARGE = W.WORKLOADS["large_skew"].with_(skew=None)
 
 CASES = {
-    # B * G = 56 < 2 SMs' worth of CTAs: split key chunks, merged
+    # B * G = 56, far fewer than four per SM: many key chunks per pair, merged
     "main_split_ragged": (MAIN, [0, 1, 63, 64, 65, 700, 1023], 1024),
-    # B * G = 320: one CTA per (sequence, group), Z written directly
-    "main_direct_batch40": (MAIN, list(np.random.default_rng(3).integers(0, 300, 40)), 320),
+    # B * G = 640 (at least four CTAs per SM of a B200 without splitting): one CTA per
+    # (sequence, group), Z written directly
+    "main_direct_batch80": (MAIN, list(np.random.default_rng(3).integers(0, 300, 80)), 320),
+    # B * G = 320: two key chunks per (sequence, group), merged
+    "main_split_batch40": (MAIN, list(np.random.default_rng(5).integers(0, 300, 40)), 320),
     "main_no_shared_hard": (MAIN.with_(shared=False, variant="hard_concat"), [9, 129, 257], 384),
     "main_all_active": (MAIN.with_(k=2), [0, 77, 500], 512),
     "wide_gqe": (WIDE, [5, 200, 511], 512),
@@ -129,8 +133,8 @@ def test_decode_matches_oracle(case):
     _check(W.generate_decode(wl, lengths, L_max))
 
 
-def test_decode_long_cache_split_and_direct():
-    """Long caches: one sequence (split into many chunks) and 64 sequences (direct)."""
+def test_decode_long_caches():
+    """Long caches: one sequence (split into many chunks) and 64 sequences (two chunks each)."""
     _check(W.generate_decode(MAIN, [8191], 8192))
     rng = np.random.default_rng(4)
     _check(W.generate_decode(MAIN, list(rng.integers(2000, 4096, 64)), 4096))
