@@ -1,4 +1,5 @@
-"""CPU oracle for the Grouped Query Experts (GQE) attention forward (prefill) pass.
+"""CPU oracle for Grouped Query Experts (GQE) attention: the forward (prefill) pass, the
+decode step with a KV cache, and the backward pass.
 
 TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.
@@ -22,7 +23,11 @@ Sources (by page title and section):
 Pins (tests/test_oracle_pins.py): brute-force routing on tiny inputs, closed forms of
 the gates and of the aux loss, torch's float64 scaled_dot_product_attention, the
 reduction to an independently written dense GQA layer at k = E, and the
-identical-experts collapse. Every function below is pinned; none is "parity unpinned".
+identical-experts collapse. The decode step (tests/test_oracle_decode_pins.py) is pinned to
+the forward's row at the new position and to the single-key closed form; the backward pass
+(tests/test_oracle_backward_pins.py) to torch autograd through an independently written
+forward and to finite differences of the forward. Every function below is pinned; none is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -418,3 +423,137 @@ def decode(layer: Layer, x: np.ndarray, K_cache: np.ndarray, V_cache: np.ndarray
     y = output_projection(Z, W_o)
     aux = aux_loss(rt.counts, rt.prob_sum, B, G, k)
     return DecodeResult(rt, K_new, V_new, Kc, Vc, Q, O, Z, y, aux)
+
+
+# ----------------------------------------------------------------------------------------
+# Backward pass: gradients of F = <dy, y> + dA * L, the top-k selection held constant
+# ([README] Usage: the aux loss joins the task loss; [Summary] Output Construction: the
+# renormalised slot is the router's differentiable path). Each step is the derivative of the
+# forward step of the same name, taken in reverse order.
+# ----------------------------------------------------------------------------------------
+
+@dataclass
+class Grads:
+    x: np.ndarray
+    W_r: np.ndarray
+    W_q: np.ndarray
+    W_k: np.ndarray
+    W_v: np.ndarray
+    W_shared: np.ndarray | None
+    W_o: np.ndarray
+
+
+def attention_rows_backward(q: np.ndarray, t_pos: np.ndarray, K: np.ndarray, V: np.ndarray,
+                            dO: np.ndarray, causal: bool):
+    """Gradients of O = softmax(q K^T / sqrt(d_h)) V (rows at positions t_pos; keys u <= t
+    when causal) with respect to q, K and V, given dO. With P the probabilities:
+    dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)), dq = dS K / sqrt(d_h),
+    dK = dS^T q / sqrt(d_h)."""
+    d_h = q.shape[1]
+    T = K.shape[0]
+    scale = 1.0 / math.sqrt(d_h)
+    s = (q @ K.T) * scale
+    if causal:
+        u = np.arange(T)[None, :]
+        s = np.where(u <= t_pos[:, None], s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    P = e / e.sum(axis=1, keepdims=True)
+    O = P @ V
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - (dO * O).sum(axis=1, keepdims=True))
+    return (dS @ K) * scale, (dS.T @ q) * scale, dV
+
+
+def backward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_shared, W_o,
+             dy: np.ndarray, dA: float = 0.0) -> Grads:
+    """Gradients of <dy, y> + dA * L (y, L: the forward's output and aux loss) with respect to
+    x and every weight. The selected sets are the forward's; see the definition's section on
+    the backward pass for what is differentiated."""
+    M = x.shape[0]
+    G, k, E, d_h, N = layer.G, layer.k, layer.E, layer.d_h, layer.N
+    fw = forward(layer, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o)
+    rt = fw.routing
+    # y = Z W_o^T
+    dW_o = dy.T @ fw.Z
+    dZ = dy @ W_o
+    # output construction (column blocks: routed g-major then r, slot, shared)
+    dO = np.zeros_like(fw.O)
+    dp_sel = np.zeros((M, G, k))
+    col = 0
+    for g in range(G):
+        for r in range(k):
+            s = g * k + r
+            blk = dZ[:, col:col + d_h]
+            col += d_h
+            if layer.variant == "weighted_concat":
+                dO[s] += rt.p_sel[:, g, r][:, None] * blk
+                dp_sel[:, g, r] += (blk * fw.O[s]).sum(axis=1)
+            else:
+                dO[s] += blk
+    if layer.variant == "gqe":
+        dslot = dZ[:, col:col + d_h]
+        col += d_h
+        dw = np.zeros((M, G, k))
+        for g in range(G):
+            for r in range(k):
+                s = g * k + r
+                dO[s] += rt.w[:, g, r][:, None] * dslot
+                dw[:, g, r] = (dslot * fw.O[s]).sum(axis=1)
+        # w = p_sel / P_t with P_t the token's sum of selected p: both are differentiated
+        P_t = rt.p_sel.sum(axis=(1, 2))
+        dp_sel += (dw - (dw * rt.w).sum(axis=(1, 2), keepdims=True)) / P_t[:, None, None]
+    if layer.shared:
+        dO[G * k] += dZ[:, col:col + d_h]
+    # router: p of the selected experts, the aux loss's mean p, the per-group softmax
+    dp = np.zeros((M, G, E))
+    mi = np.arange(M)
+    for g in range(G):
+        for r in range(k):
+            dp[mi, g, rt.sel[:, g, r]] += dp_sel[:, g, r]
+    if dA:
+        f = rt.counts.reshape(G, E).astype(np.float64) / (M * k)
+        dp += dA * (E / G) * f[None] / M  # dL / dp[t, g, j] = (1/G) E f[g, j] / M
+    dl = rt.p * (dp - (rt.p * dp).sum(axis=2, keepdims=True))
+    dl = dl.reshape(M, N)
+    dW_r = dl.T @ x
+    dx = dl @ W_r
+    # attention, per stream and sequence; K / V gradients add up over the streams of a head
+    dQ = np.zeros_like(fw.Q)
+    dK = np.zeros_like(fw.K)
+    dV = np.zeros_like(fw.V)
+    pos = np.arange(T)
+    for s in range(fw.Q.shape[0]):
+        h = stream_kv_head(s, k, G)
+        for b in range(B):
+            rows = slice(b * T, (b + 1) * T)
+            dq, dk, dv = attention_rows_backward(fw.Q[s, rows], pos, fw.K[h, rows],
+                                                 fw.V[h, rows], dO[s, rows], layer.causal)
+            dQ[s, rows] = dq
+            dK[h, rows] += dk
+            dV[h, rows] += dv
+    # projections
+    dW_k = np.zeros_like(W_k)
+    dW_v = np.zeros_like(W_v)
+    for g in range(G):
+        rg = slice(g * d_h, (g + 1) * d_h)
+        dW_k[rg] = dK[g].T @ x
+        dW_v[rg] = dV[g].T @ x
+        dx += dK[g] @ W_k[rg] + dV[g] @ W_v[rg]
+    dW_q = np.zeros_like(W_q)
+    for g in range(G):
+        for r in range(k):
+            s = g * k + r
+            for j in range(E):
+                rows = np.nonzero(rt.sel[:, g, r] == j)[0]
+                if rows.size == 0:
+                    continue
+                re = slice((g * E + j) * d_h, (g * E + j + 1) * d_h)
+                dW_q[re] += dQ[s, rows].T @ x[rows]
+                dx[rows] += dQ[s, rows] @ W_q[re]
+    dW_s = None
+    if layer.shared:
+        dW_s = dQ[G * k].T @ x
+        dx += dQ[G * k] @ W_shared
+    return Grads(dx, dW_r, dW_q, dW_k, dW_v, dW_s, dW_o)
