@@ -124,3 +124,46 @@ def test_decode_rejects_positions_outside_the_cache():
         go.decode(layer, x, Kc, Kc, [0, 4], *W)
     with pytest.raises(ValueError):
         go.decode(go.Layer(dim=16, N=4, G=2, k=1, d_h=4, causal=False), x, Kc, Kc, [0, 1], *W)
+
+
+# ---------------------------------------------------------------------------------------
+# Planted mistakes: each must make one of the pins above fail.
+# ---------------------------------------------------------------------------------------
+
+def _decode_attending_one_key_short(layer, x, K_cache, V_cache, lengths, *W):
+    """The new token left out of its own attention (keys 0 .. L-1 only)."""
+    real_rows = go.attention_rows
+
+    def short(q, t_pos, K, V, causal, chunk=1024):
+        n = K.shape[0]
+        if n == 1:  # nothing else to attend to: repeat the only key so the call stays valid
+            return real_rows(q, t_pos, K, V, causal, chunk)
+        return real_rows(q, t_pos - 1, K[:n - 1], V[:n - 1], causal, chunk)
+
+    go.attention_rows = short
+    try:
+        return _REAL_DECODE(layer, x, K_cache, V_cache, lengths, *W)
+    finally:
+        go.attention_rows = real_rows
+
+
+def _decode_writing_one_row_late(layer, x, K_cache, V_cache, lengths, *W):
+    """The new token's K/V written at position L + 1 (attended there)."""
+    lengths = np.asarray(lengths)
+    K2, V2 = K_cache.copy(), V_cache.copy()
+    r = _REAL_DECODE(layer, x, K2, V2, lengths, *W)
+    for b, L in enumerate(lengths):
+        r.K_cache[:, b, L + 1] = r.K_cache[:, b, L]
+        r.K_cache[:, b, L] = K_cache[:, b, L]
+    return r
+
+
+_REAL_DECODE = go.decode
+
+
+@pytest.mark.parametrize("mistake", [_decode_attending_one_key_short,
+                                     _decode_writing_one_row_late])
+def test_planted_decode_mistake_is_caught(mistake, monkeypatch):
+    monkeypatch.setattr(go, "decode", mistake)
+    with pytest.raises(AssertionError):
+        test_decode_equals_prefill_row(1, "gqe", True)
