@@ -466,6 +466,26 @@ def attention_rows_backward(q: np.ndarray, t_pos: np.ndarray, K: np.ndarray, V: 
     return (dS @ K) * scale, (dS.T @ q) * scale, dV
 
 
+def slot_weights_backward(dw: np.ndarray, w: np.ndarray, p_sel: np.ndarray) -> np.ndarray:
+    """Gradient reaching the selected p through the slot weights w = p_sel / P_t (P_t the
+    token's sum of selected p; numerator and denominator both differentiated):
+    dp_sel = (dw - sum(dw * w)) / P_t, per token."""
+    P_t = p_sel.sum(axis=(1, 2), keepdims=True)
+    return (dw - (dw * w).sum(axis=(1, 2), keepdims=True)) / P_t
+
+
+def aux_loss_grad_p(counts: np.ndarray, M: int, G: int, k: int) -> np.ndarray:
+    """dL / dp[t, g, j] = (1/G) E f[g, j] / M (the counts, hence f, are constant); [G, E]."""
+    E = counts.shape[0] // G
+    f = counts.reshape(G, E).astype(np.float64) / (M * k)
+    return (E / G) * f / M
+
+
+def group_softmax_backward(p: np.ndarray, dp: np.ndarray) -> np.ndarray:
+    """Logit gradient of the per-group softmax: dl = p * (dp - sum_j p dp); [M, G, E]."""
+    return p * (dp - (p * dp).sum(axis=2, keepdims=True))
+
+
 def backward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_shared, W_o,
              dy: np.ndarray, dA: float = 0.0) -> Grads:
     """Gradients of <dy, y> + dA * L (y, L: the forward's output and aux loss) with respect to
@@ -501,9 +521,7 @@ def backward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_
                 s = g * k + r
                 dO[s] += rt.w[:, g, r][:, None] * dslot
                 dw[:, g, r] = (dslot * fw.O[s]).sum(axis=1)
-        # w = p_sel / P_t with P_t the token's sum of selected p: both are differentiated
-        P_t = rt.p_sel.sum(axis=(1, 2))
-        dp_sel += (dw - (dw * rt.w).sum(axis=(1, 2), keepdims=True)) / P_t[:, None, None]
+        dp_sel += slot_weights_backward(dw, rt.w, rt.p_sel)
     if layer.shared:
         dO[G * k] += dZ[:, col:col + d_h]
     # router: p of the selected experts, the aux loss's mean p, the per-group softmax
@@ -513,10 +531,8 @@ def backward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_
         for r in range(k):
             dp[mi, g, rt.sel[:, g, r]] += dp_sel[:, g, r]
     if dA:
-        f = rt.counts.reshape(G, E).astype(np.float64) / (M * k)
-        dp += dA * (E / G) * f[None] / M  # dL / dp[t, g, j] = (1/G) E f[g, j] / M
-    dl = rt.p * (dp - (rt.p * dp).sum(axis=2, keepdims=True))
-    dl = dl.reshape(M, N)
+        dp += dA * aux_loss_grad_p(rt.counts, M, G, k)[None]
+    dl = group_softmax_backward(rt.p, dp).reshape(M, N)
     dW_r = dl.T @ x
     dx = dl @ W_r
     # attention, per stream and sequence; K / V gradients add up over the streams of a head

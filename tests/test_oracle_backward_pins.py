@@ -5,8 +5,9 @@ share none of them: torch's float64 autograd through a forward written here with
 operations (the selected sets held constant, as the definition states), and central finite
 differences of the oracle's forward pass (itself pinned in test_oracle_pins.py). Two facts
 fixed by the definition are checked exactly: hard_concat gives the router no gradient from y,
-and without any routed output the aux-loss gradient has a closed form. A planted mistake in
-the attention backward must be caught.
+and without any routed output the aux-loss gradient has a closed form. Planted mistakes in
+the attention backward and in the router's derivatives (a detached slot denominator, a
+dropped aux term, a softmax Jacobian without its off-diagonal part) must be caught.
 """
 import math
 
@@ -187,3 +188,29 @@ def test_planted_mistake_in_attention_backward_is_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_backward_matches_torch_autograd(0)
     monkeypatch.setattr(go, "attention_rows_backward", real)
+
+
+def _slot_denominator_detached(dw, w, p_sel):
+    return dw / p_sel.sum(axis=(1, 2), keepdims=True)
+
+
+def _aux_gradient_dropped(counts, M, G, k):
+    return np.zeros((G, counts.shape[0] // G))
+
+
+def _softmax_jacobian_diagonal_only(p, dp):
+    return p * dp
+
+
+@pytest.mark.parametrize("name,mistake", [
+    ("slot_weights_backward", _slot_denominator_detached),
+    ("aux_loss_grad_p", _aux_gradient_dropped),
+    ("group_softmax_backward", _softmax_jacobian_diagonal_only),
+])
+def test_planted_router_backward_mistake_is_caught(name, mistake, monkeypatch):
+    """Plausible mistakes in the router's derivatives (a detached slot denominator, a
+    forgotten aux term, the softmax Jacobian without its off-diagonal part) break the autograd
+    pin of the gqe variant with the aux loss."""
+    monkeypatch.setattr(go, name, mistake)
+    with pytest.raises(AssertionError):
+        test_backward_matches_torch_autograd(0)
