@@ -67,3 +67,27 @@ def test_active_flops_formula():
     assert wl.active_flops() == pytest.approx(want)
     assert wl.active_flops() / 1e9 == pytest.approx(274.6, abs=0.5)
     assert wl.all_active().n_streams == 17
+
+
+def test_decode_inputs_are_deterministic_exact_and_margined():
+    wl = W.WORKLOADS["main_b8_t2048"]
+    a = W.generate_decode(wl, [0, 17, 255], 256)
+    b = W.generate_decode(wl, [0, 17, 255], 256)
+    assert np.array_equal(a.k_cache, b.k_cache) and np.array_equal(a.inp.x, b.inp.x)
+    assert a.k_cache.shape == a.v_cache.shape == (wl.G, 3, 256, wl.d_h)
+    assert a.lengths.dtype == np.int32 and a.lengths.tolist() == [0, 17, 255]
+    # values exact in bf16; the raw bits round-trip
+    for name in ("k_cache", "v_cache"):
+        c = getattr(a, name)
+        assert np.array_equal(W.bf16_bits_to_f32(a.raw_cache(name)), c)
+    # the new tokens pass the margin filter; the cache spread is that of a projected K/V
+    assert W._topk_gaps(a.inp.x, a.inp.W_r, wl.G, wl.k).min() >= wl.margin
+    assert abs(a.k_cache.std() / (wl.w_std * wl.dim ** 0.5) - 1) < 0.02
+    # the new tokens and weights are those of generate() with B = 3, T = 1
+    g = W.generate(wl.with_(B=3, T=1))
+    assert np.array_equal(g.x, a.inp.x) and np.array_equal(g.W_o, a.inp.W_o)
+
+
+def test_decode_inputs_reject_positions_outside_the_cache():
+    with pytest.raises(ValueError):
+        W.generate_decode(W.WORKLOADS["main_b8_t2048"], [0, 8], 8)
