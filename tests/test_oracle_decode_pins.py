@@ -3,8 +3,10 @@
 The decode step is defined as row L_b of the prefill forward over the sequence whose first
 L_b tokens filled the cache. The pins check it against the prefill oracle (itself pinned in
 test_oracle_pins.py), against the closed form of attention over a single key (an empty
-cache: O = V of the new token), and against two invariances: cache rows at or beyond the
-new position do not matter, and the sequences of a batch do not interact.
+cache: O = V of the new token), against an independently written all-active GQA decode step
+(k = E, hard_concat, no shared head), and against two invariances: cache rows at or beyond
+the new position do not matter, and the sequences of a batch do not interact. Planted
+mistakes must be caught.
 """
 import math
 
@@ -167,3 +169,33 @@ def test_planted_decode_mistake_is_caught(mistake, monkeypatch):
     monkeypatch.setattr(go, "decode", mistake)
     with pytest.raises(AssertionError):
         test_decode_equals_prefill_row(1, "gqe", True)
+
+
+def dense_gqa_decode(x, K_cache, V_cache, lengths, W_q, W_k, W_v, W_o, N, G, d_h):
+    """An all-active GQA decode step written independently: every query head h of every new
+    token attends over its sequence's cached keys of head h // (N / G) plus the new key."""
+    B = x.shape[0]
+    E = N // G
+    out_heads = np.zeros((B, N * d_h))
+    for b in range(B):
+        L = int(lengths[b])
+        for h in range(N):
+            g = h // E
+            q = W_q[h * d_h:(h + 1) * d_h] @ x[b]
+            keys = np.vstack([K_cache[g, b, :L], W_k[g * d_h:(g + 1) * d_h] @ x[b]])
+            vals = np.vstack([V_cache[g, b, :L], W_v[g * d_h:(g + 1) * d_h] @ x[b]])
+            sc = keys @ q / math.sqrt(d_h)
+            wts = np.exp(sc - sc.max())
+            out_heads[b, h * d_h:(h + 1) * d_h] = (wts / wts.sum()) @ vals
+    return out_heads @ W_o.T
+
+
+@pytest.mark.parametrize("N,G", [(8, 4), (6, 2), (4, 4)])
+def test_all_active_decode_equals_dense_gqa_decode(N, G):
+    layer = go.Layer(dim=16, N=N, G=G, k=N // G, d_h=4, shared=False, variant="hard_concat")
+    rng = np.random.default_rng(60 + N + G)
+    lengths = [0, 3, 9]
+    W, _, x, Kc, Vc = build(layer, rng, lengths, L_max=12)
+    dec = go.decode(layer, x, Kc, Vc, lengths, *W)
+    want = dense_gqa_decode(x, Kc, Vc, lengths, W[1], W[2], W[3], W[5], N, G, layer.d_h)
+    np.testing.assert_allclose(dec.y, want, rtol=1e-10, atol=1e-12)
