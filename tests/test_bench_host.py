@@ -7,11 +7,13 @@ import os
 import bench
 
 
-def test_traffic_record_matches_current_sources():
+def test_traffic_reported_only_for_the_profiled_sources():
     rec = json.load(open(os.path.join(bench.ROOT, "profiles", "attn_traffic.json")))
-    assert rec["sources_sha256"] == bench.attention_source_sha()
-    assert bench.attention_traffic(rec["workload"]) == (
-        rec["dram_read_bytes"] + rec["dram_write_bytes"])
+    got = bench.attention_traffic(rec["workload"])
+    if rec["sources_sha256"] == bench.attention_source_sha():
+        assert got == rec["dram_read_bytes"] + rec["dram_write_bytes"]
+    else:  # the kernel changed since the capture: no traffic figure
+        assert got is None
 
 
 def test_traffic_withheld_for_other_workloads_and_changed_sources(monkeypatch):
