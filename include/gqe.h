@@ -70,8 +70,8 @@ typedef enum {
  *   G           GQA groups = dense KV heads ("num_kv_heads").
  *   k           experts kept per group per token ("top_k"), 1 <= k <= min(N/G, 8).
  *   d_h         head dimension ("head_dim"; its default dim/N is applied by the Python
- *               binding, not here). bf16: d_h in {16, 32, 48, 64, 80, 96, 112, 128};
- *               fp32: d_h % 4 == 0 and d_h <= 128.
+ *               binding, not here). d_h in {16, 32, 48, 64, 80, 96, 112, 128} for
+ *               both dtypes (GQE_ERR_UNSUPPORTED otherwise).
  *   dtype       GQE_BF16 (bf16 storage, fp32 accumulation) or GQE_F32.
  *   max_tokens  the largest B*T any gqe_forward on this handle will use.
  *
@@ -205,7 +205,7 @@ const char* gqe_stage_name(int i);
  *   mean_prob  [N] float              mean over tokens of the per-group softmax p.
  *   aux_loss   device float* or NULL  the Switch load-balancing loss (as gqe_forward).
  *
- * Scratch lives in one file-scope device array of 2.5 MiB (+256 B), held by every GPU that
+ * Scratch lives in one file-scope device array of 2.5 MiB (+512 B), held by every GPU that
  * loads the library until the process exits. Limits: M <= 131072 and M*G*k <= 262144;
  * larger calls return GQE_ERR_WORKSPACE and launch nothing. N <= 64, k <= 8
  * (GQE_ERR_UNSUPPORTED otherwise). The first call on each device looks up the array's

@@ -301,13 +301,7 @@ __global__ void __launch_bounds__(THREADS) decode_merge_kernel(const DecParams P
 template <int DH, int QPW>
 int launch_attn(const DecParams& P, cudaStream_t st) {
   using C = DecCfg<DH>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(decode_attn_kernel<DH, QPW>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once<decode_attn_kernel<DH, QPW>>(C::SMEM)) return -1;
   return launch_pdl(decode_attn_kernel<DH, QPW>, dim3(P.nc, P.G, P.B), dim3(THREADS), C::SMEM,
                     st, P) == cudaSuccess
              ? 1

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/gqe.h"
 
 namespace gqe {
@@ -49,6 +51,27 @@ inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// The dynamic shared-memory limit of a kernel is a per-device attribute: set it on the
+// current device the first time that device launches the kernel (one flag per kernel and
+// device, under a lock, so concurrent callers and handles on several devices are safe).
+template <auto Kernel>
+inline bool set_smem_limit_once(int smem) {
+  static std::mutex mu;
+  static uint64_t done = 0;  // bit d: set on device d (ordinals 0..63)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev < 0 || dev >= 64)
+    return cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+           cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((done >> dev) & 1u) return true;
+  if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return false;
+  done |= uint64_t(1) << dev;
+  return true;
 }
 
 // ---------------------------------------------------------------------------------------

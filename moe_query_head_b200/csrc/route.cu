@@ -522,14 +522,9 @@ route_fused_kernel(const float* __restrict__ logits, int M, int N, int G, int k,
 
 int launch_route_fused(gqe_ctx* h, int M, float* aux_out, cudaStream_t st) {
   const int smem = fused_smem_bytes(h->N, h->G);
-  static bool configured = false;
-  if (!configured) {
-    // the largest size any shape can ask for, so that one setting serves every handle
-    if (cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fused_smem_bytes(kMaxExperts, kMaxExperts)) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  // the largest size any shape can ask for, so that one setting serves every handle
+  if (!set_smem_limit_once<route_fused_kernel>(fused_smem_bytes(kMaxExperts, kMaxExperts)))
+    return -1;
   const int nblk = (M + kRouteBlock - 1) / kRouteBlock;
   const int grid = nblk < 4 * h->num_sms ? nblk : 4 * h->num_sms;
   const float* logits = h->ws.logits;

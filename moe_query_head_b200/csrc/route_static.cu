@@ -32,7 +32,11 @@ constexpr size_t kOffW = kOffPsel + sizeof(float) * kStaticMaxEntries;
 constexpr size_t kOffPartCounts = kOffW + sizeof(float) * kStaticMaxEntries;
 constexpr size_t kOffPartProb = kOffPartCounts + sizeof(int32_t) * kStaticMaxBlocks * kMaxExperts;
 constexpr size_t kOffOffsets = kOffPartProb + sizeof(float) * kStaticMaxBlocks * kMaxExperts;
-constexpr size_t kScratchBytes = kOffOffsets + 256;  // offsets: N + 1 <= 65 int32
+// offsets: N + 1 <= kMaxExperts + 1 int32, rounded up to the array's 256-byte alignment
+constexpr size_t kOffsetsBytes = (sizeof(int32_t) * (kMaxExperts + 1) + 255) / 256 * 256;
+constexpr size_t kScratchBytes = kOffOffsets + kOffsetsBytes;
+static_assert(kScratchBytes >= kOffOffsets + sizeof(int32_t) * (kMaxExperts + 1),
+              "the scratch must hold offsets[0 .. kMaxExperts]");
 
 // The scratch. In host code this name is only a host-side stand-in for the symbol, not a
 // device address: the device address comes from cudaGetSymbolAddress below.

@@ -58,7 +58,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int DH>
 struct Cfg {
-  static constexpr int CW = (DH % 64 == 0) ? 64 : (DH % 32 == 0) ? 32 : 16;  // chunk width
+  // Chunk width (columns per swizzle atom). Head dims with tensor-core row sums (<= 48)
+  // use 16-column chunks, so the 16 columns of ones after a V tile are exactly one chunk and
+  // the P V operand of N = d_h + 16 columns is a whole number of chunks.
+  static constexpr int CW = (DH % 64 == 0) ? 64 : (DH % 32 == 0 && DH > 48) ? 32 : 16;
   static constexpr int NC = DH / CW;                                         // chunks
   static constexpr uint32_t LAYOUT =
       CW == 64 ? kSwizzle128B : (CW == 32 ? kSwizzle64B : kSwizzle32B);
@@ -85,6 +88,8 @@ struct Cfg {
   static constexpr int P_COL = 128;
   static constexpr int O_COL = 192;
   static_assert(O_COL + N_PV <= TMEM_COLS, "TMEM budget");
+  static_assert(!SUM_MMA || CW == 16, "the ones chunk must be one 16-column chunk");
+  static_assert(N_PV % CW == 0, "P V reads whole chunks");
   static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory budget");
 };
 // Exponentials: of every 8 pairs of scores, this many go to the FMA-pipe polynomial and
@@ -672,13 +677,7 @@ template <int DH>
 int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int causal,
               int Do, cudaStream_t st) {
   using C = Cfg<DH>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(attn_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once<attn_kernel<DH>>(C::SMEM)) return -1;
   const int M = B * T;
   Params P;
   memset(&P, 0, sizeof(P));

@@ -788,13 +788,7 @@ bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
 template <bool GATHER, bool ROUTE = false, bool NARROW = false>
 int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
   constexpr int smem = Ring<NARROW>::SMEM;
-  static bool configured = false;  // one per instance
-  if (!configured) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<GATHER, ROUTE, NARROW>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  if (!set_smem_limit_once<tc_gemm_kernel<GATHER, ROUTE, NARROW>>(smem)) return -1;
   return launch_pdl(tc_gemm_kernel<GATHER, ROUTE, NARROW>, dim3(grid),
                     dim3(Lay<GATHER>::THREADS), smem, st, P) == cudaSuccess
              ? 1

@@ -255,6 +255,26 @@ def generate(wl: Workload) -> Inputs:
     return Inputs(wl, x, W_r, W_q, W_k, W_v, W_s if wl.shared else None, W_o, report)
 
 
+def router_logits_input(M: int, N: int, G: int, k: int, seed: int,
+                        margin: float = 1e-3) -> np.ndarray:
+    """Router logits [M, N] as float32, N(0, 1) from PCG64([seed, 3]), for the entry point
+    that routes precomputed logits. Rows whose gap between the k-th and (k+1)-th largest
+    logit of some group is below `margin` are redrawn, as the margin filter above does for
+    x, so that the top-k decision is the same in any precision."""
+    rng = np.random.Generator(np.random.PCG64([seed, 3]))
+    lg = rng.standard_normal((M, N)).astype(np.float32)
+    E = N // G
+    if k >= E:
+        return lg
+    for _ in range(100):
+        s = -np.sort(-lg.astype(np.float64).reshape(M, G, E), axis=2)
+        bad = np.nonzero((s[:, :, k - 1] - s[:, :, k]).min(axis=1) < margin)[0]
+        if bad.size == 0:
+            return lg
+        lg[bad] = rng.standard_normal((bad.size, N)).astype(np.float32)
+    raise RuntimeError("margin filter did not converge")
+
+
 @dataclass
 class DecodeInputs:
     """One decode step's inputs: `inp` holds the B new tokens (x [B, dim], one per

@@ -6,9 +6,9 @@ rounding) and every other cache row left bit-identical.
 
 Cases cover both ways the attention runs (one CTA per sequence and group writing Z
 directly when there are at least four such pairs per SM, and split key chunks merged by a
-second kernel), ragged positions (0, tile edges, long), the three variants, head dims
-48 / 64 / 128, a layer without the shared head, and the consistency of a decode step with
-the GPU prefill row at the same position."""
+second kernel), ragged positions (0, tile edges, long), the three variants, every head dim the ABI accepts,
+one to three queries per warp (k up to 8), a layer without the shared head, and the
+consistency of a decode step with the GPU prefill row at the same position."""
 import numpy as np
 import pytest
 import torch
@@ -124,7 +124,17 @@ CASES = {
     "wide_weighted": (WIDE.with_(variant="weighted_concat"), [1, 64, 300], 320),
     "wide_hard": (WIDE.with_(variant="hard_concat"), [130, 0, 257], 320),
     "large_d128": (LARGE, [100, 1000], 1024),
+    # two and three queries per warp: k = 4 of 4 (five queries in group 0) and k = 8 of 8
+    # with 64 experts (nine queries in group 0)
+    "wide_k4_qpw2": (WIDE.with_(k=4), [3, 200, 511], 512),
+    "n64_k8_qpw3": (MAIN.with_(N=64, G=8, k=8), [0, 65, 300], 320),
+    # one CTA per (sequence, group) at d_h = 80
+    "dh80_direct_batch80": (MAIN.with_(d_h=80),
+                            list(np.random.default_rng(6).integers(0, 200, 80)), 256),
 }
+# every head dim the ABI accepts, split key chunks with ragged positions
+for _dh in (16, 32, 80, 96, 112):
+    CASES[f"dh{_dh}_split"] = (MAIN.with_(d_h=_dh), [0, 100, 600], 640)
 
 
 @pytest.mark.parametrize("case", list(CASES))

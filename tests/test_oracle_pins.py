@@ -279,6 +279,42 @@ def test_gqe_slot_uniform_router_is_mean():
     np.testing.assert_allclose(res.y, res.Z @ W_o.T, atol=1e-14)
 
 
+def test_gqe_slot_hand_computed_non_uniform_router():
+    """The gqe slot with a non-uniform router, against values worked out by hand.
+
+    G = 2 groups of E = 2 experts, k = 1, d_h = 2, no shared head; two sequences of one
+    token each, so every stream's attention output is its head's single value row
+    (O = V_0). Token 0 = e_0 has group logits (ln 3, 0) and (ln 2, 0): it takes expert 0
+    in both groups with p = 3/4 and 2/3. Token 1 = e_1 has (0, ln 4) and (0, ln 1.5): it
+    takes expert 1 in both with p = 4/5 and 3/5. The value heads are V_0 = (1, 0) and
+    V_1 = (0, 1) for both tokens. The slot renormalises the selected p over all G k
+    selections of the token (gist.science summary, Output Construction: a weighted sum of
+    the selected expert outputs using router probabilities), so token 0's slot is
+    (3/4, 2/3) / (3/4 + 2/3) = (9/17, 8/17) and token 1's is (4/5, 3/5) / (7/5) =
+    (4/7, 3/7). Per-group gates (1 each at k = 1) or gates / G (1/2 each) give other
+    values."""
+    layer = go.Layer(dim=4, N=4, G=2, k=1, d_h=2, shared=False, variant="gqe")
+    x = np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0]])
+    W_r = np.zeros((4, 4))
+    W_r[:, 0] = [math.log(3.0), 0.0, math.log(2.0), 0.0]
+    W_r[:, 1] = [0.0, math.log(4.0), 0.0, math.log(1.5)]
+    W_v = np.zeros((4, 4))
+    W_v[0, :2] = 1.0  # head 0, column 0
+    W_v[3, :2] = 1.0  # head 1, column 1
+    rng = np.random.default_rng(11)
+    W_q = rng.standard_normal((8, 4))
+    W_k = rng.standard_normal((4, 4))
+    W_o = rng.standard_normal((4, layer.D_o))
+    res = go.forward(layer, x, 2, 1, W_r, W_q, W_k, W_v, None, W_o)
+    assert res.routing.sel[:, :, 0].tolist() == [[0, 0], [1, 1]]
+    np.testing.assert_allclose(res.routing.p_sel[:, :, 0], [[0.75, 2 / 3], [0.8, 0.6]],
+                               atol=1e-15)
+    slot = res.Z[:, 4:6]
+    np.testing.assert_allclose(slot, [[9 / 17, 8 / 17], [4 / 7, 3 / 7]], atol=1e-15)
+    # the hard-concat blocks are the heads' value rows
+    np.testing.assert_allclose(res.Z[:, 0:4], [[1, 0, 0, 1], [1, 0, 0, 1]], atol=1e-15)
+
+
 # ---------------------------------------------------------------------------------------
 # Load-balancing loss
 # ---------------------------------------------------------------------------------------
@@ -355,6 +391,14 @@ def _route_slot_per_group(x, W_r, G, k):
 _orig_route = go.route
 
 
+def _route_slot_gates_over_G(x, W_r, G, k):
+    # sums to 1 per token like the true slot weights, but ignores how the groups' selected
+    # probabilities compare
+    rt = _orig_route(x, W_r, G, k)
+    rt.w = rt.gates / G
+    return rt
+
+
 def _kv_transposed(x, W_k, W_v, G, d_h):
     K, V = _orig_kv(x, W_k, W_v, G, d_h)
     return V, K
@@ -383,7 +427,10 @@ MUTANTS = {
                                   [lambda: test_attention_closed_forms(),
                                    lambda: test_all_active_equals_dense_gqa(4, 2, True)]),
     "slot_per_group": ("route", _route_slot_per_group,
-                       [lambda: test_routing_invariants(1)]),
+                       [lambda: test_routing_invariants(1),
+                        lambda: test_gqe_slot_hand_computed_non_uniform_router()]),
+    "slot_gates_over_G": ("route", _route_slot_gates_over_G,
+                          [lambda: test_gqe_slot_hand_computed_non_uniform_router()]),
     "kv_swapped": ("kv_projection", _kv_transposed,
                    [lambda: test_all_active_equals_dense_gqa(4, 2, True)]),
     "shared_head_kv": ("stream_kv_head", _shared_reads_last_head,

@@ -69,7 +69,21 @@ SMALL = {
     "experts_3_per_group": dict(base="main_b8_t2048", B=1, T=200, N=12, G=4, k=1),
     "one_group_of_32": dict(base="main_b8_t2048", B=1, T=200, N=32, G=1, k=2),
     "one_expert_per_group": dict(base="main_b8_t2048", B=1, T=200, N=8, G=8, k=1),
+    # the largest routing shapes the ABI accepts: 64 experts, top-8 of 8 (every expert
+    # active), top-3 of 8, and one group of 64 with top-2
+    "n64_g8_k8": dict(base="main_b8_t2048", B=1, T=200, N=64, G=8, k=8),
+    "n64_g8_k3": dict(base="main_b8_t2048", B=1, T=230, N=64, G=8, k=3),
+    "n64_g1_k2": dict(base="main_b8_t2048", B=1, T=200, N=64, G=1, k=2),
+    # fp32 handles at other head dims
+    "f32_dh48_noncausal": dict(base="tiny_f32", B=2, T=150, d_h=48, causal=False),
+    "f32_dh128": dict(base="tiny_f32", B=1, T=200, d_h=128),
 }
+# every bf16 head dim the ABI accepts, causal over three query tiles with a ragged tail
+# and non-causal over two
+for _dh in (16, 32, 48, 64, 80, 96, 112, 128):
+    SMALL[f"dh{_dh}_causal"] = dict(base="main_b8_t2048", B=2, T=300, d_h=_dh)
+    SMALL[f"dh{_dh}_noncausal"] = dict(base="main_b8_t2048", B=1, T=200, d_h=_dh,
+                                       causal=False)
 
 
 @pytest.mark.parametrize("case", sorted(SMALL))
