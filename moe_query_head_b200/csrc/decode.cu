@@ -13,11 +13,13 @@
 // The work is HBM-bound (every cached K/V row is read once, shared by all query streams of
 // its group), so it runs on CUDA cores. CTA (chunk c, group g, sequence b) streams its key
 // range in tiles of 64 rows through a cp.async ring in shared memory (rows padded by 16
-// bytes so the per-key 16-byte reads are conflict-free); warp w owns queries w, w+4, w+8 of
-// the group: scores with one key per lane (two per tile), the online softmax with warp
-// shuffles, P V with each lane owning pairs of head dimensions. With one chunk per sequence
-// and group the CTA writes Z directly; otherwise it writes (m, l, O) to a partial slot and
-// decode_merge_kernel combines the chunks.
+// bytes). Each of the four warps takes 16 keys of every tile for all of the group's queries,
+// so the work is spread evenly however few queries a group has (two at k = 1 in group 0,
+// one elsewhere): a score per (key, half of the head dims) lane pair, the online softmax
+// over the warp's keys with shuffles, P V with each lane owning pairs of head dimensions.
+// After the last tile the four warps' (m, l, O) are merged in shared memory. With one chunk
+// per sequence and group the CTA writes Z directly; otherwise it writes (m, l, O) to a
+// partial slot and decode_merge_kernel combines the chunks.
 #include <string.h>
 
 #include "gqe_common.cuh"
@@ -33,6 +35,7 @@ constexpr int WARPS = THREADS / 32;
 constexpr int TKD = 64;      // keys per tile
 constexpr int STAGES = 3;    // tiles in flight
 constexpr int MAXQ = kMaxTopK + 1;
+constexpr int KPW = TKD / WARPS;  // keys of a tile per warp
 
 struct DecParams {
   const __nv_bfloat16* Knew;  // [G, B, d_h] the new tokens' keys (workspace)
@@ -66,6 +69,8 @@ struct DecCfg {
   static constexpr int CHUNKS = DH / 8;           // 16-byte pieces per row
   static constexpr int NP = (DH / 2 + 31) / 32;   // dim pairs per lane
   static constexpr int SMEM = STAGES * 2 * TILE + MAXQ * DH * 4;
+  static_assert(STAGES * 2 * TILE >= WARPS * MAXQ * (DH + 2) * 4,
+                "the ring holds the warps' states for the merge");
 };
 
 // stream index of query i of group g (routed streams first, then the shared one)
@@ -73,9 +78,9 @@ __device__ __forceinline__ int stream_of(const DecParams& P, int g, int i) {
   return i < P.k ? g * P.k + i : P.Sr;
 }
 
-// QPW: queries per warp (1 for up to four queries per group, i.e. k <= 3 with the shared
-// head; up to 3 for k = 8), a compile-time count so the per-query state stays in registers.
-template <int DH, int QPW>
+// QMAX: the most queries a group can have at this launch (k, plus the shared head in group
+// 0): 2, 4 or 9, a compile-time count so the per-query state stays in registers.
+template <int DH, int QMAX>
 __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P) {
   using C = DecCfg<DH>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -142,10 +147,16 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
     if (t < ntiles) load_tile(t, t);
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  float m[QPW], l[QPW];
-  float2 o[QPW][C::NP];
+  // Every warp takes a quarter of each tile (keys 16 w .. 16 w + 15) for every query, with
+  // its own online-softmax state; the four states are merged after the last tile. Score:
+  // lane = key (lane & 15) x half of the head dims (lane >> 4), halves summed by a shuffle.
+  // P V: lanes own dimension pairs and loop over the warp's 16 keys.
+  const int kq = lane & 15, half = lane >> 4;
+  const int krow = warp * KPW + kq;
+  float m[QMAX], l[QMAX];
+  float2 o[QMAX][C::NP];
 #pragma unroll
-  for (int a = 0; a < QPW; ++a) {
+  for (int a = 0; a < QMAX; ++a) {
     m[a] = -INFINITY;
     l[a] = 0.f;
 #pragma unroll
@@ -160,41 +171,43 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
     const int st = t % STAGES;
     const uint8_t* kt = sK + st * C::TILE;
     const uint8_t* vt = sV + st * C::TILE;
-    const int base = k0 + t * TKD;
+    const bool key_ok = k0 + t * TKD + krow < k1;
+    // this lane's half of its key's row, as floats
+    float kf[DH / 2];
+    {
+      const uint8_t* row = kt + krow * C::ROWB + half * DH;
 #pragma unroll
-    for (int a = 0; a < QPW; ++a) {
-      const int i = warp + a * WARPS;
-      if (i >= nq) break;  // warp-uniform
-      const float* q = sQ + i * DH;
-      // scores of keys lane and lane + 32
-      float sc[2];
+      for (int ch = 0; ch < DH / 16; ++ch) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + ch * 16);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = lane + 32 * h;
-        const uint8_t* row = kt + r * C::ROWB;
-        float acc = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < C::CHUNKS; ++ch) {
-          const uint4 v = *reinterpret_cast<const uint4*>(row + ch * 16);
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(p2[e]);
-            acc = fmaf(q[ch * 8 + 2 * e], f.x, acc);
-            acc = fmaf(q[ch * 8 + 2 * e + 1], f.y, acc);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(p2[e]);
+          kf[ch * 8 + 2 * e] = f.x;
+          kf[ch * 8 + 2 * e + 1] = f.y;
         }
-        sc[h] = base + r < k1 ? acc : -INFINITY;
       }
-      float mt = fmaxf(sc[0], sc[1]);
+    }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float m_new = fmaxf(m[a], mt);  // finite: every tile holds at least one key
-      const float alpha = ex2(m[a] - m_new);  // 0 when m was -inf
-      const float p0 = ex2(sc[0] - m_new), p1 = ex2(sc[1] - m_new);
-      float ps = p0 + p1;
+    for (int a = 0; a < QMAX; ++a) {
+      if (a >= nq) break;  // uniform over the CTA
+      const float* q = sQ + a * DH + half * (DH / 2);
+      float acc = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      for (int d = 0; d < DH / 2; ++d) acc = fmaf(q[d], kf[d], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+      const float sc = key_ok ? acc : -INFINITY;
+      float mt = sc;
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_new = fmaxf(m[a], mt);
+      // a warp whose keys are all masked so far keeps m = -inf, l = 0, O = 0
+      const float m_ref = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2(m[a] - m_ref);  // 0 while m is -inf
+      const float pk = ex2(sc - m_ref);       // 0 for a masked key
+      float ps = pk;
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l[a] = l[a] * alpha + ps;
       m[a] = m_new;
 #pragma unroll
@@ -202,11 +215,10 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
         o[a][p].x *= alpha;
         o[a][p].y *= alpha;
       }
-      // O += P V: lane owns dimension pairs lane, lane + 32, ...
-#pragma unroll 4
-      for (int j = 0; j < TKD; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
-        const uint8_t* row = vt + j * C::ROWB;
+#pragma unroll
+      for (int j = 0; j < KPW; ++j) {
+        const float pj = __shfl_sync(0xffffffffu, pk, j);
+        const uint8_t* row = vt + (warp * KPW + j) * C::ROWB;
 #pragma unroll
         for (int p = 0; p < C::NP; ++p) {
           const int d2 = lane + 32 * p;
@@ -222,14 +234,45 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
     __syncthreads();  // every warp is done with stage st before it is refilled
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
-  // results
+  __syncthreads();  // the ring is free: it holds the warps' states for the merge
+  // merge the four warps' (m, l, O) of every query: state of (warp, query) at
+  // sM[(warp * MAXQ + query) * (DH + 2)]: m, l, then O
+  float* sM = reinterpret_cast<float*>(smem);
 #pragma unroll
-  for (int a = 0; a < QPW; ++a) {
-    const int i = warp + a * WARPS;
-    if (i >= nq) break;
+  for (int a = 0; a < QMAX; ++a) {
+    if (a >= nq) break;
+    float* st = sM + (warp * MAXQ + a) * (DH + 2);
+    if (lane == 0) {
+      st[0] = m[a];
+      st[1] = l[a];
+    }
+#pragma unroll
+    for (int p = 0; p < C::NP; ++p) {
+      const int d2 = lane + 32 * p;
+      if (2 * d2 < DH) {
+        st[2 + 2 * d2] = o[a][p].x;
+        st[2 + 2 * d2 + 1] = o[a][p].y;
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nq * DH; e += THREADS) {
+    const int i = e / DH, d = e % DH;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) mx = fmaxf(mx, sM[(w * MAXQ + i) * (DH + 2)]);
+    const float mref = mx == -INFINITY ? 0.f : mx;
+    float lt = 0.f, ot = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const float* st = sM + (w * MAXQ + i) * (DH + 2);
+      const float f = ex2(st[0] - mref);  // 0 for a warp that saw no key
+      lt += f * st[1];
+      ot += f * st[2 + d];
+    }
     const int s = stream_of(P, g, i);
     if (P.nc == 1) {
-      float scale = 1.f / l[a];
+      float scale = 1.f / lt;
       int col;
       if (s < P.Sr) {
         col = s * DH;
@@ -237,28 +280,14 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
       } else {
         col = P.shared_col;
       }
-      __nv_bfloat16* dst = P.Z + (size_t)b * P.Do + col;
-#pragma unroll
-      for (int p = 0; p < C::NP; ++p) {
-        const int d2 = lane + 32 * p;
-        if (2 * d2 < DH)
-          *reinterpret_cast<__nv_bfloat162*>(dst + 2 * d2) =
-              __floats2bfloat162_rn(o[a][p].x * scale, o[a][p].y * scale);
-      }
+      P.Z[(size_t)b * P.Do + col + d] = __float2bfloat16_rn(ot * scale);
     } else {
       float* slot = P.part + ((((size_t)b * P.G + g) * P.nc + c) * (P.k + 1) + i) * (DH + 2);
-      if (lane == 0) {
-        slot[0] = ntiles ? m[a] : -INFINITY;
-        slot[1] = l[a];
+      if (d == 0) {
+        slot[0] = ntiles ? mx : -INFINITY;
+        slot[1] = lt;
       }
-#pragma unroll
-      for (int p = 0; p < C::NP; ++p) {
-        const int d2 = lane + 32 * p;
-        if (2 * d2 < DH) {
-          slot[2 + 2 * d2] = o[a][p].x;
-          slot[2 + 2 * d2 + 1] = o[a][p].y;
-        }
-      }
+      slot[2 + d] = ot;
     }
   }
 }
@@ -298,11 +327,11 @@ __global__ void __launch_bounds__(THREADS) decode_merge_kernel(const DecParams P
   }
 }
 
-template <int DH, int QPW>
+template <int DH, int QMAX>
 int launch_attn(const DecParams& P, cudaStream_t st) {
   using C = DecCfg<DH>;
-  if (!set_smem_limit_once<decode_attn_kernel<DH, QPW>>(C::SMEM)) return -1;
-  return launch_pdl(decode_attn_kernel<DH, QPW>, dim3(P.nc, P.G, P.B), dim3(THREADS), C::SMEM,
+  if (!set_smem_limit_once<decode_attn_kernel<DH, QMAX>>(C::SMEM)) return -1;
+  return launch_pdl(decode_attn_kernel<DH, QMAX>, dim3(P.nc, P.G, P.B), dim3(THREADS), C::SMEM,
                     st, P) == cudaSuccess
              ? 1
              : -1;
@@ -311,10 +340,9 @@ int launch_attn(const DecParams& P, cudaStream_t st) {
 template <int DH>
 int launch_dh(const DecParams& P, cudaStream_t st) {
   const int nq_max = P.k + (P.has_shared ? 1 : 0);
-  const int qpw = (nq_max + WARPS - 1) / WARPS;
-  const int r = qpw <= 1 ? launch_attn<DH, 1>(P, st)
-                : qpw == 2 ? launch_attn<DH, 2>(P, st)
-                           : launch_attn<DH, 3>(P, st);
+  const int r = nq_max <= 2 ? launch_attn<DH, 2>(P, st)
+                : nq_max <= 4 ? launch_attn<DH, 4>(P, st)
+                              : launch_attn<DH, MAXQ>(P, st);
   if (r < 0) return -1;
   if (P.nc == 1) return 1;
   return launch_pdl(decode_merge_kernel, dim3(P.G, P.B), dim3(THREADS), 0, st, P, DH) ==

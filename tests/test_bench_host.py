@@ -28,3 +28,25 @@ def test_decode_workload_is_the_papers_layer():
     wl = bench.decode_workload(A)
     assert (wl.dim, wl.N, wl.G, wl.k, wl.d_h, wl.M, wl.T) == (768, 16, 8, 1, 48, 64, 1)
     assert wl.shared and wl.variant == "gqe"
+
+
+def test_reference_arm_reports_the_time_it_ran():
+    """--impl reference runs the oracle on a bounded sample each step: ms_per_step is the
+    time those steps took (the whole command takes at least steps x ms_per_step), the value
+    is the extrapolated throughput, and the config dict is the GPU arm's."""
+    import subprocess
+    import sys
+    import time
+    t0 = time.perf_counter()
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl",
+                        "reference", "--workload", "tiny_f32", "--steps", "2", "--warmup", "3",
+                        "--cpu-rows", "64"], capture_output=True, text=True, timeout=300)
+    wall = time.perf_counter() - t0
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 2
+    assert 2 * line["ms_per_step"] / 1e3 <= wall
+    assert line["extrapolated_ms_per_full_step"] >= line["ms_per_step"]
+    wl = bench.W.WORKLOADS["tiny_f32"]
+    assert line["config"] == bench.prefill_config(wl, 1)
+    assert line["cpu_baseline"]["value"] == line["value"]
