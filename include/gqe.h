@@ -147,6 +147,49 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
                       void* stream);
 
 /*
+ * gqe_enable_backward — allocate the handle's backward workspace (cudaMalloc, on the current
+ * device; the gradients of dZ, of the stream outputs and of the query, key and value
+ * projections for max_tokens tokens, and a cuBLAS handle with its 32 MiB workspace). The
+ * handle owns it until gqe_destroy. bf16 handles with d_h <= 64 only (GQE_ERR_UNSUPPORTED
+ * otherwise); GQE_ERR_CUDA if an allocation fails. Calling it again does nothing.
+ */
+gqe_status gqe_enable_backward(gqe_handle h);
+
+/*
+ * gqe_backward — gradients of one GQE attention layer for training (README, Usage: the
+ * task loss plus 0.01 times the aux loss is back-propagated; gist.science summary, Output
+ * Construction: the renormalised slot is the router's differentiable path).
+ *
+ * Returns the gradients of F = <dy, y> + aux_grad * L, where y and L are the output and the
+ * aux loss of the handle's LAST call, which must be a gqe_forward with the same x, weights,
+ * B, T, variant, causal and presence of W_shared (its K, V, query streams, Z, routing and
+ * per-row attention log-sum-exp are reused; GQE_ERR_INVALID_ARG otherwise, or if
+ * gqe_enable_backward has not been called). The top-k selection is held constant.
+ *
+ *   x, W_*, B, T, N, G, k, d_h, variant, causal   as the forward (device, handle dtype).
+ *   dy        [B*T, dim]   upstream gradient of y, handle dtype (bf16), device.
+ *   aux_grad  host float   coefficient of the aux loss in the loss (0.01 in README, Usage).
+ *   dx        [B*T, dim]   float32, device: gradient of x.
+ *   dW_r      [N, dim], dW_q [N*d_h, dim], dW_k, dW_v [G*d_h, dim], dW_shared [d_h, dim]
+ *             (NULL exactly when W_shared is NULL), dW_o [dim, D_o]: float32, device,
+ *             overwritten (not accumulated into).
+ *
+ * Enqueued on `stream`; allocates nothing and does not synchronise. Hand-written kernels
+ * form the combine/router backward and the attention backward (tcgen05); the dense weight
+ * and input gradient GEMMs run in cuBLAS. The result is the same from run to run (no
+ * atomics). Errors as gqe_forward.
+ */
+gqe_status gqe_backward(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                        const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
+                        const void* W_o, int N, int G, int k, int d_h, int variant, int causal,
+                        const void* dy, float aux_grad, float* dx, float* dW_r, float* dW_q,
+                        float* dW_k, float* dW_v, float* dW_shared, float* dW_o, void* stream);
+
+/* gqe_backward_launches — kernels of this library the last gqe_backward launched (the cuBLAS
+ * GEMMs are not counted). */
+int gqe_backward_launches(gqe_handle h);
+
+/*
  * gqe_get_routing — copy the routing of the last gqe_forward on this handle.
  *   sel        [M, G, k] int32   selected expert index j within the group, ascending.
  *   gates      [M, G, k] float   p renormalised within the group (sums to 1 per group).
@@ -171,6 +214,31 @@ gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void
  * outside its cache, GQE_ERR_CUDA if the stream reports an error, else GQE_OK.
  */
 gqe_status gqe_check_device_status(gqe_handle h, void* stream);
+
+/*
+ * gqe_set_group_range — make the handle compute only groups g0 .. g1-1 of the layer, for
+ * group-parallel execution over several GPUs (one rank per range): routing is per group
+ * (README, Algorithm Overview), so the ranges split the layer with no exchange except the
+ * sum of their outputs.
+ *
+ * After this call gqe_forward still takes the WHOLE router W_r [N, dim] (every rank routes
+ * every group, so the slot weights and the aux loss are the whole layer's, bit-identical on
+ * every rank), but only the range's rows of the other weights:
+ *   W_q       [(g1-g0)*E*d_h, dim]  rows of experts g0*E .. g1*E-1;
+ *   W_k, W_v  [(g1-g0)*d_h, dim]    rows of heads g0 .. g1-1;
+ *   W_shared  the shared head, on the range with g0 == 0 only (NULL elsewhere;
+ *             GQE_ERR_INVALID_ARG otherwise);
+ *   W_o       [dim, D_o'] the columns of the range's blocks of Z, in Z's order: its routed
+ *             streams, the slot (variant gqe), the shared block (g0 == 0): D_o' =
+ *             ((g1-g0)*k + [gqe] + [shared here]) * d_h.
+ * `out` then receives this range's share of y; the layer's y is the sum over ranges (one
+ * all-reduce or reduce-scatter over the ranks). K, V, the query streams and Z of
+ * gqe_get_tensor hold the range's heads only. bf16 handles whose routing runs in the dense
+ * projection (N a power of two up to 32) only, else GQE_ERR_UNSUPPORTED; gqe_decode and
+ * gqe_backward return GQE_ERR_UNSUPPORTED unless the range is the whole layer
+ * (gqe_set_group_range(h, 0, G) restores it). GQE_ERR_INVALID_ARG unless 0 <= g0 < g1 <= G.
+ */
+gqe_status gqe_set_group_range(gqe_handle h, int g0, int g1);
 
 /* gqe_set_spin_limit — iteration cap of the device-side waits (0 = default). For tests
  * of the timeout path: a tiny limit makes the waits give up and report GQE_ERR_TIMEOUT. */

@@ -79,7 +79,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
     if jobs or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [cc, "-shared", *ARCH, "-o", LIB, *objs]
+        cmd = [cc, "-shared", *ARCH, "-o", LIB, *objs, "-lcublas"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             raise RuntimeError("link failed:\n" + r.stdout + r.stderr)

@@ -51,6 +51,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.V = take((size_t)G * M * d_h * esz);
   w.Q = take((size_t)S * M * d_h * esz);
   w.Z = take((size_t)M * Do * esz);
+  w.lse = (float*)take((size_t)S * M * 4);
   w.logits = (float*)take((size_t)M * N * 4);
   w.sel = (int32_t*)take((size_t)M * Gk * 4);
   w.psel = (float*)take((size_t)M * Gk * 4);
@@ -113,6 +114,8 @@ gqe_status gqe_create(gqe_handle* out, int dim, int N, int G, int k, int d_h, gq
   h->k = k;
   h->d_h = d_h;
   h->E = N / G;
+  h->g0 = 0;
+  h->g1 = G;
   h->dtype = dtype;
   h->max_tokens = max_tokens;
   h->esz = dtype == GQE_F32 ? 4 : 2;
@@ -148,7 +151,19 @@ void gqe_destroy(gqe_handle h) {
   if (!h) return;
   cudaDeviceSynchronize();
   cudaFree(h->ws.base);
+  backward_release(h);
   delete h;
+}
+
+gqe_status gqe_set_group_range(gqe_handle h, int g0, int g1) {
+  if (!h || g0 < 0 || g1 > h->G || g0 >= g1) return GQE_ERR_INVALID_ARG;
+  // a part of the layer needs the routing inside the dense projection (it routes every
+  // group, so slot weights and the aux loss stay the whole layer's)
+  if ((g0 != 0 || g1 != h->G) && !(h->dtype == GQE_BF16 && tc_dense_routes(h)))
+    return GQE_ERR_UNSUPPORTED;
+  h->g0 = g0;
+  h->g1 = g1;
+  return GQE_OK;
 }
 
 gqe_status gqe_set_spin_limit(gqe_handle h, int64_t limit) {
@@ -195,12 +210,15 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
     if (!aligned16(p)) return GQE_ERR_INVALID_ARG;
   if (W_shared && !aligned16(W_shared)) return GQE_ERR_INVALID_ARG;
   if (aux_loss && (reinterpret_cast<uintptr_t>(aux_loss) & 3u)) return GQE_ERR_INVALID_ARG;
+  // the shared head reads KV head 0: only the group range that holds group 0 computes it
+  if (W_shared && h->g0 != 0) return GQE_ERR_INVALID_ARG;
   const int64_t M64 = (int64_t)B * T;
   if (M64 > h->max_tokens) return GQE_ERR_WORKSPACE;
   const int M = (int)M64;
   const int has_shared = W_shared != nullptr;
-  const int S = G * k + has_shared;
-  const int Do = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
+  const int Gl = h->g1 - h->g0;  // the groups this handle computes
+  const int S = Gl * k + has_shared;
+  const int Do = (Gl * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   int launches = 0;
@@ -244,6 +262,12 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   h->last_S = S;
   h->last_Do = Do;
   h->last_launches = launches;
+  h->last_kind = ok ? 1 : 0;
+  h->last_B = B;
+  h->last_T = T;
+  h->last_variant = variant;
+  h->last_causal = causal;
+  h->last_shared = has_shared;
   return ok ? GQE_OK : GQE_ERR_CUDA;
 }
 
@@ -265,6 +289,7 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
   if (reinterpret_cast<uintptr_t>(lengths) & 3u) return GQE_ERR_INVALID_ARG;
   if (aux_loss && (reinterpret_cast<uintptr_t>(aux_loss) & 3u)) return GQE_ERR_INVALID_ARG;
   if (h->dtype != GQE_BF16) return GQE_ERR_UNSUPPORTED;
+  if (h->g0 != 0 || h->g1 != h->G) return GQE_ERR_UNSUPPORTED;  // whole layers only
   if (B > 65535) return GQE_ERR_UNSUPPORTED;  // one grid row per sequence
   if (B > h->max_tokens) return GQE_ERR_WORKSPACE;
   const int M = B;
@@ -305,6 +330,7 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
   h->last_S = S;
   h->last_Do = Do;
   h->last_launches = launches;
+  h->last_kind = ok ? 2 : 0;
   return ok ? GQE_OK : GQE_ERR_CUDA;
 }
 
@@ -332,8 +358,8 @@ gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void
   const void* src = nullptr;
   size_t n = 0;
   switch (which) {
-    case GQE_T_K: src = h->ws.K; n = (size_t)h->G * M * h->d_h * h->esz; break;
-    case GQE_T_V: src = h->ws.V; n = (size_t)h->G * M * h->d_h * h->esz; break;
+    case GQE_T_K: src = h->ws.K; n = (size_t)(h->g1 - h->g0) * M * h->d_h * h->esz; break;
+    case GQE_T_V: src = h->ws.V; n = (size_t)(h->g1 - h->g0) * M * h->d_h * h->esz; break;
     case GQE_T_Q: src = h->ws.Q; n = (size_t)h->last_S * M * h->d_h * h->esz; break;
     case GQE_T_Z: src = h->ws.Z; n = M * h->last_Do * h->esz; break;
     case GQE_T_PSEL: src = h->ws.psel; n = M * h->G * h->k * 4; break;

@@ -1,0 +1,367 @@
+// Backward pass of one GQE attention layer: gqe_enable_backward and gqe_backward.
+//
+// Training adds the load-balancing loss to the task loss and back-propagates through the
+// layer ("GQE: Grouped Query Experts" README, Usage); the renormalised slot gives the router
+// a differentiable path (gist.science summary, Output Construction). Given dy = dF/dy and the
+// aux coefficient dA, the gradients of F = <dy, y> + dA L are formed in this order:
+//   1. dZ = dy W_o and dW_o = dy^T Z                         (plain GEMMs, cuBLAS)
+//   2. combine_bwd_kernel, one warp per token: the stream gradients dO from dZ by variant
+//      (routed blocks, the slot's share w dslot, the shared block), D = rowsum(dO * O), the
+//      selected probabilities' gradients (slot weights with their denominator, or the raw p
+//      of weighted_concat), the aux term dA (E/G) f / M on every p, and the per-group
+//      softmax Jacobian: the router logits' gradient dl [M, N]
+//   3. the attention backward (tc_attention_bwd.cu): dQ into dQ_exp [M, N d_h] (each routed
+//      row at the column block of its expert, zero elsewhere) and dQ_sh, dK and dV [M, G d_h]
+//   4. the weight gradients dW = (gradient)^T x and dx = sum of (gradient) W over the router,
+//      the N query heads (dQ_exp: the unselected heads' blocks are zero, so one dense GEMM
+//      serves every expert), the K, V and shared projections (plain GEMMs, cuBLAS)
+// The top-k selection is held constant (its sets are the forward's).
+#include <cublas_v2.h>
+#include <string.h>
+
+#include "gqe_common.cuh"
+
+namespace gqe {
+
+namespace {
+
+struct CombBwd {
+  const float* dZ;          // [M, Do]
+  const __nv_bfloat16* Z;   // [M, Do]
+  const float* psel;        // [M, G k]
+  const float* w;           // [M, G k]
+  const int32_t* sel;       // [M, G k]
+  const float* logits;      // [M, N]
+  const int32_t* counts;    // [N]
+  __nv_bfloat16* dO;        // [S, M, d_h]
+  float* dsum;              // [S, M]
+  __nv_bfloat16* dl;        // [M, N]
+  int M, N, G, E, k, Sr, d_h, Do, variant, has_shared, shared_col;
+  float dA;
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+constexpr int kCombWarps = 8;
+
+// One warp per token; lane l holds head dims l and l + 32 (d_h <= 64).
+__global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const CombBwd P) {
+  __shared__ float s_g[kCombWarps][kMaxExperts];  // per routed stream: dw (gqe) / dp (wc)
+  pdl_wait();
+  pdl_allow_next();
+  const int wi = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t t = (int64_t)blockIdx.x * kCombWarps + wi;
+  if (t >= P.M) return;
+  const int DH = P.d_h;
+  const bool v0 = lane < DH, v1 = lane + 32 < DH;
+  const float* dz = P.dZ + t * P.Do;
+  const __nv_bfloat16* z = P.Z + t * P.Do;
+  const bool gqe = P.variant == GQE_VARIANT_GQE;
+  const bool wcat = P.variant == GQE_VARIANT_WEIGHTED_CONCAT;
+  float ds0 = 0.f, ds1 = 0.f;  // the slot's gradient
+  if (gqe) {
+    const int c = P.Sr * DH;
+    ds0 = v0 ? dz[c + lane] : 0.f;
+    ds1 = v1 ? dz[c + lane + 32] : 0.f;
+  }
+  float* g = s_g[wi];
+  // routed streams
+  for (int s = 0; s < P.Sr; ++s) {
+    const int c = s * DH;
+    float o0 = v0 ? __bfloat162float(z[c + lane]) : 0.f;
+    float o1 = v1 ? __bfloat162float(z[c + lane + 32]) : 0.f;
+    const float b0 = v0 ? dz[c + lane] : 0.f;
+    const float b1 = v1 ? dz[c + lane + 32] : 0.f;
+    float d0, d1, gs = 0.f;
+    if (wcat) {
+      // Z holds p O: O = Z / p; dO = p dZ; dp = <dZ, O>
+      const float p = P.psel[t * P.Sr + s];
+      o0 /= p;
+      o1 /= p;
+      d0 = p * b0;
+      d1 = p * b1;
+      gs = warp_sum(b0 * o0 + b1 * o1);
+    } else if (gqe) {
+      // dO = dZ + w dslot; dw = <dslot, O>
+      const float ww = P.w[t * P.Sr + s];
+      d0 = fmaf(ww, ds0, b0);
+      d1 = fmaf(ww, ds1, b1);
+      gs = warp_sum(ds0 * o0 + ds1 * o1);
+    } else {
+      d0 = b0;
+      d1 = b1;
+    }
+    // D from the bf16 dO the attention backward reads
+    d0 = bf16_round(d0);
+    d1 = bf16_round(d1);
+    const float D = warp_sum(d0 * o0 + d1 * o1);
+    __nv_bfloat16* dst = P.dO + ((int64_t)s * P.M + t) * DH;
+    if (v0) dst[lane] = __float2bfloat16_rn(d0);
+    if (v1) dst[lane + 32] = __float2bfloat16_rn(d1);
+    if (lane == 0) {
+      P.dsum[(int64_t)s * P.M + t] = D;
+      g[s] = gs;
+    }
+  }
+  if (P.has_shared) {
+    const int c = P.shared_col;
+    const float o0 = v0 ? __bfloat162float(z[c + lane]) : 0.f;
+    const float o1 = v1 ? __bfloat162float(z[c + lane + 32]) : 0.f;
+    const float d0 = v0 ? bf16_round(dz[c + lane]) : 0.f;
+    const float d1 = v1 ? bf16_round(dz[c + lane + 32]) : 0.f;
+    const float D = warp_sum(d0 * o0 + d1 * o1);
+    __nv_bfloat16* dst = P.dO + ((int64_t)P.Sr * P.M + t) * DH;
+    if (v0) dst[lane] = __float2bfloat16_rn(d0);
+    if (v1) dst[lane + 32] = __float2bfloat16_rn(d1);
+    if (lane == 0) P.dsum[(int64_t)P.Sr * P.M + t] = D;
+  }
+  __syncwarp();
+  // gradients of the selected probabilities
+  if (gqe) {
+    // w = p_sel / P_t: dp_sel = (dw - sum(dw w)) / P_t
+    float pt = 0.f, dww = 0.f;
+    for (int s = lane; s < P.Sr; s += 32) {
+      const float ww = P.w[t * P.Sr + s];
+      pt += P.psel[t * P.Sr + s];
+      dww += g[s] * ww;
+    }
+    pt = warp_sum(pt);
+    dww = warp_sum(dww);
+    __syncwarp();
+    for (int s = lane; s < P.Sr; s += 32) g[s] = (g[s] - dww) / pt;
+  } else if (!wcat) {
+    for (int s = lane; s < P.Sr; s += 32) g[s] = 0.f;
+  }
+  __syncwarp();
+  // router logits: dp on every p of the group (selected terms and the aux term), then the
+  // per-group softmax Jacobian dl = p (dp - sum p dp)
+  const float aux_c = P.dA * (float)P.E / (float)P.G / ((float)P.M * (float)P.k * (float)P.M);
+  for (int gg = 0; gg < P.G; ++gg) {
+    const int e0 = gg * P.E;
+    for (int jb = 0; jb < P.E; jb += 32) {
+      const int j = jb + lane;
+      const bool in = j < P.E;
+      const float l = in ? P.logits[t * P.N + e0 + j] : -INFINITY;
+      // the group's softmax over all E experts (E may exceed 32: reduce over the chunks)
+      float mx = -INFINITY;
+      for (int jj = lane; jj < P.E; jj += 32) mx = fmaxf(mx, P.logits[t * P.N + e0 + jj]);
+      mx = warp_max(mx);
+      float den = 0.f;
+      for (int jj = lane; jj < P.E; jj += 32) den += expf(P.logits[t * P.N + e0 + jj] - mx);
+      den = warp_sum(den);
+      const float p = in ? expf(l - mx) / den : 0.f;
+      float dp = in ? aux_c * (float)P.counts[e0 + j] : 0.f;
+      for (int r = 0; r < P.k; ++r)
+        if (in && P.sel[t * P.Sr + gg * P.k + r] == j) dp += g[gg * P.k + r];
+      // sum over the group of p dp
+      float spd = 0.f;
+      for (int jj = lane; jj < P.E; jj += 32) {
+        const float lj = P.logits[t * P.N + e0 + jj];
+        const float pj = expf(lj - mx) / den;
+        float dpj = aux_c * (float)P.counts[e0 + jj];
+        for (int r = 0; r < P.k; ++r)
+          if (P.sel[t * P.Sr + gg * P.k + r] == jj) dpj += g[gg * P.k + r];
+        spd += pj * dpj;
+      }
+      spd = warp_sum(spd);
+      if (in) P.dl[t * P.N + e0 + j] = __float2bfloat16_rn(p * (dp - spd));
+    }
+  }
+}
+
+// Row-major C[m x n] (fp32) = op(A)[m x k] op(B)[k x n] + beta C, bf16 operands: the
+// column-major call computes C^T = op(B)^T op(A)^T with the same transpose letters.
+bool gemm_rm(cublasHandle_t hb, bool ta, bool tb, int m, int n, int k, const void* A, int lda,
+             const void* B, int ldb, float* C, int ldc, float beta) {
+  const float alpha = 1.f;
+  return cublasGemmEx(hb, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, n, m,
+                      k, &alpha, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda, &beta, C,
+                      CUDA_R_32F, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) ==
+         CUBLAS_STATUS_SUCCESS;
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+constexpr size_t kCublasWorkspace = size_t(32) << 20;
+
+// Backward workspace layout; with base == nullptr only the size.
+size_t bwd_layout(BwdBuffers& b, char* base, const gqe_ctx* h) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  };
+  const int64_t M = h->max_tokens;
+  const int64_t S = (int64_t)h->G * h->k + 1;
+  const int64_t Do = ((int64_t)h->G * h->k + 2) * h->d_h;
+  b.dZ = (float*)take((size_t)M * Do * 4);
+  b.dO = (__nv_bfloat16*)take((size_t)S * M * h->d_h * 2);
+  b.dsum = (float*)take((size_t)S * M * 4);
+  b.dl = (__nv_bfloat16*)take((size_t)M * h->N * 2);
+  b.dq_exp = (__nv_bfloat16*)take((size_t)M * h->N * h->d_h * 2);
+  b.dq_sh = (__nv_bfloat16*)take((size_t)M * h->d_h * 2);
+  b.dk = (__nv_bfloat16*)take((size_t)M * h->G * h->d_h * 2);
+  b.dv = (__nv_bfloat16*)take((size_t)M * h->G * h->d_h * 2);
+  b.counter = (int*)take(16 * sizeof(int));
+  b.cublas_ws = take(kCublasWorkspace);
+  return off;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+void backward_release(gqe_ctx* h) {
+  if (h->cublas) cublasDestroy(static_cast<cublasHandle_t>(h->cublas));
+  if (h->bwd_base) cudaFree(h->bwd_base);
+  h->cublas = nullptr;
+  h->bwd_base = nullptr;
+}
+
+}  // namespace gqe
+
+using namespace gqe;
+
+extern "C" {
+
+gqe_status gqe_enable_backward(gqe_handle h) {
+  if (!h) return GQE_ERR_INVALID_ARG;
+  if (!tc_backward_supported(h)) return GQE_ERR_UNSUPPORTED;
+  if (h->bwd_base) return GQE_OK;
+  const size_t bytes = bwd_layout(h->bwd, nullptr, h);
+  void* base = nullptr;
+  if (cudaMalloc(&base, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return GQE_ERR_CUDA;
+  }
+  if (cudaMemset(base, 0, bytes) != cudaSuccess) {
+    cudaFree(base);
+    return GQE_ERR_CUDA;
+  }
+  cublasHandle_t hb = nullptr;
+  if (cublasCreate(&hb) != CUBLAS_STATUS_SUCCESS) {
+    cudaFree(base);
+    return GQE_ERR_CUDA;
+  }
+  bwd_layout(h->bwd, static_cast<char*>(base), h);
+  if (cublasSetWorkspace(hb, h->bwd.cublas_ws, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS) {
+    cublasDestroy(hb);
+    cudaFree(base);
+    return GQE_ERR_CUDA;
+  }
+  h->bwd_base = base;
+  h->bwd_bytes = bytes;
+  h->cublas = hb;
+  return GQE_OK;
+}
+
+gqe_status gqe_backward(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                        const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
+                        const void* W_o, int N, int G, int k, int d_h, int variant, int causal,
+                        const void* dy, float aux_grad, float* dx, float* dW_r, float* dW_q,
+                        float* dW_k, float* dW_v, float* dW_shared, float* dW_o, void* stream) {
+  if (!h) return GQE_ERR_INVALID_ARG;
+  if (!h->bwd_base) return GQE_ERR_INVALID_ARG;  // gqe_enable_backward first
+  if (h->g0 != 0 || h->g1 != h->G) return GQE_ERR_UNSUPPORTED;  // whole layers only
+  if (N != h->N || G != h->G || k != h->k || d_h != h->d_h) return GQE_ERR_INVALID_ARG;
+  if (B < 1 || T < 1) return GQE_ERR_INVALID_ARG;
+  if (variant < GQE_VARIANT_GQE || variant > GQE_VARIANT_HARD_CONCAT) return GQE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQE_ERR_INVALID_ARG;
+  if (!x || !W_r || !W_q || !W_k || !W_v || !W_o || !dy || !dx || !dW_r || !dW_q || !dW_k ||
+      !dW_v || !dW_o)
+    return GQE_ERR_INVALID_ARG;
+  if ((W_shared == nullptr) != (dW_shared == nullptr)) return GQE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_r, W_q, W_k, W_v, W_o, dy, dx, dW_r, dW_q, dW_k, dW_v, dW_o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GQE_ERR_INVALID_ARG;
+  if (W_shared && (!aligned16(W_shared) || !aligned16(dW_shared))) return GQE_ERR_INVALID_ARG;
+  const int64_t M64 = (int64_t)B * T;
+  if (M64 > h->max_tokens) return GQE_ERR_WORKSPACE;
+  const int M = (int)M64;
+  const int has_shared = W_shared != nullptr;
+  // the saved state must be this layer's last forward
+  if (h->last_kind != 1 || h->last_M != M || h->last_B != B || h->last_T != T ||
+      h->last_variant != variant || h->last_causal != causal || h->last_shared != has_shared)
+    return GQE_ERR_INVALID_ARG;
+  const int S = G * k + has_shared;
+  const int Do = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
+  const int dim = h->dim;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cublasHandle_t hb = static_cast<cublasHandle_t>(h->cublas);
+  if (cublasSetStream(hb, st) != CUBLAS_STATUS_SUCCESS) return GQE_ERR_CUDA;
+  const BwdBuffers& b = h->bwd;
+  int launches = 0;
+  bool ok = true;
+  // 1. dZ = dy W_o; dW_o = dy^T Z
+  ok = ok && gemm_rm(hb, false, false, M, Do, dim, dy, dim, W_o, Do, b.dZ, Do, 0.f);
+  ok = ok && gemm_rm(hb, true, false, dim, Do, M, dy, dim, h->ws.Z, Do, dW_o, Do, 0.f);
+  // 2. dQ_exp is zero outside the selected heads' blocks
+  ok = ok && cudaMemsetAsync(b.dq_exp, 0, (size_t)M * N * d_h * 2, st) == cudaSuccess;
+  if (ok) {
+    CombBwd c;
+    c.dZ = b.dZ;
+    c.Z = static_cast<const __nv_bfloat16*>(h->ws.Z);
+    c.psel = h->ws.psel;
+    c.w = h->ws.w;
+    c.sel = h->ws.sel;
+    c.logits = h->ws.logits;
+    c.counts = h->ws.counts;
+    c.dO = b.dO;
+    c.dsum = b.dsum;
+    c.dl = b.dl;
+    c.M = M;
+    c.N = N;
+    c.G = G;
+    c.E = h->E;
+    c.k = k;
+    c.Sr = G * k;
+    c.d_h = d_h;
+    c.Do = Do;
+    c.variant = variant;
+    c.has_shared = has_shared;
+    c.shared_col = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0)) * d_h;
+    c.dA = aux_grad;
+    combine_bwd_kernel<<<(M + kCombWarps - 1) / kCombWarps, kCombWarps * 32, 0, st>>>(c);
+    ok = cudaGetLastError() == cudaSuccess;
+    ++launches;
+  }
+  // 3. attention backward
+  if (ok) {
+    const int n = launch_tc_attention_backward(h, b, B, T, S, has_shared, causal, st);
+    ok = n >= 0;
+    launches += n > 0 ? n : 0;
+  }
+  // 4. weight gradients and dx
+  const int Nd = N * d_h, Gd = G * d_h;
+  ok = ok && gemm_rm(hb, true, false, Nd, dim, M, b.dq_exp, Nd, x, dim, dW_q, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dk, Gd, x, dim, dW_k, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dv, Gd, x, dim, dW_v, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, N, dim, M, b.dl, N, x, dim, dW_r, dim, 0.f);
+  if (has_shared)
+    ok = ok && gemm_rm(hb, true, false, d_h, dim, M, b.dq_sh, d_h, x, dim, dW_shared, dim, 0.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Nd, b.dq_exp, Nd, W_q, dim, dx, dim, 0.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dk, Gd, W_k, dim, dx, dim, 1.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dv, Gd, W_v, dim, dx, dim, 1.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, N, b.dl, N, W_r, dim, dx, dim, 1.f);
+  if (has_shared)
+    ok = ok && gemm_rm(hb, false, false, M, dim, d_h, b.dq_sh, d_h, W_shared, dim, dx, dim, 1.f);
+  h->last_bwd_launches = launches;
+  return ok ? GQE_OK : GQE_ERR_CUDA;
+}
+
+int gqe_backward_launches(gqe_handle h) { return h ? h->last_bwd_launches : -1; }
+
+}  // extern "C"

@@ -105,6 +105,7 @@ struct Workspace {
   void* V = nullptr;        // [G, M, d_h]
   void* Q = nullptr;        // [S, M, d_h]
   void* Z = nullptr;        // [M, D_o]
+  float* lse = nullptr;     // [S, M] attention log2-sum-exp2 per (stream, token) (bf16 path)
   float* logits = nullptr;  // [M, N]
   int32_t* sel = nullptr;   // [M, G, k]
   float* psel = nullptr;    // [M, G, k]
@@ -132,10 +133,26 @@ struct Workspace {
   size_t bytes = 0;
 };
 
+// Backward-pass workspace (gqe_enable_backward), sized for max_tokens.
+struct BwdBuffers {
+  float* dZ = nullptr;                // [M, D_o] gradient of the concatenation
+  __nv_bfloat16* dO = nullptr;        // [S, M, d_h] gradients of the stream outputs
+  float* dsum = nullptr;              // [S, M] rowsum(dO * O)
+  __nv_bfloat16* dl = nullptr;        // [M, N] gradient of the router logits
+  __nv_bfloat16* dq_exp = nullptr;    // [M, N d_h] routed query gradients at their expert
+  __nv_bfloat16* dq_sh = nullptr;     // [M, d_h] shared-head query gradient
+  __nv_bfloat16* dk = nullptr;        // [M, G d_h] key gradients, token-major
+  __nv_bfloat16* dv = nullptr;        // [M, G d_h] value gradients, token-major
+  int* counter = nullptr;             // [4] work counters of the two attention kernels
+  void* cublas_ws = nullptr;          // cuBLAS workspace
+};
+
 }  // namespace gqe
 
 struct gqe_ctx {
   int dim, N, G, k, d_h, E;
+  // the groups this handle computes, [g0, g1) (gqe_set_group_range; all G by default)
+  int g0 = 0, g1 = 0;
   gqe_dtype dtype;
   int64_t max_tokens;
   int esz;  // bytes per stored element
@@ -148,7 +165,17 @@ struct gqe_ctx {
   int n_stage_events = 0;
   // state of the last forward
   int last_M = 0, last_S = 0, last_Do = 0, last_launches = 0;
+  // what the last call was (1 gqe_forward, 2 gqe_decode) and its arguments, which a
+  // gqe_backward must repeat
+  int last_kind = 0, last_B = 0, last_T = 0, last_variant = -1, last_causal = -1,
+      last_shared = -1;
   int route_set = 0;  // the dense-projection routing's cursor set for the next call
+  // backward pass (gqe_enable_backward)
+  void* bwd_base = nullptr;
+  size_t bwd_bytes = 0;
+  void* cublas = nullptr;  // cublasHandle_t
+  gqe::BwdBuffers bwd;
+  int last_bwd_launches = 0;
 };
 
 namespace gqe {
@@ -196,5 +223,10 @@ int launch_tc_decode_attention(gqe_ctx* h, int B, int S, int has_shared, int var
                                void* k_cache, void* v_cache, int L_max, const int32_t* lengths,
                                cudaStream_t st);
 int decode_chunks(const gqe_ctx* h, int B, int L_max);
+// Backward pass (tc_attention_bwd.cu, backward.cu): bf16 handles with d_h <= 64.
+bool tc_backward_supported(const gqe_ctx* h);
+int launch_tc_attention_backward(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S,
+                                 int has_shared, int causal, cudaStream_t st);
+void backward_release(gqe_ctx* h);
 
 }  // namespace gqe

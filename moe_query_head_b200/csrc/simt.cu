@@ -235,7 +235,7 @@ attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __r
 // routed block, fp32 accumulation, one 16-byte store.
 template <typename T>
 __global__ void slot_kernel(T* __restrict__ Z, const float* __restrict__ w, int M, int Sr,
-                            int d_h, int Do) {
+                            int d_h, int Do, int w_stride, int w_off) {
   constexpr int VEC = 16 / sizeof(T);
   pdl_wait();  // Z and the slot weights are complete from here on
   pdl_allow_next();
@@ -255,7 +255,7 @@ __global__ void slot_kernel(T* __restrict__ Z, const float* __restrict__ w, int 
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const bool in = s0 + u < Sr;
-      ws[u] = in ? w[t * Sr + s0 + u] : 0.f;
+      ws[u] = in ? w[t * w_stride + w_off + s0 + u] : 0.f;
       raw[u] = in ? *reinterpret_cast<const uint4*>(zt + (int64_t)(s0 + u) * d_h)
                   : make_uint4(0, 0, 0, 0);
     }
@@ -358,16 +358,18 @@ int launch_simt_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int v
 
 int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st) {
   if (variant != GQE_VARIANT_GQE) return 0;  // weighted_concat is applied in attention
-  const int Sr = h->G * h->k;
+  // the handle's routed streams; the slot weights are the whole layer's [M, G k]
+  const int Sr = (h->g1 - h->g0) * h->k;
+  const int w_stride = h->G * h->k, w_off = h->g0 * h->k;
   const int64_t n = (int64_t)M * h->d_h / (16 / h->esz);
   const int blocks = (int)((n + 255) / 256);
   if (h->dtype == GQE_F32)
     slot_kernel<float><<<blocks, 256, 0, st>>>(static_cast<float*>(h->ws.Z), h->ws.w, M, Sr,
-                                               h->d_h, Do);
+                                               h->d_h, Do, w_stride, w_off);
   else
     return launch_pdl(slot_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
                       static_cast<__nv_bfloat16*>(h->ws.Z), static_cast<const float*>(h->ws.w),
-                      M, Sr, h->d_h, Do) == cudaSuccess
+                      M, Sr, h->d_h, Do, w_stride, w_off) == cudaSuccess
                ? 1
                : -1;
   return cudaGetLastError() == cudaSuccess ? 1 : -1;

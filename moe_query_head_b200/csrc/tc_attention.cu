@@ -102,8 +102,10 @@ constexpr int kFmaPairsOf8 = GQE_ATTN_FMA_PAIRS_OF_8;
 struct Params {
   CUtensorMap tm_q, tm_k, tm_v;
   __nv_bfloat16* Z;
-  const float* psel;
+  float* lse;  // [S, M] per-row log2-sum-exp2 of the scaled scores (for the backward pass)
+  const float* psel;  // [M, psel_stride]: stream s's p at column psel_off + s
   int M, T, B, S, Sr, k, Do, shared_col, weighted, causal;
+  int psel_stride, psel_off;
   int nq, items;
   int chunked;  // 1: tm_q / tm_k / tm_v are 3D chunked maps, one copy per tile
   float scale_log2;
@@ -629,10 +631,12 @@ attn_kernel(const __grid_constant__ Params P) {
         l = __uint_as_float(r[0]);
       }
       float scale = 1.f / l;
+      // the row's log2-sum-exp2 of its scaled scores: p = exp2(s * scale_log2 - lse)
+      if (valid) P.lse[(int64_t)it.s * P.M + tok] = m_used + __log2f(l);
       int col;
       if (it.s < P.Sr) {
         col = it.s * DH;
-        if (P.weighted && valid) scale *= P.psel[tok * P.Sr + it.s];
+        if (P.weighted && valid) scale *= P.psel[tok * P.psel_stride + P.psel_off + it.s];
       } else {
         col = P.shared_col;
       }
@@ -685,23 +689,27 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
                                 : C::CW == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                               : CU_TENSOR_MAP_SWIZZLE_32B;
   // One copy per tile where the driver accepts the chunked 3D maps, else one per chunk.
+  const uint64_t kv_rows = (uint64_t)(h->g1 - h->g0) * M;  // this handle's KV heads
   P.chunked = C::NC > 1 &&
               tmap_bf16_chunked(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, TQ, sw) &&
-              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw) &&
-              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw);
+              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, kv_rows, DH, C::CW, TK, sw) &&
+              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, kv_rows, DH, C::CW, TK, sw);
   if (!P.chunked &&
       (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, TQ, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, TK, sw)))
+       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, kv_rows, DH, C::CW, TK, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, kv_rows, DH, C::CW, TK, sw)))
     return -1;
   P.Z = static_cast<__nv_bfloat16*>(h->ws.Z);
+  P.lse = h->ws.lse;
   P.psel = h->ws.psel;
   P.M = M;
   P.T = T;
   P.B = B;
   P.S = S;
-  P.Sr = h->G * h->k;
+  P.Sr = (h->g1 - h->g0) * h->k;
   P.k = h->k;
+  P.psel_stride = h->G * h->k;
+  P.psel_off = h->g0 * h->k;
   P.Do = Do;
   P.shared_col = shared_col;
   P.weighted = weighted;
@@ -724,7 +732,7 @@ int launch_dh(gqe_ctx* h, int B, int T, int S, int shared_col, int weighted, int
 int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,
                         int causal, int Do, cudaStream_t st) {
   (void)has_shared;
-  const int Sr = h->G * h->k;
+  const int Sr = (h->g1 - h->g0) * h->k;
   const int shared_col = (Sr + (variant == GQE_VARIANT_GQE ? 1 : 0)) * h->d_h;
   const int weighted = variant == GQE_VARIANT_WEIGHTED_CONCAT;
   switch (h->d_h) {

@@ -1,0 +1,919 @@
+// Tensor-core (tcgen05) backward pass of the GQE attention: the gradients of the query
+// streams, keys and values, given the forward's per-row log2-sum-exp2 (lse), the upstream
+// gradient dO of every stream's output and D = rowsum(dO * O).
+//
+// Stream s < G*k holds the routed queries of group s / k and reads that group's KV head; the
+// last stream is the always-on shared head and reads KV head 0 ("GQE: Grouped Query
+// Experts" README, Algorithm Overview; gist.science summary, Output Construction). With
+// P = softmax(Q K^T / sqrt(d_h)) (causal or not), dP = dO V^T and dS = P * (dP - D):
+//   dQ = dS K / sqrt(d_h),   dK = sum over the head's streams of dS^T Q / sqrt(d_h),
+//   dV = sum over the head's streams of P^T dO.
+//
+// Two kernels, neither with atomics (every output row is written by one CTA, so the result
+// is the same from run to run):
+//   attn_bwd_dq_kernel    work item = (sequence, stream, 128-query tile); for each key tile
+//                         S = Q K^T and dP = dO V^T (both operands from shared memory) into
+//                         TMEM, the softmax warpgroup forms dS in bf16 in TMEM, and
+//                         dQ += dS K (A from TMEM, K as an MN-major shared-memory operand)
+//                         accumulates in TMEM. The routed stream (g, r) of token t lands in
+//                         row t of dQ_exp [M, N d_h] at the column block of its expert
+//                         g E + sel[t, g, r]; the shared stream in dQ_sh [M, d_h].
+//   attn_bwd_dkdv_kernel  work item = (sequence, KV head, 128-key tile); for each query tile
+//                         of each stream that reads the head, S^T = K Q^T and dP^T = V dO^T
+//                         into TMEM, the softmax warpgroup (one key per thread) forms P^T
+//                         and dS^T in bf16 in TMEM, and dV += P^T dO, dK += dS^T Q
+//                         accumulate in TMEM over all of the head's streams. dK, dV land
+//                         token-major in [M, G d_h] (head g at column g d_h).
+// Warps: 0 TMA loads, 1 TMEM owner and MMA issue, 2-3 idle, 4-7 softmax and epilogue. One
+// CTA per SM (TMEM: 512 columns), persistent, heaviest items first. Head dims up to 64.
+#include <cudaTypedefs.h>
+
+#include "gqe_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace gqe {
+
+bool tmap_bf16_2d_ext(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                      uint64_t ld, uint32_t box_cols, uint32_t box_rows,
+                      CUtensorMapSwizzle sw);
+bool tmap_bf16_chunked(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
+                       uint64_t ld, uint32_t chunk_cols, uint32_t box_rows,
+                       CUtensorMapSwizzle sw);
+
+namespace {
+
+using namespace tc;
+
+constexpr int THREADS = 256;
+constexpr int TQ = 128;  // query rows of a tile
+constexpr int TK = 128;  // key rows of a tile
+
+template <int DH>
+struct BCfg {
+  static_assert(DH % 16 == 0 && DH <= 64, "the backward kernels take head dims up to 64");
+  // the forward's chunking: 64-column chunks (128-byte swizzle) for 64, else 16-column
+  // chunks (32-byte swizzle)
+  static constexpr int CW = (DH % 64 == 0) ? 64 : 16;
+  static constexpr int NC = DH / CW;
+  static constexpr uint32_t LAYOUT = CW == 64 ? kSwizzle128B : kSwizzle32B;
+  static constexpr int ROW_BYTES = CW * 2;
+  static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;
+  static constexpr int TILE_BYTES = 128 * DH * 2;
+  static constexpr int STAGES = 2;  // ring of tile pairs
+  // two fixed tiles, the ring of pairs, alignment, barriers, lse / D buffers
+  static constexpr int SMEM = 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 512 + 2 * 2 * 128 * 4;
+  static constexpr int TMEM_COLS = 512;
+};
+
+// TMEM columns. dQ kernel: S, dP (fp32), dS (bf16 pairs), dQ (fp32).
+constexpr int Q_S = 0, Q_DP = 128, Q_DS = 256, Q_DQ = 320;
+// dK / dV kernel: S^T, dP^T (fp32), P^T, dS^T (bf16 pairs), dV, dK (fp32, up to 64 each).
+constexpr int K_S = 0, K_DP = 128, K_P = 256, K_DS = 320, K_DV = 384, K_DK = 448;
+
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO [S M, d_h]; K, V [G M, d_h]
+  const float* lse;     // [S, M]
+  const float* dsum;    // [S, M] rowsum(dO * O)
+  const int32_t* sel;   // [M, G, k]
+  __nv_bfloat16* dq_exp;  // [M, N d_h]
+  __nv_bfloat16* dq_sh;   // [M, d_h]
+  __nv_bfloat16* dk;      // [M, G d_h]
+  __nv_bfloat16* dv;      // [M, G d_h]
+  int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, items, chunked;
+  float scale_log2;  // log2(e) / sqrt(d_h)
+  float scale;       // 1 / sqrt(d_h)
+  int* counter;      // [2] item counter and exit counter (zero at launch; reset by the last CTA)
+  int32_t* status;
+  int64_t spin;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const BwdParams& P,
+                                          volatile int* abort_flag) {
+  const bool ok = !__any_sync(0xffffffffu, !mbar_wait(bar, parity, P.spin));
+  if (!ok && (threadIdx.x & 31) == 0) {
+    *abort_flag = 1;
+    atomicExch(P.status, kStatusTimeout);
+  }
+  return ok;
+}
+__device__ __forceinline__ bool lane_wait(uint64_t* bar, uint32_t parity, const BwdParams& P,
+                                          volatile int* abort_flag) {
+  if (mbar_wait(bar, parity, P.spin)) return true;
+  *abort_flag = 1;
+  atomicExch(P.status, kStatusTimeout);
+  return false;
+}
+
+template <int DH>
+__device__ __forceinline__ void load_tile(const BwdParams& P, const CUtensorMap* map,
+                                          uint8_t* dst, int row, uint64_t* bar) {
+  using C = BCfg<DH>;
+  if (C::NC > 1 && P.chunked) {
+    tma_load_3d(dst, map, 0, row, 0, bar);
+  } else {
+#pragma unroll
+    for (int c = 0; c < C::NC; ++c) tma_load_2d(dst + c * C::CHUNK_BYTES, map, c * C::CW, row, bar);
+  }
+}
+
+// K-major descriptor offset (16-byte units) of head-dim columns kk*16 .. kk*16+15.
+template <int DH>
+__device__ __forceinline__ uint32_t kmajor_off(int kk) {
+  using C = BCfg<DH>;
+  return (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4;
+}
+
+// bf16 pairs of the packed row -> 16 TMEM columns at a time
+__device__ __forceinline__ void store_packed32(uint32_t taddr, const uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c0 = 0; c0 < 32; c0 += 16) {
+    uint32_t r[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) r[x] = pk[c0 + x];
+    tmem_st16(taddr + c0, r);
+  }
+}
+__device__ __forceinline__ void store_packed64(uint32_t taddr, const uint32_t (&pk)[64]) {
+#pragma unroll
+  for (int c0 = 0; c0 < 64; c0 += 16) {
+    uint32_t r[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) r[x] = pk[c0 + x];
+    tmem_st16(taddr + c0, r);
+  }
+}
+
+struct Shared {
+  uint64_t* q_full;   // fixed pair loaded (dq: Q, dO; dkdv: K, V)
+  uint64_t* q_empty;
+  uint64_t* r_full;   // [STAGES] ring pairs (dq: K, V; dkdv: Q, dO)
+  uint64_t* r_empty;  // [STAGES]
+  uint64_t* sdp_full;
+  uint64_t* s_free;
+  uint64_t* d_ready;  // dS (and P^T) written to TMEM
+  uint64_t* d_free;   // their MMAs are done
+  uint64_t* acc_full;
+  uint64_t* acc_free;
+  uint64_t* item_full;   // [2]
+  uint64_t* item_empty;  // [2]
+  uint64_t* l_bar;       // [2] the softmax warpgroup has filled sL / sD buffer 0 / 1
+  volatile int* item_ring;
+  uint32_t* tmem_holder;
+  volatile int* abort_flag;
+  float* sL;  // [2][128] lse of the job's queries (dkdv)
+  float* sD;  // [2][128]
+};
+
+template <int DH>
+__device__ __forceinline__ Shared carve(uint8_t* smem, uint8_t*& sFix0, uint8_t*& sFix1,
+                                        uint8_t*& sR0, uint8_t*& sR1) {
+  using C = BCfg<DH>;
+  sFix0 = smem;
+  sFix1 = smem + C::TILE_BYTES;
+  sR0 = sFix1 + C::TILE_BYTES;                  // ring: first tile of each pair
+  sR1 = sR0 + C::STAGES * C::TILE_BYTES;        // ring: second tile of each pair
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sR1 + C::STAGES * C::TILE_BYTES);
+  Shared sh;
+  sh.q_full = bar;
+  sh.q_empty = bar + 1;
+  sh.r_full = bar + 2;
+  sh.r_empty = sh.r_full + C::STAGES;
+  sh.sdp_full = sh.r_empty + C::STAGES;
+  sh.s_free = sh.sdp_full + 1;
+  sh.d_ready = sh.s_free + 1;
+  sh.d_free = sh.d_ready + 1;
+  sh.acc_full = sh.d_free + 1;
+  sh.acc_free = sh.acc_full + 1;
+  sh.item_full = sh.acc_free + 1;
+  sh.item_empty = sh.item_full + 2;
+  sh.l_bar = sh.item_empty + 2;
+  sh.item_ring = reinterpret_cast<volatile int*>(sh.l_bar + 2);
+  sh.tmem_holder = reinterpret_cast<uint32_t*>(sh.l_bar + 3);
+  sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_holder + 1);
+  sh.sL = reinterpret_cast<float*>(sh.l_bar + 4);
+  sh.sD = sh.sL + 256;
+  return sh;
+}
+
+__device__ __forceinline__ void init_shared(const Shared& sh, int stages) {
+  mbar_init(sh.q_full, 1);
+  mbar_init(sh.q_empty, 1);
+  for (int s = 0; s < stages; ++s) {
+    mbar_init(&sh.r_full[s], 1);
+    mbar_init(&sh.r_empty[s], 1);
+  }
+  mbar_init(sh.sdp_full, 1);
+  mbar_init(sh.s_free, 4);
+  mbar_init(sh.d_ready, 4);
+  mbar_init(sh.d_free, 1);
+  mbar_init(sh.acc_full, 1);
+  mbar_init(sh.acc_free, 4);
+  for (int r = 0; r < 2; ++r) {
+    mbar_init(&sh.item_full[r], 1);
+    mbar_init(&sh.item_empty[r], 5);  // the MMA warp and the four softmax warps
+    mbar_init(&sh.l_bar[r], 128);     // every softmax thread
+  }
+  *sh.abort_flag = 0;
+  fence_barrier_init();
+}
+
+// Claims items for the CTA (lane 0 of warp 0) and publishes them through the two-slot ring;
+// -1 ends the CTA's work.
+__device__ __forceinline__ bool publish_item(const Shared& sh, const BwdParams& P, int& islot,
+                                             uint32_t& iphase, int& i) {
+  if (!lane_wait(&sh.item_empty[islot], iphase ^ 1, P, sh.abort_flag)) return false;
+  i = atomicAdd(P.counter, 1);
+  if (i >= P.items) i = -1;
+  sh.item_ring[islot] = i;
+  mbar_arrive(&sh.item_full[islot]);
+  if (++islot == 2) {
+    islot = 0;
+    iphase ^= 1;
+  }
+  return true;
+}
+__device__ __forceinline__ bool next_item(const Shared& sh, const BwdParams& P, int& islot,
+                                          uint32_t& iphase, int& i) {
+  if (!warp_wait(&sh.item_full[islot], iphase, P, sh.abort_flag)) return false;
+  i = sh.item_ring[islot];
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.item_empty[islot]);
+  if (++islot == 2) {
+    islot = 0;
+    iphase ^= 1;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void finish(const BwdParams& P, uint32_t tmem, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && atomicAdd(P.counter + 1, 1) == (int)gridDim.x - 1) {
+    P.counter[0] = 0;
+    P.counter[1] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// dQ: item (b, s, query tile), heaviest (last) query tiles first when causal.
+// ---------------------------------------------------------------------------------------
+struct QItem {
+  int b, s, qt, nk;
+};
+__device__ __forceinline__ QItem decode_q(const BwdParams& P, int i) {
+  QItem it;
+  const int bs = P.B * P.S;
+  it.qt = P.causal ? P.nq - 1 - i / bs : i / bs;
+  const int r = i % bs;
+  it.s = r % P.S;
+  it.b = r / P.S;
+  it.nk = P.causal ? it.qt + 1 : P.nq;
+  return it;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
+  using C = BCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t *sQ, *sdO, *sK, *sV;
+  const Shared sh = carve<DH>(smem, sQ, sdO, sK, sV);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) init_shared(sh, C::STAGES);
+  if (warp == 1) {
+    tmem_alloc(sh.tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&P.tm_q);
+    prefetch_tmap(&P.tm_k);
+    prefetch_tmap(&P.tm_v);
+    prefetch_tmap(&P.tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sh.tmem_holder;
+  pdl_wait();
+  pdl_allow_next();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ loads
+    if (lane == 0) {
+      int st = 0, islot = 0;
+      uint32_t r_phase = 0, q_phase = 0, iphase = 0;
+      while (!*sh.abort_flag) {
+        int i;
+        if (!publish_item(sh, P, islot, iphase, i) || i < 0) break;
+        const QItem it = decode_q(P, i);
+        if (!lane_wait(sh.q_empty, q_phase ^ 1, P, sh.abort_flag)) break;
+        q_phase ^= 1;
+        mbar_arrive_expect_tx(sh.q_full, 2 * C::TILE_BYTES);
+        const int qrow = it.s * P.M + it.b * P.T + it.qt * TQ;
+        load_tile<DH>(P, &P.tm_q, sQ, qrow, sh.q_full);
+        load_tile<DH>(P, &P.tm_do, sdO, qrow, sh.q_full);
+        const int kvh = it.s < P.Sr ? it.s / P.k : 0;
+        const int krow0 = kvh * P.M + it.b * P.T;
+        for (int j = 0; j < it.nk; ++j) {
+          if (!lane_wait(&sh.r_empty[st], r_phase ^ 1, P, sh.abort_flag)) break;
+          mbar_arrive_expect_tx(&sh.r_full[st], 2 * C::TILE_BYTES);
+          load_tile<DH>(P, &P.tm_k, sK + st * C::TILE_BYTES, krow0 + j * TK, &sh.r_full[st]);
+          load_tile<DH>(P, &P.tm_v, sV + st * C::TILE_BYTES, krow0 + j * TK, &sh.r_full[st]);
+          if (++st == C::STAGES) {
+            st = 0;
+            r_phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issue
+    const uint32_t idesc_s = idesc_bf16_f32(TQ, TK);
+    const uint32_t idesc_dq = idesc_bf16_f32(TQ, DH) | (1u << 16);  // B (K) MN-major
+    const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t do_desc = smem_desc(smem_u32(sdO), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t v_desc = smem_desc(smem_u32(sV), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t kmn_desc =
+        smem_desc_mn(smem_u32(sK), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kStep = C::TILE_BYTES >> 4;
+    int st = 0, islot = 0;
+    uint32_t r_phase = 0, q_phase = 0, iphase = 0;
+    uint32_t n_sf = 0, n_dr = 0, n_items = 0;
+    bool ok = true;
+    // S = Q K^T and dP = dO V^T of the next key tile
+    auto issue_sdp = [&](int stage, uint32_t phase) -> bool {
+      if (!warp_wait(&sh.r_full[stage], phase, P, sh.abort_flag)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t kd = k_desc + (uint64_t)(stage * kStep);
+        const uint64_t vd = v_desc + (uint64_t)(stage * kStep);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t o = kmajor_off<DH>(kk);
+          mma_ss(tmem + Q_S, q_desc + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t o = kmajor_off<DH>(kk);
+          mma_ss(tmem + Q_DP, do_desc + o, vd + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(sh.sdp_full);
+      }
+      __syncwarp();
+      return true;
+    };
+    while (ok && !*sh.abort_flag) {
+      int i;
+      if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
+      const QItem it = decode_q(P, i);
+      if (!warp_wait(sh.q_full, q_phase, P, sh.abort_flag)) break;
+      q_phase ^= 1;
+      int st_next = st;
+      uint32_t ph_next = r_phase;
+      if (!issue_sdp(st_next, ph_next)) break;
+      for (int j = 0; j < it.nk; ++j) {
+        const int st_j = st_next;
+        if (++st_next == C::STAGES) {
+          st_next = 0;
+          ph_next ^= 1;
+        }
+        if (j + 1 < it.nk) {
+          // the softmax warps hold S(j), dP(j) in registers: the next pair may be written
+          if (!warp_wait(sh.s_free, n_sf & 1, P, sh.abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!issue_sdp(st_next, ph_next)) { ok = false; break; }
+        }
+        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_dr;
+        if (j == 0 && n_items > 0 &&
+            !warp_wait(sh.acc_free, (n_items - 1) & 1, P, sh.abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          // dQ (+)= dS K: A = dS (queries x keys, TMEM), B = K tile (N = head dim,
+          // K = keys; MN-major)
+          const uint64_t kd = kmn_desc + (uint64_t)(st_j * kStep);
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk)
+            mma_ts(tmem + Q_DQ, tmem + Q_DS + kk * 8,
+                   kd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_dq,
+                   (j == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&sh.r_empty[st_j]);
+          mma_commit(sh.d_free);
+          if (j + 1 == it.nk) {
+            mma_commit(sh.acc_full);
+            mma_commit(sh.q_empty);
+          }
+        }
+        __syncwarp();
+      }
+      st = st_next;
+      r_phase = ph_next;
+      ++n_items;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t t_base = tmem + lane_off;
+    uint32_t n_sdp = 0, n_ds = 0, n_acc = 0;
+    int islot = 0;
+    uint32_t iphase = 0;
+    const float c2 = P.scale_log2;
+    while (!*sh.abort_flag) {
+      int i;
+      if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
+      const QItem it = decode_q(P, i);
+      const int q0 = it.qt * TQ;
+      const int q = q0 + row;
+      const bool valid = q < P.T;
+      const int64_t tok = (int64_t)it.b * P.T + q;
+      const float lse = valid ? P.lse[(int64_t)it.s * P.M + tok] : 0.f;
+      const float dsum = valid ? P.dsum[(int64_t)it.s * P.M + tok] : 0.f;
+      const int lim = !valid ? 0 : (P.causal ? q + 1 : P.T);  // keys < lim are live
+      bool ok = true;
+      for (int j = 0; j < it.nk; ++j) {
+        if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_sdp;
+        tc_fence_after();
+        const int kv0 = j * TK;
+        uint32_t pk[64];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64], dr[64];
+          tmem_ld64_wait(t_base + Q_S + h * 64, sr);
+          tmem_ld64_wait(t_base + Q_DP + h * 64, dr);
+          if (h == 1 && j + 1 < it.nk) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sh.s_free);
+          }
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int c = h * 64 + 2 * x;
+            float d0 = 0.f, d1 = 0.f;
+            if (kv0 + c < lim) {
+              const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
+              d0 = p * (__uint_as_float(dr[2 * x]) - dsum);
+            }
+            if (kv0 + c + 1 < lim) {
+              const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
+              d1 = p * (__uint_as_float(dr[2 * x + 1]) - dsum);
+            }
+            pk[h * 32 + x] = pack_bf16x2(d0, d1);
+          }
+        }
+        // the previous dQ product has read dS: it may be overwritten
+        if (n_ds > 0 && !warp_wait(sh.d_free, (n_ds - 1) & 1, P, sh.abort_flag)) {
+          ok = false;
+          break;
+        }
+        ++n_ds;
+        store_packed64(t_base + Q_DS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.d_ready);
+      }
+      if (!ok) break;
+      // epilogue: dQ / sqrt(d_h) into its destination row
+      if (!warp_wait(sh.acc_full, n_acc & 1, P, sh.abort_flag)) break;
+      ++n_acc;
+      tc_fence_after();
+      __nv_bfloat16* dst = nullptr;
+      if (valid) {
+        if (it.s < P.Sr) {
+          const int g = it.s / P.k;
+          const int e = g * P.E + P.sel[tok * (int64_t)P.Sr + it.s];
+          dst = P.dq_exp + tok * (int64_t)P.N * DH + (int64_t)e * DH;
+        } else {
+          dst = P.dq_sh + tok * DH;
+        }
+      }
+#pragma unroll
+      for (int c0 = 0; c0 < DH; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16_wait(t_base + Q_DQ + c0, r);
+        if (valid) {
+          uint4 v0, v1;
+          const float sc = P.scale;
+          v0.x = pack_bf16x2(__uint_as_float(r[0]) * sc, __uint_as_float(r[1]) * sc);
+          v0.y = pack_bf16x2(__uint_as_float(r[2]) * sc, __uint_as_float(r[3]) * sc);
+          v0.z = pack_bf16x2(__uint_as_float(r[4]) * sc, __uint_as_float(r[5]) * sc);
+          v0.w = pack_bf16x2(__uint_as_float(r[6]) * sc, __uint_as_float(r[7]) * sc);
+          v1.x = pack_bf16x2(__uint_as_float(r[8]) * sc, __uint_as_float(r[9]) * sc);
+          v1.y = pack_bf16x2(__uint_as_float(r[10]) * sc, __uint_as_float(r[11]) * sc);
+          v1.z = pack_bf16x2(__uint_as_float(r[12]) * sc, __uint_as_float(r[13]) * sc);
+          v1.w = pack_bf16x2(__uint_as_float(r[14]) * sc, __uint_as_float(r[15]) * sc);
+          *reinterpret_cast<uint4*>(dst + c0) = v0;
+          *reinterpret_cast<uint4*>(dst + c0 + 8) = v1;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sh.acc_free);
+    }
+  }
+  finish(P, tmem, warp);
+}
+
+// ---------------------------------------------------------------------------------------
+// dK, dV: item (b, KV head g, key tile), first key tiles first when causal (they meet the
+// most query tiles). Jobs of an item: every (stream reading g, query tile at or after the
+// key tile when causal).
+// ---------------------------------------------------------------------------------------
+struct KItem {
+  int b, g, kt, ns, qt0, nj;
+};
+__device__ __forceinline__ KItem decode_k(const BwdParams& P, int i) {
+  KItem it;
+  const int bg = P.B * P.G;
+  it.kt = i / bg;
+  const int r = i % bg;
+  it.g = r % P.G;
+  it.b = r / P.G;
+  it.ns = P.k + ((it.g == 0 && P.has_shared) ? 1 : 0);
+  it.qt0 = P.causal ? it.kt : 0;
+  it.nj = it.ns * (P.nq - it.qt0);
+  return it;
+}
+__device__ __forceinline__ void job_of(const BwdParams& P, const KItem& it, int j, int& s,
+                                       int& qt) {
+  const int per = P.nq - it.qt0;
+  const int si = j / per;
+  qt = it.qt0 + j % per;
+  s = si < P.k ? it.g * P.k + si : P.Sr;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
+  using C = BCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t *sK, *sV, *sQ, *sdO;
+  const Shared sh = carve<DH>(smem, sK, sV, sQ, sdO);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) init_shared(sh, C::STAGES);
+  if (warp == 1) {
+    tmem_alloc(sh.tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&P.tm_q);
+    prefetch_tmap(&P.tm_k);
+    prefetch_tmap(&P.tm_v);
+    prefetch_tmap(&P.tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sh.tmem_holder;
+  pdl_wait();
+  pdl_allow_next();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ loads
+    if (lane == 0) {
+      int st = 0, islot = 0;
+      uint32_t r_phase = 0, q_phase = 0, iphase = 0;
+      while (!*sh.abort_flag) {
+        int i;
+        if (!publish_item(sh, P, islot, iphase, i) || i < 0) break;
+        const KItem it = decode_k(P, i);
+        if (!lane_wait(sh.q_empty, q_phase ^ 1, P, sh.abort_flag)) break;
+        q_phase ^= 1;
+        mbar_arrive_expect_tx(sh.q_full, 2 * C::TILE_BYTES);
+        const int krow = it.g * P.M + it.b * P.T + it.kt * TK;
+        load_tile<DH>(P, &P.tm_k, sK, krow, sh.q_full);
+        load_tile<DH>(P, &P.tm_v, sV, krow, sh.q_full);
+        for (int j = 0; j < it.nj; ++j) {
+          int s, qt;
+          job_of(P, it, j, s, qt);
+          if (!lane_wait(&sh.r_empty[st], r_phase ^ 1, P, sh.abort_flag)) break;
+          mbar_arrive_expect_tx(&sh.r_full[st], 2 * C::TILE_BYTES);
+          const int qrow = s * P.M + it.b * P.T + qt * TQ;
+          load_tile<DH>(P, &P.tm_q, sQ + st * C::TILE_BYTES, qrow, &sh.r_full[st]);
+          load_tile<DH>(P, &P.tm_do, sdO + st * C::TILE_BYTES, qrow, &sh.r_full[st]);
+          if (++st == C::STAGES) {
+            st = 0;
+            r_phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issue
+    const uint32_t idesc_s = idesc_bf16_f32(TK, TQ);
+    const uint32_t idesc_kv = idesc_bf16_f32(TK, DH) | (1u << 16);  // B (Q, dO) MN-major
+    const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t v_desc = smem_desc(smem_u32(sV), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t do_desc = smem_desc(smem_u32(sdO), 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t qmn_desc =
+        smem_desc_mn(smem_u32(sQ), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    const uint64_t domn_desc =
+        smem_desc_mn(smem_u32(sdO), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kStep = C::TILE_BYTES >> 4;
+    int st = 0, islot = 0;
+    uint32_t r_phase = 0, q_phase = 0, iphase = 0;
+    uint32_t n_sf = 0, n_dr = 0, n_items = 0;
+    bool ok = true;
+    // S^T = K Q^T and dP^T = V dO^T of the next job
+    auto issue_sdp = [&](int stage, uint32_t phase) -> bool {
+      if (!warp_wait(&sh.r_full[stage], phase, P, sh.abort_flag)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t qd = q_desc + (uint64_t)(stage * kStep);
+        const uint64_t dd = do_desc + (uint64_t)(stage * kStep);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t o = kmajor_off<DH>(kk);
+          mma_ss(tmem + K_S, k_desc + o, qd + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t o = kmajor_off<DH>(kk);
+          mma_ss(tmem + K_DP, v_desc + o, dd + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(sh.sdp_full);
+      }
+      __syncwarp();
+      return true;
+    };
+    while (ok && !*sh.abort_flag) {
+      int i;
+      if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
+      const KItem it = decode_k(P, i);
+      if (!warp_wait(sh.q_full, q_phase, P, sh.abort_flag)) break;
+      q_phase ^= 1;
+      int st_next = st;
+      uint32_t ph_next = r_phase;
+      if (!issue_sdp(st_next, ph_next)) break;
+      for (int j = 0; j < it.nj; ++j) {
+        const int st_j = st_next;
+        if (++st_next == C::STAGES) {
+          st_next = 0;
+          ph_next ^= 1;
+        }
+        if (j + 1 < it.nj) {
+          if (!warp_wait(sh.s_free, n_sf & 1, P, sh.abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!issue_sdp(st_next, ph_next)) { ok = false; break; }
+        }
+        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_dr;
+        if (j == 0 && n_items > 0 &&
+            !warp_wait(sh.acc_free, (n_items - 1) & 1, P, sh.abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t dd = domn_desc + (uint64_t)(st_j * kStep);
+          const uint64_t qd = qmn_desc + (uint64_t)(st_j * kStep);
+          // dV (+)= P^T dO and dK (+)= dS^T Q: A from TMEM (keys x queries), B = dO / Q
+          // tile (N = head dim, K = queries; MN-major)
+#pragma unroll
+          for (int kk = 0; kk < TQ / 16; ++kk)
+            mma_ts(tmem + K_DV, tmem + K_P + kk * 8,
+                   dd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
+                   (j == 0 && kk == 0) ? 0u : 1u);
+#pragma unroll
+          for (int kk = 0; kk < TQ / 16; ++kk)
+            mma_ts(tmem + K_DK, tmem + K_DS + kk * 8,
+                   qd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
+                   (j == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&sh.r_empty[st_j]);
+          mma_commit(sh.d_free);
+          if (j + 1 == it.nj) {
+            mma_commit(sh.acc_full);
+            mma_commit(sh.q_empty);
+          }
+        }
+        __syncwarp();
+      }
+      st = st_next;
+      r_phase = ph_next;
+      ++n_items;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row of the tile (TMEM lane)
+    const int tid = threadIdx.x - 128;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t t_base = tmem + lane_off;
+    uint32_t n_sdp = 0, n_pd = 0, n_acc = 0, n_job = 0;
+    int islot = 0;
+    uint32_t iphase = 0;
+    const float c2 = P.scale_log2;
+    while (!*sh.abort_flag) {
+      int i;
+      if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
+      const KItem it = decode_k(P, i);
+      const int u = it.kt * TK + row;  // key position
+      const bool key_ok = u < P.T;
+      bool ok = true;
+      for (int j = 0; j < it.nj; ++j, ++n_job) {
+        int s, qt;
+        job_of(P, it, j, s, qt);
+        // the job's per-query lse and D, one per thread, into this job's buffer; the
+        // buffer's barrier completes when all 128 threads have written (a bounded wait)
+        const int buf = n_job & 1;
+        float* sL = sh.sL + buf * 128;
+        float* sD = sh.sD + buf * 128;
+        {
+          const int qq = qt * TQ + tid;
+          const bool qv = qq < P.T;
+          const int64_t idx = (int64_t)s * P.M + (int64_t)it.b * P.T + qq;
+          sL[tid] = qv ? P.lse[idx] : 0.f;
+          sD[tid] = qv ? P.dsum[idx] : 0.f;
+        }
+        mbar_arrive(&sh.l_bar[buf]);
+        if (!warp_wait(&sh.l_bar[buf], (n_job >> 1) & 1, P, sh.abort_flag)) { ok = false; break; }
+        if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_sdp;
+        tc_fence_after();
+        const int q0 = qt * TQ;
+        // live queries of this key: q < T, and q >= u when causal
+        const int qlo = P.causal ? u : 0;
+        uint32_t pp[32], pd[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64], dr[64];
+          tmem_ld64_wait(t_base + K_S + h * 64, sr);
+          tmem_ld64_wait(t_base + K_DP + h * 64, dr);
+          if (h == 1) {
+            if (j + 1 < it.nj) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(sh.s_free);
+            }
+            // the first half goes to TMEM once the previous job's products have read it
+            if (n_pd > 0 && !warp_wait(sh.d_free, (n_pd - 1) & 1, P, sh.abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++n_pd;
+            store_packed32(t_base + K_P, pp);
+            store_packed32(t_base + K_DS, pd);
+          }
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int c = h * 64 + 2 * x;
+            float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+            const int qa = q0 + c, qb = q0 + c + 1;
+            if (key_ok && qa < P.T && qa >= qlo) {
+              p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -sL[c]));
+              d0 = p0 * (__uint_as_float(dr[2 * x]) - sD[c]);
+            }
+            if (key_ok && qb < P.T && qb >= qlo) {
+              p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -sL[c + 1]));
+              d1 = p1 * (__uint_as_float(dr[2 * x + 1]) - sD[c + 1]);
+            }
+            pp[x] = pack_bf16x2(p0, p1);
+            pd[x] = pack_bf16x2(d0, d1);
+          }
+        }
+        if (!ok) break;
+        store_packed32(t_base + K_P + 32, pp);
+        store_packed32(t_base + K_DS + 32, pd);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.d_ready);
+      }
+      if (!ok) break;
+      // epilogue: dK / sqrt(d_h) and dV into their token-major rows
+      if (!warp_wait(sh.acc_full, n_acc & 1, P, sh.abort_flag)) break;
+      ++n_acc;
+      tc_fence_after();
+      const int64_t tok = (int64_t)it.b * P.T + u;
+      const int64_t off = tok * (int64_t)P.G * DH + (int64_t)it.g * DH;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? P.dk : P.dv) + off;
+        const float sc = which == 0 ? P.scale : 1.f;
+        const uint32_t col = which == 0 ? K_DK : K_DV;
+#pragma unroll
+        for (int c0 = 0; c0 < DH; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16_wait(t_base + col + c0, r);
+          if (key_ok) {
+            uint4 v0, v1;
+            v0.x = pack_bf16x2(__uint_as_float(r[0]) * sc, __uint_as_float(r[1]) * sc);
+            v0.y = pack_bf16x2(__uint_as_float(r[2]) * sc, __uint_as_float(r[3]) * sc);
+            v0.z = pack_bf16x2(__uint_as_float(r[4]) * sc, __uint_as_float(r[5]) * sc);
+            v0.w = pack_bf16x2(__uint_as_float(r[6]) * sc, __uint_as_float(r[7]) * sc);
+            v1.x = pack_bf16x2(__uint_as_float(r[8]) * sc, __uint_as_float(r[9]) * sc);
+            v1.y = pack_bf16x2(__uint_as_float(r[10]) * sc, __uint_as_float(r[11]) * sc);
+            v1.z = pack_bf16x2(__uint_as_float(r[12]) * sc, __uint_as_float(r[13]) * sc);
+            v1.w = pack_bf16x2(__uint_as_float(r[14]) * sc, __uint_as_float(r[15]) * sc);
+            *reinterpret_cast<uint4*>(dst + c0) = v0;
+            *reinterpret_cast<uint4*>(dst + c0 + 8) = v1;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sh.acc_free);
+    }
+  }
+  finish(P, tmem, warp);
+}
+
+template <int DH>
+int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has_shared,
+                  int causal, cudaStream_t st) {
+  using C = BCfg<DH>;
+  if (!set_smem_limit_once<attn_bwd_dq_kernel<DH>>(C::SMEM)) return -1;
+  if (!set_smem_limit_once<attn_bwd_dkdv_kernel<DH>>(C::SMEM)) return -1;
+  const int M = B * T;
+  BwdParams P;
+  memset(&P, 0, sizeof(P));
+  const CUtensorMapSwizzle sw = C::CW == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B;
+  P.chunked = C::NC > 1 &&
+              tmap_bf16_chunked(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw);
+  if (!P.chunked &&
+      (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw)))
+    return -1;
+  P.lse = h->ws.lse;
+  P.dsum = bb.dsum;
+  P.sel = h->ws.sel;
+  P.dq_exp = bb.dq_exp;
+  P.dq_sh = bb.dq_sh;
+  P.dk = bb.dk;
+  P.dv = bb.dv;
+  P.M = M;
+  P.T = T;
+  P.B = B;
+  P.S = S;
+  P.Sr = h->G * h->k;
+  P.k = h->k;
+  P.G = h->G;
+  P.E = h->E;
+  P.N = h->N;
+  P.has_shared = has_shared;
+  P.causal = causal;
+  P.nq = (T + TQ - 1) / TQ;
+  P.scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
+  P.scale = 1.f / sqrtf((float)DH);
+  P.status = h->ws.status;
+  P.spin = h->spin_limit > 0 ? h->spin_limit : (int64_t)1 << 22;
+  P.counter = bb.counter;
+  // dQ
+  P.items = B * S * P.nq;
+  int grid = P.items < h->num_sms ? P.items : h->num_sms;
+  if (launch_pdl(attn_bwd_dq_kernel<DH>, dim3(grid), dim3(THREADS), C::SMEM, st, P) !=
+      cudaSuccess)
+    return -1;
+  // dK, dV
+  P.items = B * h->G * P.nq;
+  P.counter = bb.counter + 2;
+  grid = P.items < h->num_sms ? P.items : h->num_sms;
+  if (launch_pdl(attn_bwd_dkdv_kernel<DH>, dim3(grid), dim3(THREADS), C::SMEM, st, P) !=
+      cudaSuccess)
+    return -1;
+  return 2;
+}
+
+}  // namespace
+
+bool tc_backward_supported(const gqe_ctx* h) {
+  return h->dtype == GQE_BF16 && h->d_h <= 64;
+}
+
+int launch_tc_attention_backward(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S,
+                                 int has_shared, int causal, cudaStream_t st) {
+  switch (h->d_h) {
+    case 16: return launch_bwd_dh<16>(h, bb, B, T, S, has_shared, causal, st);
+    case 32: return launch_bwd_dh<32>(h, bb, B, T, S, has_shared, causal, st);
+    case 48: return launch_bwd_dh<48>(h, bb, B, T, S, has_shared, causal, st);
+    case 64: return launch_bwd_dh<64>(h, bb, B, T, S, has_shared, causal, st);
+    default: return -1;
+  }
+}
+
+}  // namespace gqe

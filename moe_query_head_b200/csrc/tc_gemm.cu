@@ -121,6 +121,10 @@ struct Params {
   const int32_t* rc;
   const unsigned long long* rpsum;      // probability sums, fixed point
   int nexp;
+  // experts whose buckets this projection computes: [e_lo, e_hi) (a group range of the
+  // layer, see gqe_set_group_range); W_q holds their rows only and their query streams
+  // are numbered from the range's first group
+  int e_lo, e_hi;
   StatsOut so;
   __nv_bfloat16* Q;                     // query streams [S, M, d_h]
   // dense projection with routing (the ROUTE instance): problem 0 = W_r
@@ -371,7 +375,7 @@ __device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0) {
     int nt = 0;
     for (int x = 0; x < N; ++x) {
       s_t0[x] = nt;
-      nt += (s_cnt[x] + BM - 1) / BM;
+      if (x >= P.e_lo && x < P.e_hi) nt += (s_cnt[x] + BM - 1) / BM;
     }
     s_t0[N] = nt;
   }
@@ -562,8 +566,8 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
           }
           if (elect_one()) {
             mbar_arrive_expect_tx(&full[stage], b_bytes);
-            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK, e * P.d_h,
-                        &full[stage]);
+            tma_load_2d(sB + stage * B_STAGE_BYTES, &P.tmap_b[0], kb * BK,
+                        (e - P.e_lo) * P.d_h, &full[stage]);
           }
           const uint32_t dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const int kcol = kb * BK + c * 8;
@@ -670,7 +674,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       if constexpr (GATHER) {
         __nv_bfloat16* dst = nullptr;
         if (valid) {
-          const int g = ti.p / P.E;
+          const int g = (ti.p - P.e_lo) / P.E;  // the group within the range
           const int64_t s = (int64_t)g * P.k + min(ent & 7, P.k - 1);
           dst = P.Q + (s * P.M + min(ent >> 3, P.M - 1)) * P.d_h;
         }
@@ -866,7 +870,7 @@ bool tc_dense_routes(const gqe_ctx* h) { return h->N <= 32 && (h->N & (h->N - 1)
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
                          const void* W_v, const void* W_shared, int route_set,
                          cudaStream_t st) {
-  const int d_h = h->d_h, G = h->G, dim = h->dim;
+  const int d_h = h->d_h, G = h->g1 - h->g0, dim = h->dim;  // this handle's KV heads
   const int S = G * h->k + (W_shared ? 1 : 0);
   Params P;
   memset(&P, 0, sizeof(P));
@@ -896,7 +900,7 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   P.col_major = 1;
   P.status = h->ws.status;
   P.spin = spin_limit(h);
-  P.G = G;
+  P.G = h->G;  // routing covers every group
   P.k = h->k;
   const Workspace& w = h->ws;
   const int cur = route_set & 1, other = cur ^ 1;
@@ -918,8 +922,10 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route
   if (!tmap_bf16_2d(&P.tmap_a, x, h->dim, M, h->dim, BK, 1, CU_TENSOR_MAP_SWIZZLE_128B))
     return -1;
   P.prob[0] = make_problem(h->d_h, OutMap{});
-  if (!tmap_bf16_2d(&P.tmap_b[0], W_q, h->dim, (uint64_t)h->N * h->d_h, h->dim, BK,
-                    P.prob[0].box_n, CU_TENSOR_MAP_SWIZZLE_128B))
+  P.e_lo = h->g0 * h->E;
+  P.e_hi = h->g1 * h->E;
+  if (!tmap_bf16_2d(&P.tmap_b[0], W_q, h->dim, (uint64_t)(P.e_hi - P.e_lo) * h->d_h, h->dim,
+                    BK, P.prob[0].box_n, CU_TENSOR_MAP_SWIZZLE_128B))
     return -1;
   P.nprob = 1;
   P.M = M;

@@ -24,7 +24,8 @@ EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_check_device_status", "gqe_set_spin_limit", "gqe_destroy", "gqe_status_str",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
             "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma", "gqe_selftest_timeout",
-            "gqe_decode")
+            "gqe_decode", "gqe_enable_backward", "gqe_backward", "gqe_backward_launches",
+            "gqe_set_group_range")
 GQE_NUM_STAGES = 6
 
 
@@ -73,6 +74,15 @@ def _load() -> ctypes.CDLL:
     lib.gqe_exp2_fma.restype = I
     lib.gqe_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     lib.gqe_selftest_timeout.restype = I
+    lib.gqe_set_group_range.argtypes = [P, I, I]
+    lib.gqe_set_group_range.restype = I
+    lib.gqe_enable_backward.argtypes = [P]
+    lib.gqe_enable_backward.restype = I
+    lib.gqe_backward.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P,
+                                 ctypes.c_float, P, P, P, P, P, P, P, P]
+    lib.gqe_backward.restype = I
+    lib.gqe_backward_launches.argtypes = [P]
+    lib.gqe_backward_launches.restype = I
     return lib
 
 
@@ -122,6 +132,31 @@ def gqe_decode(h, x, B, k_cache, v_cache, L_max, lengths, W_r, W_q, W_k, W_v, W_
                           _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(W_shared), _ptr(W_o),
                           N, G, k, d_h, variant, _ptr(out), _ptr(aux_loss), _stream(stream)),
            "gqe_decode")
+
+
+def gqe_set_group_range(h, g0: int, g1: int) -> None:
+    """Restricts the handle to groups g0 .. g1-1 of the layer (see include/gqe.h)."""
+    _check(lib.gqe_set_group_range(h, int(g0), int(g1)), "gqe_set_group_range")
+
+
+def gqe_enable_backward(h) -> None:
+    """Allocates the handle's backward workspace (see include/gqe.h)."""
+    _check(lib.gqe_enable_backward(h), "gqe_enable_backward")
+
+
+def gqe_backward(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, variant, causal,
+                 dy, aux_grad, dx, dW_r, dW_q, dW_k, dW_v, dW_shared, dW_o, stream=None) -> None:
+    """Gradients of <dy, y> + aux_grad * aux_loss of the handle's last gqe_forward (same
+    arguments); every gradient is a float32 device tensor (see include/gqe.h)."""
+    _check(lib.gqe_backward(h, _ptr(x), B, T, _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v),
+                            _ptr(W_shared), _ptr(W_o), N, G, k, d_h, variant, causal, _ptr(dy),
+                            float(aux_grad), _ptr(dx), _ptr(dW_r), _ptr(dW_q), _ptr(dW_k),
+                            _ptr(dW_v), _ptr(dW_shared), _ptr(dW_o), _stream(stream)),
+           "gqe_backward")
+
+
+def gqe_backward_launches(h) -> int:
+    return int(lib.gqe_backward_launches(h))
 
 
 def gqe_get_routing(h, sel=None, gates=None, counts=None, mean_prob=None, stream=None) -> None:

@@ -1,0 +1,112 @@
+"""Group-parallel execution of one GQE layer over several GPUs (one process per GPU).
+
+Routing is per group ("GQE: Grouped Query Experts" README, Algorithm Overview: a softmax
+over the experts of each group, then top-k), and each group has its own dense KV head, so
+the layer splits by groups: rank r computes groups [g0, g1) (its KV heads, its experts'
+query heads, their attention and their share of the output projection) and the layer's
+output is the sum of the ranks' shares: one all-reduce (or reduce-scatter) of y. Every rank
+routes every group (the router is N x dim, tiny), so the renormalised slot weights, which
+divide by the selected probabilities of all groups, and the load-balancing loss are the
+whole layer's on every rank with no exchange. The shared head reads KV head 0 and runs on
+the rank that holds group 0.
+
+This module holds the host-side plan (which groups, which weight rows and columns each rank
+takes) and a runner that calls the C ABI's gqe_set_group_range / gqe_forward and sums the
+shares with torch.distributed (NCCL on GPUs).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def group_ranges(G: int, world: int) -> list[tuple[int, int]]:
+    """Contiguous group ranges, one per rank, sizes differing by at most one (the first
+    G % world ranks take one more). Needs 1 <= world <= G."""
+    if not 1 <= world <= G:
+        raise ValueError("need 1 <= world <= G")
+    base, extra = divmod(G, world)
+    out, g = [], 0
+    for r in range(world):
+        n = base + (1 if r < extra else 0)
+        out.append((g, g + n))
+        g += n
+    return out
+
+
+def z_columns(G: int, k: int, d_h: int, variant: str, shared: bool, g0: int, g1: int) -> np.ndarray:
+    """Columns of the layer's Z (and of W_o) that the range [g0, g1) produces, in the order
+    of its own Z: its routed streams (g*k + r for g in the range), the slot (variant gqe:
+    every rank adds its streams' share of the one slot), the shared block (the rank with
+    g0 == 0)."""
+    blocks = list(range(g0 * k, g1 * k))
+    nxt = G * k
+    if variant == "gqe":
+        blocks.append(nxt)
+        nxt += 1
+    if shared and g0 == 0:
+        blocks.append(nxt)
+    return np.concatenate([np.arange(b * d_h, (b + 1) * d_h) for b in blocks])
+
+
+def rank_weights(W_q, W_k, W_v, W_shared, W_o, *, N: int, G: int, k: int, d_h: int,
+                 variant: str, g0: int, g1: int) -> dict:
+    """The weights a rank passes to gqe_forward after gqe_set_group_range(g0, g1): W_q rows
+    of its experts, W_k / W_v rows of its heads, W_shared on the rank with group 0 only, the
+    W_o columns of its Z blocks. Works on numpy arrays and torch tensors (contiguous copies)."""
+    E = N // G
+    cols = z_columns(G, k, d_h, variant, W_shared is not None, g0, g1)
+
+    def rows(a, lo, hi):
+        r = a[lo:hi]
+        return r.contiguous() if hasattr(r, "contiguous") else np.ascontiguousarray(r)
+
+    if hasattr(W_o, "index_select"):
+        import torch
+        Wo = W_o.index_select(1, torch.as_tensor(cols, device=W_o.device)).contiguous()
+    else:
+        Wo = np.ascontiguousarray(W_o[:, cols])
+    return {
+        "W_q": rows(W_q, g0 * E * d_h, g1 * E * d_h),
+        "W_k": rows(W_k, g0 * d_h, g1 * d_h),
+        "W_v": rows(W_v, g0 * d_h, g1 * d_h),
+        "W_shared": W_shared if g0 == 0 else None,
+        "W_o": Wo,
+    }
+
+
+class GroupShard:
+    """One rank's share of a GQE layer on the current CUDA device: a handle restricted to
+    groups [g0, g1) and the rank's weight slices. forward() returns the rank's share of y;
+    forward_allreduce() sums the shares over the process group."""
+
+    def __init__(self, *, dim, N, G, k, d_h, variant, causal, max_tokens, g0, g1, W_r, W_q,
+                 W_k, W_v, W_shared, W_o):
+        import torch
+        from . import gqe as GQ
+        self.GQ = GQ
+        self.dim, self.N, self.G, self.k, self.d_h = dim, N, G, k, d_h
+        self.variant, self.causal = variant, causal
+        self.h = GQ.gqe_create(dim, N, G, k, d_h, GQ.GQE_BF16, max_tokens)
+        GQ.gqe_set_group_range(self.h, g0, g1)
+        self.W_r = W_r
+        self.w = rank_weights(W_q, W_k, W_v, W_shared, W_o, N=N, G=G, k=k, d_h=d_h,
+                              variant=variant, g0=g0, g1=g1)
+        self.aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    def forward(self, x, B, T, out, stream=None):
+        from .workloads import VARIANT_IDS
+        w = self.w
+        self.GQ.gqe_forward(self.h, x, B, T, self.W_r, w["W_q"], w["W_k"], w["W_v"],
+                            w["W_shared"], w["W_o"], self.N, self.G, self.k, self.d_h,
+                            VARIANT_IDS[self.variant], int(self.causal), out, self.aux, stream)
+        return out
+
+    def forward_allreduce(self, x, B, T, out, dist, group=None):
+        self.forward(x, B, T, out)
+        dist.all_reduce(out, group=group)
+        return out
+
+    def close(self):
+        if self.h:
+            self.GQ.gqe_destroy(self.h)
+            self.h = None

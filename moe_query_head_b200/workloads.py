@@ -275,6 +275,13 @@ def router_logits_input(M: int, N: int, G: int, k: int, seed: int,
     raise RuntimeError("margin filter did not converge")
 
 
+def grad_output(wl: Workload, seed_offset: int = 0) -> np.ndarray:
+    """An upstream gradient dy [M, dim] for the backward pass: N(0, 1) from
+    PCG64([seed, 4 + seed_offset]), rounded to the workload's dtype."""
+    rng = np.random.Generator(np.random.PCG64([wl.seed, 4 + seed_offset]))
+    return quantize(rng.standard_normal((wl.M, wl.dim)), wl.dtype)
+
+
 @dataclass
 class DecodeInputs:
     """One decode step's inputs: `inp` holds the B new tokens (x [B, dim], one per
