@@ -46,6 +46,7 @@ from moe_query_head_b200 import workloads as W  # noqa: E402
 
 METRIC = "GQE prefill tokens/s @1 B200; % bf16 tensor peak (active FLOPs); speedup vs k=E"
 DECODE_METRIC = "GQE decode tokens/s @1 B200 (one new token per sequence over its KV cache)"
+BACKWARD_METRIC = "GQE training-step tokens/s @1 B200 (layer forward + backward)"
 DECODE_BASE = "main_b8_t2048"  # the paper's layer shapes: dim 768, N 16, G 8, k 1, d_h 48
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
@@ -61,11 +62,15 @@ def parse_args():
     ap.add_argument("--variant", default=None, choices=["gqe", "weighted_concat", "hard_concat"],
                     help="output construction (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"],
-                    help="prefill (default, the headline) or one decode step with a KV cache")
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode", "backward"],
+                    help="prefill (default, the headline), one decode step with a KV cache, "
+                         "or a training step of the layer (forward + backward)")
     ap.add_argument("--decode-batch", type=int, default=64, help="decode: sequences per step")
     ap.add_argument("--decode-len", type=int, default=8192,
                     help="decode: tokens already cached per sequence")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "groups"],
+                    help="N > 1: independent replicas (default, weak scaling) or one layer "
+                         "split by groups over the ranks with an all-reduce of y (strong)")
     ap.add_argument("--cpu-rows", type=int, default=2048,
                     help="query rows in the oracle's bounded sample")
     a = ap.parse_args()
@@ -645,6 +650,195 @@ def bench_decode(args, rank, world, dist):
     return res, wl
 
 
+# ----------------------------------------------------------------------------------------
+# Backward mode: one training step of the layer (gqe_forward + gqe_backward).
+# ----------------------------------------------------------------------------------------
+
+def backward_flops(wl) -> dict:
+    """Algorithmic FLOPs (2 per multiply-add) of the backward pass: attention 2.5 times the
+    forward's (dV = P^T dO, dP = dO V^T, dQ = dS K, dK = dS^T Q against the forward's two
+    products), and every projection's two gradient GEMMs (weights and input) at its active
+    size."""
+    M, d, h = wl.M, wl.dim, wl.d_h
+    S = wl.n_streams
+    att_fwd = (2.0 * wl.B * h * wl.T * (wl.T + 1) * S if wl.causal
+               else 4.0 * wl.B * h * wl.T * wl.T * S)
+    proj = 2.0 * (2.0 * M * d * (wl.N + (2 * wl.G + (1 if wl.shared else 0)) * h
+                                 + h * wl.G * wl.k) + 2.0 * M * wl.D_o * d)
+    return {"attention": 2.5 * att_fwd, "projections": proj, "total": 2.5 * att_fwd + proj}
+
+
+def bench_backward(args, rank, world, dist):
+    import torch
+    from moe_query_head_b200 import gqe as G
+
+    wl = W.WORKLOADS[args.workload]
+    if args.variant:
+        wl = wl.with_(variant=args.variant)
+    inp = W.generate(wl)
+    dev = _upload(inp, torch)
+    variant = W.VARIANT_IDS[wl.variant]
+    W_s = dev["W_shared"] if wl.shared else None
+    h = G.gqe_create(wl.dim, wl.N, wl.G, wl.k, wl.d_h, G.GQE_BF16, wl.M)
+    G.gqe_enable_backward(h)
+    out = torch.empty((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+    aux = torch.zeros(1, dtype=torch.float32, device="cuda")
+    dy = torch.from_numpy(W.f32_to_bf16_bits(W.grad_output(wl)).view(np.int16)).view(
+        torch.bfloat16).cuda()
+    f32 = lambda *s: torch.empty(s, dtype=torch.float32, device="cuda")  # noqa: E731
+    g = [f32(wl.M, wl.dim), f32(wl.N, wl.dim), f32(wl.N * wl.d_h, wl.dim),
+         f32(wl.G * wl.d_h, wl.dim), f32(wl.G * wl.d_h, wl.dim),
+         f32(wl.d_h, wl.dim) if wl.shared else None, f32(wl.dim, wl.D_o)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def fwd():
+        G.gqe_forward(h, dev["x"], wl.B, wl.T, dev["W_r"], dev["W_q"], dev["W_k"], dev["W_v"],
+                      W_s, dev["W_o"], wl.N, wl.G, wl.k, wl.d_h, variant, int(wl.causal), out,
+                      aux)
+
+    def bwd():
+        G.gqe_backward(h, dev["x"], wl.B, wl.T, dev["W_r"], dev["W_q"], dev["W_k"], dev["W_v"],
+                       W_s, dev["W_o"], wl.N, wl.G, wl.k, wl.d_h, variant, int(wl.causal), dy,
+                       0.01, *g)
+
+    gpu_id = torch.cuda.get_device_properties(0).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    if G.gqe_check_device_status(h) != G.GQE_OK:
+        raise RuntimeError("device status after warm-up")
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    tot, tf, tb = 0.0, 0.0, 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        ev[0].record()
+        fwd()
+        ev[1].record()
+        bwd()
+        ev[2].record()
+        torch.cuda.synchronize()
+        tf += ev[0].elapsed_time(ev[1])
+        tb += ev[1].elapsed_time(ev[2])
+        tot += ev[0].elapsed_time(ev[2])
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    if G.gqe_check_device_status(h) != G.GQE_OK:
+        raise RuntimeError("device status after timing")
+    launches = G.gqe_kernel_launches(h) + G.gqe_backward_launches(h)
+    if dist:
+        tot, tf, tb = reduce_max_over_ranks([tot, tf, tb], dist, "cuda")
+    peaks, peak_src = load_peaks()
+    ms, msf, msb = tot / args.steps, tf / args.steps, tb / args.steps
+    bf = backward_flops(wl)
+    fflops = wl.active_flops()
+    peak = float(peaks["bf16_tflops"])
+    res = {
+        "metric": BACKWARD_METRIC, "value": wl.M * world / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal inputs, upstream gradient and random-init weights "
+                "of the layer shapes)",
+        "config": dict(prefill_config(wl, world), aux_grad=0.01),
+        "forward_ms": msf, "backward_ms": msb,
+        "active_tflops": (fflops + bf["total"]) / (ms / 1e3) / 1e12,
+        "frac_of_bf16_peak": (fflops + bf["total"]) / (ms / 1e3) / 1e12 / peak,
+        "backward_active_tflops": bf["total"] / (msb / 1e3) / 1e12,
+        "backward_flops": bf,
+        "roofline": {"kernel": "backward pass (all kernels)", "bound": "tensor",
+                     "achieved": bf["total"] / (msb / 1e3) / 1e12, "peak": peak,
+                     "unit": "TFLOP/s", "frac": bf["total"] / (msb / 1e3) / 1e12 / peak,
+                     "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": None},
+        "e2e": None,
+        "gpu_launches": int(launches * args.steps),
+        "clocks": clocks,
+    }
+    G.gqe_destroy(h)
+    return res
+
+
+# ----------------------------------------------------------------------------------------
+# Group-parallel prefill: one layer split by groups over the ranks (strong scaling).
+# ----------------------------------------------------------------------------------------
+
+def bench_groups(args, rank, world, dist):
+    """Rank r computes groups group_ranges(G, world)[r] of the layer (gqe_set_group_range with
+    its weight slices) and the ranks' shares of y are summed by one NCCL all-reduce; a step
+    is the forward of every rank plus the all-reduce, timed on the device, max over ranks."""
+    import torch
+    from moe_query_head_b200 import gqe as G
+    from moe_query_head_b200 import group_parallel as GP
+
+    wl = W.WORKLOADS[args.workload]
+    if args.variant:
+        wl = wl.with_(variant=args.variant)
+    inp = W.generate(wl)
+    dev = _upload(inp, torch)
+    g0, g1 = GP.group_ranges(wl.G, world)[rank]
+    sh = GP.GroupShard(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, variant=wl.variant,
+                       causal=wl.causal, max_tokens=wl.M, g0=g0, g1=g1, W_r=dev["W_r"],
+                       W_q=dev["W_q"], W_k=dev["W_k"], W_v=dev["W_v"],
+                       W_shared=dev["W_shared"] if wl.shared else None, W_o=dev["W_o"])
+    out = torch.empty((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step():
+        sh.forward_allreduce(dev["x"], wl.B, wl.T, out, dist)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if G.gqe_check_device_status(sh.h) != G.GQE_OK:
+        raise RuntimeError("device status after warm-up")
+    gpu_id = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
+    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        s_ev.record()
+        step()
+        e_ev.record()
+        torch.cuda.synchronize()
+        total += s_ev.elapsed_time(e_ev)
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    launches = G.gqe_kernel_launches(sh.h)
+    if dist:
+        (total,) = reduce_max_over_ranks([total], dist, "cuda")
+    peaks, peak_src = load_peaks()
+    ms = total / args.steps
+    peak = float(peaks["bf16_tflops"])
+    flops = wl.active_flops()
+    res = {
+        "metric": METRIC, "value": wl.M / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal inputs and random-init weights of the layer shapes)",
+        "config": dict(prefill_config(wl, world), parallelism=f"groups x{world}"),
+        "active_tflops": flops / (ms / 1e3) / 1e12,
+        "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / peak / world,
+        "roofline": None, "e2e": None,
+        "gpu_launches": int(launches * args.steps), "clocks": clocks,
+    }
+    sh.close()
+    return res
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -716,6 +910,21 @@ def main():
         dist = td
     else:
         torch.cuda.set_device(0)
+    if args.parallel == "groups" and world > 1 and args.mode == "prefill":
+        res = bench_groups(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res))
+        dist.barrier()
+        dist.destroy_process_group()
+        return 0
+    if args.mode == "backward":
+        res = bench_backward(args, rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res))
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
     if args.mode == "decode":
         res, wl = bench_decode(args, rank, world, dist)
         if rank == 0:
