@@ -463,19 +463,30 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.s_free);
           }
+          if (kv0 + TK <= lim) {
+            // every key of the tile is live for this query: no masks
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int c = h * 64 + 2 * x;
-            float d0 = 0.f, d1 = 0.f;
-            if (kv0 + c < lim) {
-              const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
-              d0 = p * (__uint_as_float(dr[2 * x]) - dsum);
+            for (int x = 0; x < 32; ++x) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
+              pk[h * 32 + x] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * x]) - dsum),
+                                           p1 * (__uint_as_float(dr[2 * x + 1]) - dsum));
             }
-            if (kv0 + c + 1 < lim) {
-              const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
-              d1 = p * (__uint_as_float(dr[2 * x + 1]) - dsum);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const int c = h * 64 + 2 * x;
+              float d0 = 0.f, d1 = 0.f;
+              if (kv0 + c < lim) {
+                const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
+                d0 = p * (__uint_as_float(dr[2 * x]) - dsum);
+              }
+              if (kv0 + c + 1 < lim) {
+                const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
+                d1 = p * (__uint_as_float(dr[2 * x + 1]) - dsum);
+              }
+              pk[h * 32 + x] = pack_bf16x2(d0, d1);
             }
-            pk[h * 32 + x] = pack_bf16x2(d0, d1);
           }
         }
         // the previous dQ product has read dS: it may be overwritten
@@ -730,21 +741,28 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
       const int u = it.kt * TK + row;  // key position
       const bool key_ok = u < P.T;
       bool ok = true;
+      // a job's per-query lse and D (one value of each per thread), loaded one job ahead
+      auto fetch = [&](int jj, float& lv, float& dv) {
+        int ss, qq_t;
+        job_of(P, it, jj, ss, qq_t);
+        const int qq = qq_t * TQ + tid;
+        const int64_t idx = (int64_t)ss * P.M + (int64_t)it.b * P.T + qq;
+        lv = qq < P.T ? P.lse[idx] : 0.f;
+        dv = qq < P.T ? P.dsum[idx] : 0.f;
+      };
+      float nl = 0.f, nd = 0.f;
+      fetch(0, nl, nd);
       for (int j = 0; j < it.nj; ++j, ++n_job) {
         int s, qt;
         job_of(P, it, j, s, qt);
-        // the job's per-query lse and D, one per thread, into this job's buffer; the
-        // buffer's barrier completes when all 128 threads have written (a bounded wait)
+        // this job's values into its buffer; the buffer's barrier completes when all 128
+        // threads have written (a bounded wait); the next job's values are requested now
         const int buf = n_job & 1;
         float* sL = sh.sL + buf * 128;
         float* sD = sh.sD + buf * 128;
-        {
-          const int qq = qt * TQ + tid;
-          const bool qv = qq < P.T;
-          const int64_t idx = (int64_t)s * P.M + (int64_t)it.b * P.T + qq;
-          sL[tid] = qv ? P.lse[idx] : 0.f;
-          sD[tid] = qv ? P.dsum[idx] : 0.f;
-        }
+        sL[tid] = nl;
+        sD[tid] = nd;
+        if (j + 1 < it.nj) fetch(j + 1, nl, nd);
         mbar_arrive(&sh.l_bar[buf]);
         if (!warp_wait(&sh.l_bar[buf], (n_job >> 1) & 1, P, sh.abort_flag)) { ok = false; break; }
         if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
@@ -753,6 +771,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
         const int q0 = qt * TQ;
         // live queries of this key: q < T, and q >= u when causal
         const int qlo = P.causal ? u : 0;
+        const bool all_live = key_ok && q0 >= qlo && q0 + TQ <= P.T;
         uint32_t pp[32], pd[32];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -774,21 +793,40 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
             store_packed32(t_base + K_P, pp);
             store_packed32(t_base + K_DS, pd);
           }
+          if (all_live) {
+            // every query of the tile is live for this key: no masks
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int c = h * 64 + 2 * x;
-            float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-            const int qa = q0 + c, qb = q0 + c + 1;
-            if (key_ok && qa < P.T && qa >= qlo) {
-              p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -sL[c]));
-              d0 = p0 * (__uint_as_float(dr[2 * x]) - sD[c]);
+            for (int x4 = 0; x4 < 16; ++x4) {
+              const float4 L4 = reinterpret_cast<const float4*>(sL + h * 64)[x4];
+              const float4 D4 = reinterpret_cast<const float4*>(sD + h * 64)[x4];
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4]), c2, -L4.x));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4 + 1]), c2, -L4.y));
+              const float p2 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4 + 2]), c2, -L4.z));
+              const float p3 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4 + 3]), c2, -L4.w));
+              pp[2 * x4] = pack_bf16x2(p0, p1);
+              pp[2 * x4 + 1] = pack_bf16x2(p2, p3);
+              pd[2 * x4] = pack_bf16x2(p0 * (__uint_as_float(dr[4 * x4]) - D4.x),
+                                       p1 * (__uint_as_float(dr[4 * x4 + 1]) - D4.y));
+              pd[2 * x4 + 1] = pack_bf16x2(p2 * (__uint_as_float(dr[4 * x4 + 2]) - D4.z),
+                                           p3 * (__uint_as_float(dr[4 * x4 + 3]) - D4.w));
             }
-            if (key_ok && qb < P.T && qb >= qlo) {
-              p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -sL[c + 1]));
-              d1 = p1 * (__uint_as_float(dr[2 * x + 1]) - sD[c + 1]);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const int c = h * 64 + 2 * x;
+              float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+              const int qa = q0 + c, qb = q0 + c + 1;
+              if (key_ok && qa < P.T && qa >= qlo) {
+                p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -sL[c]));
+                d0 = p0 * (__uint_as_float(dr[2 * x]) - sD[c]);
+              }
+              if (key_ok && qb < P.T && qb >= qlo) {
+                p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -sL[c + 1]));
+                d1 = p1 * (__uint_as_float(dr[2 * x + 1]) - sD[c + 1]);
+              }
+              pp[x] = pack_bf16x2(p0, p1);
+              pd[x] = pack_bf16x2(d0, d1);
             }
-            pp[x] = pack_bf16x2(p0, p1);
-            pd[x] = pack_bf16x2(d0, d1);
           }
         }
         if (!ok) break;
