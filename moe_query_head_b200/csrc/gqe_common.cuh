@@ -25,7 +25,7 @@ constexpr int kStatusBadInput = 2;  // a decode position outside its cache
 // Partial-result slots of the decode attention: (sequence, group, key chunk) triples whose
 // (m, l, O) are merged by a second kernel. Bounded independently of the cache length (the
 // chunks grow with it), so the handle's workspace holds them.
-constexpr int kDecodeSlots = 1024;
+constexpr int kDecodeSlots = 4096;
 
 // ---------------------------------------------------------------------------------------
 // Programmatic dependent launch. The forward's kernels are launched with it: a kernel may

@@ -71,7 +71,9 @@ constexpr int Q_S = 0, Q_DP = 128, Q_DS = 256, Q_DQ = 320;
 constexpr int K_S = 0, K_DP = 128, K_P = 256, K_DS = 320, K_DV = 384, K_DK = 448;
 
 struct BwdParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO [S M, d_h]; K, V [G M, d_h]
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO [S M, d_h]; K, V [G M, d_h]; 128-row boxes
+  CUtensorMap tm_k64, tm_v64;           // K, V with 64-row boxes (the dQ kernel)
+  CUtensorMap tm_q64, tm_do64;          // Q, dO with 64-row boxes (the dK / dV kernel)
   const float* lse;     // [S, M]
   const float* dsum;    // [S, M] rowsum(dO * O)
   const int32_t* sel;   // [M, G, k]
@@ -79,7 +81,7 @@ struct BwdParams {
   __nv_bfloat16* dq_sh;   // [M, d_h]
   __nv_bfloat16* dk;      // [M, G d_h]
   __nv_bfloat16* dv;      // [M, G d_h]
-  int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, items, chunked;
+  int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, nq64, items, chunked;
   float scale_log2;  // log2(e) / sqrt(d_h)
   float scale;       // 1 / sqrt(d_h)
   int* counter;      // [2] item counter and exit counter (zero at launch; reset by the last CTA)
@@ -110,7 +112,8 @@ __device__ __forceinline__ bool lane_wait(uint64_t* bar, uint32_t parity, const 
   return false;
 }
 
-template <int DH>
+// One tile of ROWS rows (128 or 64): chunk after chunk, each ROWS x CW.
+template <int DH, int ROWS = 128>
 __device__ __forceinline__ void load_tile(const BwdParams& P, const CUtensorMap* map,
                                           uint8_t* dst, int row, uint64_t* bar) {
   using C = BCfg<DH>;
@@ -118,15 +121,17 @@ __device__ __forceinline__ void load_tile(const BwdParams& P, const CUtensorMap*
     tma_load_3d(dst, map, 0, row, 0, bar);
   } else {
 #pragma unroll
-    for (int c = 0; c < C::NC; ++c) tma_load_2d(dst + c * C::CHUNK_BYTES, map, c * C::CW, row, bar);
+    for (int c = 0; c < C::NC; ++c)
+      tma_load_2d(dst + c * ROWS * C::ROW_BYTES, map, c * C::CW, row, bar);
   }
 }
 
-// K-major descriptor offset (16-byte units) of head-dim columns kk*16 .. kk*16+15.
-template <int DH>
+// K-major descriptor offset (16-byte units) of head-dim columns kk*16 .. kk*16+15 in a
+// tile of ROWS rows.
+template <int DH, int ROWS = 128>
 __device__ __forceinline__ uint32_t kmajor_off(int kk) {
   using C = BCfg<DH>;
-  return (((kk * 16) / C::CW) * C::CHUNK_BYTES + ((kk * 16) % C::CW) * 2) >> 4;
+  return (((kk * 16) / C::CW) * ROWS * C::ROW_BYTES + ((kk * 16) % C::CW) * 2) >> 4;
 }
 
 // bf16 pairs of the packed row -> 16 TMEM columns at a time
@@ -170,21 +175,22 @@ struct Shared {
   float* sD;  // [2][128]
 };
 
-template <int DH>
-__device__ __forceinline__ Shared carve(uint8_t* smem, uint8_t*& sFix0, uint8_t*& sFix1,
-                                        uint8_t*& sR0, uint8_t*& sR1) {
-  using C = BCfg<DH>;
+// Shared memory: two fixed tiles of fix_bytes, a ring of `stages` tile pairs of ring_bytes,
+// then the barriers and the lse / D buffers.
+__device__ __forceinline__ Shared carve(uint8_t* smem, int fix_bytes, int ring_bytes, int stages,
+                                        uint8_t*& sFix0, uint8_t*& sFix1, uint8_t*& sR0,
+                                        uint8_t*& sR1) {
   sFix0 = smem;
-  sFix1 = smem + C::TILE_BYTES;
-  sR0 = sFix1 + C::TILE_BYTES;                  // ring: first tile of each pair
-  sR1 = sR0 + C::STAGES * C::TILE_BYTES;        // ring: second tile of each pair
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sR1 + C::STAGES * C::TILE_BYTES);
+  sFix1 = smem + fix_bytes;
+  sR0 = sFix1 + fix_bytes;              // ring: first tile of each pair
+  sR1 = sR0 + stages * ring_bytes;      // ring: second tile of each pair
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sR1 + stages * ring_bytes);
   Shared sh;
   sh.q_full = bar;
   sh.q_empty = bar + 1;
   sh.r_full = bar + 2;
-  sh.r_empty = sh.r_full + C::STAGES;
-  sh.sdp_full = sh.r_empty + C::STAGES;
+  sh.r_empty = sh.r_full + stages;
+  sh.sdp_full = sh.r_empty + stages;
   sh.s_free = sh.sdp_full + 1;
   sh.d_ready = sh.s_free + 1;
   sh.d_free = sh.d_ready + 1;
@@ -251,12 +257,13 @@ __device__ __forceinline__ bool next_item(const Shared& sh, const BwdParams& P, 
   return true;
 }
 
-__device__ __forceinline__ void finish(const BwdParams& P, uint32_t tmem, int warp) {
+__device__ __forceinline__ void finish(const BwdParams& P, uint32_t tmem, int warp,
+                                       uint32_t cols) {
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, cols);
   }
   if (threadIdx.x == 0 && atomicAdd(P.counter + 1, 1) == (int)gridDim.x - 1) {
     P.counter[0] = 0;
@@ -281,24 +288,44 @@ __device__ __forceinline__ QItem decode_q(const BwdParams& P, int i) {
   return it;
 }
 
+// The dQ kernel runs two CTAs per SM with 64-key steps, so that each CTA's TMEM (S, dP,
+// dS, dQ) fits in 256 columns and two softmax warpgroups share an SM; warpgroup 0 (loads,
+// MMA, two idle warps) gives most of its registers to the softmax warpgroup.
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
+struct QCfg {
   using C = BCfg<DH>;
+  static constexpr int TKD = 64;                     // keys per step
+  static constexpr int KT_BYTES = TKD * DH * 2;      // one 64-row K or V tile
+  static constexpr int STAGES = 3;
+  static constexpr int SMEM = 2 * C::TILE_BYTES + STAGES * 2 * KT_BYTES + 1024 + 512 + 2048;
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int S_COL = 0, DP_COL = 64, DS_COL = 128, DQ_COL = 160;
+  static_assert(DQ_COL + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+constexpr int kQSmallRegs = 48, kQLargeRegs = 208;
+static_assert(kQSmallRegs * 128 + kQLargeRegs * 128 == THREADS * (65536 / (2 * THREADS)),
+              "register split must equal the launch allocation");
+
+template <int DH>
+__global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
+  using C = BCfg<DH>;
+  using Q = QCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t *sQ, *sdO, *sK, *sV;
-  const Shared sh = carve<DH>(smem, sQ, sdO, sK, sV);
+  const Shared sh = carve(smem, C::TILE_BYTES, Q::KT_BYTES, Q::STAGES, sQ, sdO, sK, sV);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) init_shared(sh, C::STAGES);
+  if (threadIdx.x == 0) init_shared(sh, Q::STAGES);
   if (warp == 1) {
-    tmem_alloc(sh.tmem_holder, C::TMEM_COLS);
+    tmem_alloc(sh.tmem_holder, Q::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&P.tm_q);
-    prefetch_tmap(&P.tm_k);
-    prefetch_tmap(&P.tm_v);
+    prefetch_tmap(&P.tm_k64);
+    prefetch_tmap(&P.tm_v64);
     prefetch_tmap(&P.tm_do);
   }
   tc_fence_before();
@@ -308,6 +335,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
   pdl_wait();
   pdl_allow_next();
 
+  if (warp < 4) {
+  setmaxnreg_dec<kQSmallRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------------ loads
     if (lane == 0) {
@@ -325,12 +354,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
         load_tile<DH>(P, &P.tm_do, sdO, qrow, sh.q_full);
         const int kvh = it.s < P.Sr ? it.s / P.k : 0;
         const int krow0 = kvh * P.M + it.b * P.T;
-        for (int j = 0; j < it.nk; ++j) {
+        const int nsteps = 2 * it.nk;  // 64-key steps over the item's 128-key tiles
+        for (int j = 0; j < nsteps; ++j) {
           if (!lane_wait(&sh.r_empty[st], r_phase ^ 1, P, sh.abort_flag)) break;
-          mbar_arrive_expect_tx(&sh.r_full[st], 2 * C::TILE_BYTES);
-          load_tile<DH>(P, &P.tm_k, sK + st * C::TILE_BYTES, krow0 + j * TK, &sh.r_full[st]);
-          load_tile<DH>(P, &P.tm_v, sV + st * C::TILE_BYTES, krow0 + j * TK, &sh.r_full[st]);
-          if (++st == C::STAGES) {
+          mbar_arrive_expect_tx(&sh.r_full[st], 2 * Q::KT_BYTES);
+          load_tile<DH, Q::TKD>(P, &P.tm_k64, sK + st * Q::KT_BYTES, krow0 + j * Q::TKD,
+                                &sh.r_full[st]);
+          load_tile<DH, Q::TKD>(P, &P.tm_v64, sV + st * Q::KT_BYTES, krow0 + j * Q::TKD,
+                                &sh.r_full[st]);
+          if (++st == Q::STAGES) {
             st = 0;
             r_phase ^= 1;
           }
@@ -339,20 +371,21 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issue
-    const uint32_t idesc_s = idesc_bf16_f32(TQ, TK);
+    const uint32_t idesc_s = idesc_bf16_f32(TQ, Q::TKD);
     const uint32_t idesc_dq = idesc_bf16_f32(TQ, DH) | (1u << 16);  // B (K) MN-major
     const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t do_desc = smem_desc(smem_u32(sdO), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t v_desc = smem_desc(smem_u32(sV), 8 * C::ROW_BYTES, C::LAYOUT);
+    // K as the MN-major B operand of dQ: 64-row chunks
     const uint64_t kmn_desc =
-        smem_desc_mn(smem_u32(sK), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
-    constexpr uint32_t kStep = C::TILE_BYTES >> 4;
+        smem_desc_mn(smem_u32(sK), Q::TKD * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kStep = Q::KT_BYTES >> 4;
     int st = 0, islot = 0;
     uint32_t r_phase = 0, q_phase = 0, iphase = 0;
     uint32_t n_sf = 0, n_dr = 0, n_items = 0;
     bool ok = true;
-    // S = Q K^T and dP = dO V^T of the next key tile
+    // S = Q K^T and dP = dO V^T of the next 64-key tile
     auto issue_sdp = [&](int stage, uint32_t phase) -> bool {
       if (!warp_wait(&sh.r_full[stage], phase, P, sh.abort_flag)) return false;
       tc_fence_after();
@@ -360,15 +393,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
         const uint64_t kd = k_desc + (uint64_t)(stage * kStep);
         const uint64_t vd = v_desc + (uint64_t)(stage * kStep);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t o = kmajor_off<DH>(kk);
-          mma_ss(tmem + Q_S, q_desc + o, kd + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < DH / 16; ++kk)
+          mma_ss(tmem + Q::S_COL, q_desc + kmajor_off<DH>(kk), kd + kmajor_off<DH, Q::TKD>(kk),
+                 idesc_s, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t o = kmajor_off<DH>(kk);
-          mma_ss(tmem + Q_DP, do_desc + o, vd + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < DH / 16; ++kk)
+          mma_ss(tmem + Q::DP_COL, do_desc + kmajor_off<DH>(kk), vd + kmajor_off<DH, Q::TKD>(kk),
+                 idesc_s, kk > 0 ? 1u : 0u);
         mma_commit(sh.sdp_full);
       }
       __syncwarp();
@@ -382,14 +413,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
       q_phase ^= 1;
       int st_next = st;
       uint32_t ph_next = r_phase;
+      const int nsteps = 2 * it.nk;
       if (!issue_sdp(st_next, ph_next)) break;
-      for (int j = 0; j < it.nk; ++j) {
+      for (int j = 0; j < nsteps; ++j) {
         const int st_j = st_next;
-        if (++st_next == C::STAGES) {
+        if (++st_next == Q::STAGES) {
           st_next = 0;
           ph_next ^= 1;
         }
-        if (j + 1 < it.nk) {
+        if (j + 1 < nsteps) {
           // the softmax warps hold S(j), dP(j) in registers: the next pair may be written
           if (!warp_wait(sh.s_free, n_sf & 1, P, sh.abort_flag)) { ok = false; break; }
           ++n_sf;
@@ -404,17 +436,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
         }
         tc_fence_after();
         if (elect_one()) {
-          // dQ (+)= dS K: A = dS (queries x keys, TMEM), B = K tile (N = head dim,
+          // dQ (+)= dS K: A = dS (queries x 64 keys, TMEM), B = the K tile (N = head dim,
           // K = keys; MN-major)
           const uint64_t kd = kmn_desc + (uint64_t)(st_j * kStep);
 #pragma unroll
-          for (int kk = 0; kk < TK / 16; ++kk)
-            mma_ts(tmem + Q_DQ, tmem + Q_DS + kk * 8,
+          for (int kk = 0; kk < Q::TKD / 16; ++kk)
+            mma_ts(tmem + Q::DQ_COL, tmem + Q::DS_COL + kk * 8,
                    kd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_dq,
                    (j == 0 && kk == 0) ? 0u : 1u);
           mma_commit(&sh.r_empty[st_j]);
           mma_commit(sh.d_free);
-          if (j + 1 == it.nk) {
+          if (j + 1 == nsteps) {
             mma_commit(sh.acc_full);
             mma_commit(sh.q_empty);
           }
@@ -425,8 +457,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
       r_phase = ph_next;
       ++n_items;
     }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    setmaxnreg_inc<kQLargeRegs>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -446,36 +480,36 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
       const float lse = valid ? P.lse[(int64_t)it.s * P.M + tok] : 0.f;
       const float dsum = valid ? P.dsum[(int64_t)it.s * P.M + tok] : 0.f;
       const int lim = !valid ? 0 : (P.causal ? q + 1 : P.T);  // keys < lim are live
+      const int nsteps = 2 * it.nk;
       bool ok = true;
-      for (int j = 0; j < it.nk; ++j) {
+      for (int j = 0; j < nsteps; ++j) {
         if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
         ++n_sdp;
         tc_fence_after();
-        const int kv0 = j * TK;
-        uint32_t pk[64];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        const int kv0 = j * Q::TKD;
+        uint32_t pk[32];
+        {
           uint32_t sr[64], dr[64];
-          tmem_ld64_wait(t_base + Q_S + h * 64, sr);
-          tmem_ld64_wait(t_base + Q_DP + h * 64, dr);
-          if (h == 1 && j + 1 < it.nk) {
+          tmem_ld64_wait(t_base + Q::S_COL, sr);
+          tmem_ld64_wait(t_base + Q::DP_COL, dr);
+          if (j + 1 < nsteps) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.s_free);
           }
-          if (kv0 + TK <= lim) {
+          if (kv0 + Q::TKD <= lim) {
             // every key of the tile is live for this query: no masks
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
               const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
               const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
-              pk[h * 32 + x] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * x]) - dsum),
-                                           p1 * (__uint_as_float(dr[2 * x + 1]) - dsum));
+              pk[x] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * x]) - dsum),
+                                  p1 * (__uint_as_float(dr[2 * x + 1]) - dsum));
             }
           } else {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              const int c = h * 64 + 2 * x;
+              const int c = 2 * x;
               float d0 = 0.f, d1 = 0.f;
               if (kv0 + c < lim) {
                 const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x]), c2, -lse));
@@ -485,7 +519,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
                 const float p = fast_exp2(fmaf(__uint_as_float(sr[2 * x + 1]), c2, -lse));
                 d1 = p * (__uint_as_float(dr[2 * x + 1]) - dsum);
               }
-              pk[h * 32 + x] = pack_bf16x2(d0, d1);
+              pk[x] = pack_bf16x2(d0, d1);
             }
           }
         }
@@ -495,7 +529,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
           break;
         }
         ++n_ds;
-        store_packed64(t_base + Q_DS, pk);
+        store_packed32(t_base + Q::DS_COL, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -519,7 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
 #pragma unroll
       for (int c0 = 0; c0 < DH; c0 += 16) {
         uint32_t r[16];
-        tmem_ld16_wait(t_base + Q_DQ + c0, r);
+        tmem_ld16_wait(t_base + Q::DQ_COL + c0, r);
         if (valid) {
           uint4 v0, v1;
           const float sc = P.scale;
@@ -540,7 +574,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
       if (lane == 0) mbar_arrive(sh.acc_free);
     }
   }
-  finish(P, tmem, warp);
+  finish(P, tmem, warp, QCfg<DH>::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -551,6 +585,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dq_kernel(const __grid_co
 struct KItem {
   int b, g, kt, ns, qt0, nj;
 };
+// Jobs of an item: (stream si of the head, 64-query tile qt0 + r) for si < ns, r < per.
 __device__ __forceinline__ KItem decode_k(const BwdParams& P, int i) {
   KItem it;
   const int bg = P.B * P.G;
@@ -559,37 +594,55 @@ __device__ __forceinline__ KItem decode_k(const BwdParams& P, int i) {
   it.g = r % P.G;
   it.b = r / P.G;
   it.ns = P.k + ((it.g == 0 && P.has_shared) ? 1 : 0);
-  it.qt0 = P.causal ? it.kt : 0;
-  it.nj = it.ns * (P.nq - it.qt0);
+  it.qt0 = P.causal ? 2 * it.kt : 0;  // 64-query tiles at or after the key tile
+  it.nj = it.ns * (P.nq64 - it.qt0);
   return it;
 }
 __device__ __forceinline__ void job_of(const BwdParams& P, const KItem& it, int j, int& s,
                                        int& qt) {
-  const int per = P.nq - it.qt0;
+  const int per = P.nq64 - it.qt0;
   const int si = j / per;
   qt = it.qt0 + j % per;
   s = si < P.k ? it.g * P.k + si : P.Sr;
 }
 
+// The dK / dV kernel runs two CTAs per SM with 64-query jobs: S^T and dP^T (64 columns
+// each) share their TMEM columns with P^T and dS^T, so the next job's S^T waits until the
+// current job's dV and dK products are done; the other CTA of the SM fills those gaps.
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
+struct KCfg {
   using C = BCfg<DH>;
+  static constexpr int TQJ = 64;                    // queries per job
+  static constexpr int QT_BYTES = TQJ * DH * 2;     // one 64-row Q or dO tile
+  static constexpr int STAGES = 3;
+  static constexpr int SMEM = 2 * C::TILE_BYTES + STAGES * 2 * QT_BYTES + 1024 + 512 + 2048;
+  static constexpr int TMEM_COLS = 256;
+  // S^T (P^T in its first 32 columns once read), dP^T (dS^T likewise), dV, dK
+  static constexpr int S_COL = 0, DP_COL = 64, DV_COL = 128, DK_COL = 128 + DH;
+  static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+
+template <int DH>
+__global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
+  using C = BCfg<DH>;
+  using K = KCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t *sK, *sV, *sQ, *sdO;
-  const Shared sh = carve<DH>(smem, sK, sV, sQ, sdO);
+  const Shared sh = carve(smem, C::TILE_BYTES, K::QT_BYTES, K::STAGES, sK, sV, sQ, sdO);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) init_shared(sh, C::STAGES);
+  if (threadIdx.x == 0) init_shared(sh, K::STAGES);
   if (warp == 1) {
-    tmem_alloc(sh.tmem_holder, C::TMEM_COLS);
+    tmem_alloc(sh.tmem_holder, K::TMEM_COLS);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&P.tm_q);
+    prefetch_tmap(&P.tm_q64);
     prefetch_tmap(&P.tm_k);
     prefetch_tmap(&P.tm_v);
-    prefetch_tmap(&P.tm_do);
+    prefetch_tmap(&P.tm_do64);
   }
   tc_fence_before();
   __syncthreads();
@@ -598,6 +651,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
   pdl_wait();
   pdl_allow_next();
 
+  if (warp < 4) {
+  setmaxnreg_dec<kQSmallRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------------ loads
     if (lane == 0) {
@@ -617,11 +672,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
           int s, qt;
           job_of(P, it, j, s, qt);
           if (!lane_wait(&sh.r_empty[st], r_phase ^ 1, P, sh.abort_flag)) break;
-          mbar_arrive_expect_tx(&sh.r_full[st], 2 * C::TILE_BYTES);
-          const int qrow = s * P.M + it.b * P.T + qt * TQ;
-          load_tile<DH>(P, &P.tm_q, sQ + st * C::TILE_BYTES, qrow, &sh.r_full[st]);
-          load_tile<DH>(P, &P.tm_do, sdO + st * C::TILE_BYTES, qrow, &sh.r_full[st]);
-          if (++st == C::STAGES) {
+          mbar_arrive_expect_tx(&sh.r_full[st], 2 * K::QT_BYTES);
+          const int qrow = s * P.M + it.b * P.T + qt * K::TQJ;
+          load_tile<DH, K::TQJ>(P, &P.tm_q64, sQ + st * K::QT_BYTES, qrow, &sh.r_full[st]);
+          load_tile<DH, K::TQJ>(P, &P.tm_do64, sdO + st * K::QT_BYTES, qrow, &sh.r_full[st]);
+          if (++st == K::STAGES) {
             st = 0;
             r_phase ^= 1;
           }
@@ -630,65 +685,36 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issue
-    const uint32_t idesc_s = idesc_bf16_f32(TK, TQ);
+    const uint32_t idesc_s = idesc_bf16_f32(TK, K::TQJ);
     const uint32_t idesc_kv = idesc_bf16_f32(TK, DH) | (1u << 16);  // B (Q, dO) MN-major
     const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t v_desc = smem_desc(smem_u32(sV), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t do_desc = smem_desc(smem_u32(sdO), 8 * C::ROW_BYTES, C::LAYOUT);
+    // Q and dO as MN-major B operands: 64-row chunks
     const uint64_t qmn_desc =
-        smem_desc_mn(smem_u32(sQ), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+        smem_desc_mn(smem_u32(sQ), K::TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t domn_desc =
-        smem_desc_mn(smem_u32(sdO), C::CHUNK_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
-    constexpr uint32_t kStep = C::TILE_BYTES >> 4;
+        smem_desc_mn(smem_u32(sdO), K::TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+    constexpr uint32_t kStep = K::QT_BYTES >> 4;
     int st = 0, islot = 0;
     uint32_t r_phase = 0, q_phase = 0, iphase = 0;
-    uint32_t n_sf = 0, n_dr = 0, n_items = 0;
+    uint32_t n_dr = 0, n_df = 0, n_items = 0;
     bool ok = true;
-    // S^T = K Q^T and dP^T = V dO^T of the next job
-    auto issue_sdp = [&](int stage, uint32_t phase) -> bool {
-      if (!warp_wait(&sh.r_full[stage], phase, P, sh.abort_flag)) return false;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t qd = q_desc + (uint64_t)(stage * kStep);
-        const uint64_t dd = do_desc + (uint64_t)(stage * kStep);
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t o = kmajor_off<DH>(kk);
-          mma_ss(tmem + K_S, k_desc + o, qd + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t o = kmajor_off<DH>(kk);
-          mma_ss(tmem + K_DP, v_desc + o, dd + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(sh.sdp_full);
-      }
-      __syncwarp();
-      return true;
-    };
     while (ok && !*sh.abort_flag) {
       int i;
       if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
       const KItem it = decode_k(P, i);
       if (!warp_wait(sh.q_full, q_phase, P, sh.abort_flag)) break;
       q_phase ^= 1;
-      int st_next = st;
-      uint32_t ph_next = r_phase;
-      if (!issue_sdp(st_next, ph_next)) break;
       for (int j = 0; j < it.nj; ++j) {
-        const int st_j = st_next;
-        if (++st_next == C::STAGES) {
-          st_next = 0;
-          ph_next ^= 1;
+        // S^T = K Q^T and dP^T = V dO^T of job j; their columns hold the previous job's
+        // P^T and dS^T until that job's products are done
+        if (!warp_wait(&sh.r_full[st], r_phase, P, sh.abort_flag)) { ok = false; break; }
+        if (n_df > 0 && !warp_wait(sh.d_free, (n_df - 1) & 1, P, sh.abort_flag)) {
+          ok = false;
+          break;
         }
-        if (j + 1 < it.nj) {
-          if (!warp_wait(sh.s_free, n_sf & 1, P, sh.abort_flag)) { ok = false; break; }
-          ++n_sf;
-          if (!issue_sdp(st_next, ph_next)) { ok = false; break; }
-        }
-        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
-        ++n_dr;
         if (j == 0 && n_items > 0 &&
             !warp_wait(sh.acc_free, (n_items - 1) & 1, P, sh.abort_flag)) {
           ok = false;
@@ -696,21 +722,38 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
         }
         tc_fence_after();
         if (elect_one()) {
-          const uint64_t dd = domn_desc + (uint64_t)(st_j * kStep);
-          const uint64_t qd = qmn_desc + (uint64_t)(st_j * kStep);
-          // dV (+)= P^T dO and dK (+)= dS^T Q: A from TMEM (keys x queries), B = dO / Q
-          // tile (N = head dim, K = queries; MN-major)
+          const uint64_t qd = q_desc + (uint64_t)(st * kStep);
+          const uint64_t dd = do_desc + (uint64_t)(st * kStep);
 #pragma unroll
-          for (int kk = 0; kk < TQ / 16; ++kk)
-            mma_ts(tmem + K_DV, tmem + K_P + kk * 8,
-                   dd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
+          for (int kk = 0; kk < DH / 16; ++kk)
+            mma_ss(tmem + K::S_COL, k_desc + kmajor_off<DH>(kk), qd + kmajor_off<DH, K::TQJ>(kk),
+                   idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < DH / 16; ++kk)
+            mma_ss(tmem + K::DP_COL, v_desc + kmajor_off<DH>(kk),
+                   dd + kmajor_off<DH, K::TQJ>(kk), idesc_s, kk > 0 ? 1u : 0u);
+          mma_commit(sh.sdp_full);
+        }
+        __syncwarp();
+        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_dr;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint64_t dmn = domn_desc + (uint64_t)(st * kStep);
+          const uint64_t qmn = qmn_desc + (uint64_t)(st * kStep);
+          // dV (+)= P^T dO and dK (+)= dS^T Q: A from TMEM (keys x 64 queries), B = the
+          // dO / Q tile (N = head dim, K = queries; MN-major)
+#pragma unroll
+          for (int kk = 0; kk < K::TQJ / 16; ++kk)
+            mma_ts(tmem + K::DV_COL, tmem + K::S_COL + kk * 8,
+                   dmn + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
                    (j == 0 && kk == 0) ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < TQ / 16; ++kk)
-            mma_ts(tmem + K_DK, tmem + K_DS + kk * 8,
-                   qd + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
+          for (int kk = 0; kk < K::TQJ / 16; ++kk)
+            mma_ts(tmem + K::DK_COL, tmem + K::DP_COL + kk * 8,
+                   qmn + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
                    (j == 0 && kk == 0) ? 0u : 1u);
-          mma_commit(&sh.r_empty[st_j]);
+          mma_commit(&sh.r_empty[st]);
           mma_commit(sh.d_free);
           if (j + 1 == it.nj) {
             mma_commit(sh.acc_full);
@@ -718,19 +761,24 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
           }
         }
         __syncwarp();
+        ++n_df;
+        if (++st == K::STAGES) {
+          st = 0;
+          r_phase ^= 1;
+        }
       }
-      st = st_next;
-      r_phase = ph_next;
       ++n_items;
     }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    setmaxnreg_inc<kQLargeRegs>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row of the tile (TMEM lane)
     const int tid = threadIdx.x - 128;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_base = tmem + lane_off;
-    uint32_t n_sdp = 0, n_pd = 0, n_acc = 0, n_job = 0;
+    uint32_t n_sdp = 0, n_acc = 0, n_job = 0;
     int islot = 0;
     uint32_t iphase = 0;
     const float c2 = P.scale_log2;
@@ -741,64 +789,47 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
       const int u = it.kt * TK + row;  // key position
       const bool key_ok = u < P.T;
       bool ok = true;
-      // a job's per-query lse and D (one value of each per thread), loaded one job ahead
+      // a job's per-query lse and D (threads 0..63 load one value of each), one job ahead
       auto fetch = [&](int jj, float& lv, float& dv) {
         int ss, qq_t;
         job_of(P, it, jj, ss, qq_t);
-        const int qq = qq_t * TQ + tid;
+        const int qq = qq_t * K::TQJ + (tid & 63);
         const int64_t idx = (int64_t)ss * P.M + (int64_t)it.b * P.T + qq;
         lv = qq < P.T ? P.lse[idx] : 0.f;
         dv = qq < P.T ? P.dsum[idx] : 0.f;
       };
       float nl = 0.f, nd = 0.f;
-      fetch(0, nl, nd);
+      if (tid < 64) fetch(0, nl, nd);
       for (int j = 0; j < it.nj; ++j, ++n_job) {
         int s, qt;
         job_of(P, it, j, s, qt);
-        // this job's values into its buffer; the buffer's barrier completes when all 128
-        // threads have written (a bounded wait); the next job's values are requested now
         const int buf = n_job & 1;
         float* sL = sh.sL + buf * 128;
         float* sD = sh.sD + buf * 128;
-        sL[tid] = nl;
-        sD[tid] = nd;
-        if (j + 1 < it.nj) fetch(j + 1, nl, nd);
+        if (tid < 64) {
+          sL[tid] = nl;
+          sD[tid] = nd;
+          if (j + 1 < it.nj) fetch(j + 1, nl, nd);
+        }
         mbar_arrive(&sh.l_bar[buf]);
         if (!warp_wait(&sh.l_bar[buf], (n_job >> 1) & 1, P, sh.abort_flag)) { ok = false; break; }
         if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
         ++n_sdp;
         tc_fence_after();
-        const int q0 = qt * TQ;
+        const int q0 = qt * K::TQJ;
         // live queries of this key: q < T, and q >= u when causal
         const int qlo = P.causal ? u : 0;
-        const bool all_live = key_ok && q0 >= qlo && q0 + TQ <= P.T;
+        const bool all_live = key_ok && q0 >= qlo && q0 + K::TQJ <= P.T;
         uint32_t pp[32], pd[32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        {
           uint32_t sr[64], dr[64];
-          tmem_ld64_wait(t_base + K_S + h * 64, sr);
-          tmem_ld64_wait(t_base + K_DP + h * 64, dr);
-          if (h == 1) {
-            if (j + 1 < it.nj) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(sh.s_free);
-            }
-            // the first half goes to TMEM once the previous job's products have read it
-            if (n_pd > 0 && !warp_wait(sh.d_free, (n_pd - 1) & 1, P, sh.abort_flag)) {
-              ok = false;
-              break;
-            }
-            ++n_pd;
-            store_packed32(t_base + K_P, pp);
-            store_packed32(t_base + K_DS, pd);
-          }
+          tmem_ld64_wait(t_base + K::S_COL, sr);
+          tmem_ld64_wait(t_base + K::DP_COL, dr);
           if (all_live) {
-            // every query of the tile is live for this key: no masks
 #pragma unroll
             for (int x4 = 0; x4 < 16; ++x4) {
-              const float4 L4 = reinterpret_cast<const float4*>(sL + h * 64)[x4];
-              const float4 D4 = reinterpret_cast<const float4*>(sD + h * 64)[x4];
+              const float4 L4 = reinterpret_cast<const float4*>(sL)[x4];
+              const float4 D4 = reinterpret_cast<const float4*>(sD)[x4];
               const float p0 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4]), c2, -L4.x));
               const float p1 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4 + 1]), c2, -L4.y));
               const float p2 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4 + 2]), c2, -L4.z));
@@ -813,7 +844,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
           } else {
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              const int c = h * 64 + 2 * x;
+              const int c = 2 * x;
               float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
               const int qa = q0 + c, qb = q0 + c + 1;
               if (key_ok && qa < P.T && qa >= qlo) {
@@ -829,9 +860,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
             }
           }
         }
-        if (!ok) break;
-        store_packed32(t_base + K_P + 32, pp);
-        store_packed32(t_base + K_DS + 32, pd);
+        // P^T and dS^T over the columns just read (the MMA warp issues nothing into them
+        // until this job's products are done)
+        store_packed32(t_base + K::S_COL, pp);
+        store_packed32(t_base + K::DP_COL, pd);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -848,7 +880,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* dst = (which == 0 ? P.dk : P.dv) + off;
         const float sc = which == 0 ? P.scale : 1.f;
-        const uint32_t col = which == 0 ? K_DK : K_DV;
+        const uint32_t col = which == 0 ? K::DK_COL : K::DV_COL;
 #pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 16) {
           uint32_t r[16];
@@ -873,15 +905,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_dkdv_kernel(const __grid_
       if (lane == 0) mbar_arrive(sh.acc_free);
     }
   }
-  finish(P, tmem, warp);
+  finish(P, tmem, warp, KCfg<DH>::TMEM_COLS);
 }
 
 template <int DH>
 int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has_shared,
                   int causal, cudaStream_t st) {
   using C = BCfg<DH>;
-  if (!set_smem_limit_once<attn_bwd_dq_kernel<DH>>(C::SMEM)) return -1;
-  if (!set_smem_limit_once<attn_bwd_dkdv_kernel<DH>>(C::SMEM)) return -1;
+  if (!set_smem_limit_once<attn_bwd_dq_kernel<DH>>(QCfg<DH>::SMEM)) return -1;
+  if (!set_smem_limit_once<attn_bwd_dkdv_kernel<DH>>(KCfg<DH>::SMEM)) return -1;
   const int M = B * T;
   BwdParams P;
   memset(&P, 0, sizeof(P));
@@ -890,12 +922,20 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
               tmap_bf16_chunked(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
               tmap_bf16_chunked(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
               tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
-              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw);
+              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
+              tmap_bf16_chunked(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
+              tmap_bf16_chunked(&P.tm_q64, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 64, sw) &&
+              tmap_bf16_chunked(&P.tm_do64, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 64, sw);
   if (!P.chunked &&
       (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
        !tmap_bf16_2d_ext(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
        !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw)))
+       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_q64, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 64, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_do64, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 64, sw)))
     return -1;
   P.lse = h->ws.lse;
   P.dsum = bb.dsum;
@@ -916,6 +956,7 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   P.has_shared = has_shared;
   P.causal = causal;
   P.nq = (T + TQ - 1) / TQ;
+  P.nq64 = (T + 63) / 64;
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   P.scale = 1.f / sqrtf((float)DH);
   P.status = h->ws.status;
@@ -923,15 +964,15 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   P.counter = bb.counter;
   // dQ
   P.items = B * S * P.nq;
-  int grid = P.items < h->num_sms ? P.items : h->num_sms;
-  if (launch_pdl(attn_bwd_dq_kernel<DH>, dim3(grid), dim3(THREADS), C::SMEM, st, P) !=
+  int grid = P.items < 2 * h->num_sms ? P.items : 2 * h->num_sms;  // two CTAs per SM
+  if (launch_pdl(attn_bwd_dq_kernel<DH>, dim3(grid), dim3(THREADS), QCfg<DH>::SMEM, st, P) !=
       cudaSuccess)
     return -1;
   // dK, dV
   P.items = B * h->G * P.nq;
   P.counter = bb.counter + 2;
-  grid = P.items < h->num_sms ? P.items : h->num_sms;
-  if (launch_pdl(attn_bwd_dkdv_kernel<DH>, dim3(grid), dim3(THREADS), C::SMEM, st, P) !=
+  grid = P.items < 2 * h->num_sms ? P.items : 2 * h->num_sms;  // two CTAs per SM
+  if (launch_pdl(attn_bwd_dkdv_kernel<DH>, dim3(grid), dim3(THREADS), KCfg<DH>::SMEM, st, P) !=
       cudaSuccess)
     return -1;
   return 2;

@@ -101,6 +101,11 @@ WORKLOADS = {
                           seed=3, balance=0.10),
     # Wider groups: E = 4 per group, k = 2.
     "wide_k2": Workload("wide_k2", dim=2048, N=32, G=8, k=2, d_h=64, B=2, T=8192, seed=4),
+    # Contexts beyond 32K: the long-context layer at 64K and 128K tokens (the pages quote the
+    # prefill speedup from 4K up to 1024K tokens).
+    "long_t64k": Workload("long_t64k", dim=768, N=16, G=8, k=1, d_h=48, B=1, T=65536, seed=6),
+    "long_t128k": Workload("long_t128k", dim=768, N=16, G=8, k=1, d_h=48, B=1, T=131072,
+                           seed=7),
     # Large and skewed: 70% of tokens to expert 0 of each group.
     "large_skew": Workload("large_skew", dim=4096, N=32, G=8, k=1, d_h=128, B=1, T=32768,
                            seed=5, skew=0.70),

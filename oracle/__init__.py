@@ -8,5 +8,5 @@ from .gqe_oracle import (  # noqa: F401
     top_k_per_group, route, kv_projection, routed_queries, shared_query, stream_kv_head,
     attention_rows, attention, combine, output_projection, aux_loss, forward, forward_rows,
     DecodeResult, decode, Grads, attention_rows_backward, slot_weights_backward,
-    aux_loss_grad_p, group_softmax_backward, backward,
+    aux_loss_grad_p, group_softmax_backward, backward, backward_x_rows,
 )

@@ -573,3 +573,97 @@ def backward(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v, W_
         dW_s = dQ[G * k].T @ x
         dx += dQ[G * k] @ W_shared
     return Grads(dx, dW_r, dW_q, dW_k, dW_v, dW_s, dW_o)
+
+
+def backward_x_rows(layer: Layer, x: np.ndarray, B: int, T: int, W_r, W_q, W_k, W_v,
+                    W_shared, W_o, dy: np.ndarray, dA: float, t_min: int) -> np.ndarray:
+    """Rows of dx (the input gradient of backward) for the positions t >= t_min of every
+    sequence, causal layers only, without the work of the earlier rows.
+
+    Causally, key t is read only by queries at positions >= t, so dK and dV of the rows at
+    t >= t_min, like dQ and the router gradient of those rows, depend only on the queries at
+    positions >= t_min (each attending over its whole prefix). The steps are backward's,
+    restricted to those query rows. Returns dx [B * (T - t_min), dim], sequence by sequence.
+    """
+    if not layer.causal:
+        raise ValueError("the row restriction needs a causal layer")
+    G, k, E, d_h, N = layer.G, layer.k, layer.E, layer.d_h, layer.N
+    M = x.shape[0]
+    rt = route(x, W_r, G, k)
+    K, V = kv_projection(x, W_k, W_v, G, d_h)
+    rows = np.concatenate([np.arange(b * T + t_min, (b + 1) * T) for b in range(B)])
+    xs = x[rows]
+    R = rows.size
+    sel = rt.sel[rows]
+    Q = routed_queries(xs, W_q, sel, G, E, d_h)
+    if layer.shared:
+        Q = np.concatenate([Q, shared_query(xs, W_shared)[None]], axis=0)
+    S = Q.shape[0]
+    pos = np.arange(t_min, T)
+    nr = T - t_min
+    O = np.empty((S, R, d_h))
+    for s in range(S):
+        h = stream_kv_head(s, k, G)
+        for b in range(B):
+            m = slice(b * nr, (b + 1) * nr)
+            seq = slice(b * T, (b + 1) * T)
+            O[s, m] = attention_rows(Q[s, m], pos, K[h, seq], V[h, seq], True)
+    sub = Routing(rt.logits[rows], rt.p[rows], sel, rt.p_sel[rows], rt.gates[rows], rt.w[rows],
+                  rt.counts, rt.prob_sum)
+    # output construction and router, as in backward, for these rows
+    dZ = dy[rows] @ W_o
+    dO = np.zeros_like(O)
+    dp_sel = np.zeros((R, G, k))
+    col = 0
+    for g in range(G):
+        for r in range(k):
+            s = g * k + r
+            blk = dZ[:, col:col + d_h]
+            col += d_h
+            if layer.variant == "weighted_concat":
+                dO[s] += sub.p_sel[:, g, r][:, None] * blk
+                dp_sel[:, g, r] += (blk * O[s]).sum(axis=1)
+            else:
+                dO[s] += blk
+    if layer.variant == "gqe":
+        dslot = dZ[:, col:col + d_h]
+        col += d_h
+        dw = np.zeros((R, G, k))
+        for g in range(G):
+            for r in range(k):
+                s = g * k + r
+                dO[s] += sub.w[:, g, r][:, None] * dslot
+                dw[:, g, r] = (dslot * O[s]).sum(axis=1)
+        dp_sel += slot_weights_backward(dw, sub.w, sub.p_sel)
+    if layer.shared:
+        dO[G * k] += dZ[:, col:col + d_h]
+    dp = np.zeros((R, G, E))
+    ri = np.arange(R)
+    for g in range(G):
+        for r in range(k):
+            dp[ri, g, sel[:, g, r]] += dp_sel[:, g, r]
+    if dA:
+        dp += dA * aux_loss_grad_p(rt.counts, M, G, k)[None]
+    dl = group_softmax_backward(sub.p, dp).reshape(R, N)
+    dx = dl @ W_r
+    # attention: the queries at t >= t_min give dQ of their rows and all of dK, dV at
+    # t >= t_min
+    for s in range(S):
+        h = stream_kv_head(s, k, G)
+        for b in range(B):
+            m = slice(b * nr, (b + 1) * nr)
+            seq = slice(b * T, (b + 1) * T)
+            dq, dk, dv = attention_rows_backward(Q[s, m], pos, K[h, seq], V[h, seq], dO[s, m],
+                                                 True)
+            rg = slice(h * d_h, (h + 1) * d_h)
+            dx[m] += dk[t_min:] @ W_k[rg] + dv[t_min:] @ W_v[rg]
+            if s < G * k:
+                g, r = divmod(s, k)
+                for j in range(E):
+                    sel_rows = np.nonzero(sel[m, g, r] == j)[0]
+                    if sel_rows.size:
+                        re = slice((g * E + j) * d_h, (g * E + j + 1) * d_h)
+                        dx[m][sel_rows] += dq[sel_rows] @ W_q[re]
+            else:
+                dx[m] += dq @ W_shared
+    return dx

@@ -152,3 +152,29 @@ def test_backward_unsupported_shapes():
         G.gqe_enable_backward(h)
     assert e.value.status == G.GQE_ERR_UNSUPPORTED
     G.gqe_destroy(h)
+
+
+@pytest.mark.parametrize("name", ["long_t16k", "main_b8_t2048"])
+def test_backward_full_size_last_rows(name):
+    """At the benchmark's full sizes, in its launch configuration: the input gradient of the
+    last 256 positions of every sequence against the oracle's row-restricted backward (which
+    needs only the queries at those positions), within the bf16 tolerance."""
+    import oracle
+    wl = W.WORKLOADS[name]
+    inp = W.cached(name)
+    dy = W.grad_output(wl)
+    run = GpuRun(inp).forward()
+    got = _gpu_backward(run, dy, 0.01)
+    run.close()
+    t_min = wl.T - 256
+    f = inp.f64
+    layer = oracle.Layer(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, shared=wl.shared,
+                         variant=wl.variant, causal=wl.causal)
+    ref = oracle.backward_x_rows(layer, f("x"), wl.B, wl.T, f("W_r"), f("W_q"), f("W_k"),
+                                 f("W_v"), f("W_shared"), f("W_o"), dy.astype(np.float64), 0.01,
+                                 t_min)
+    rows = np.concatenate([np.arange(b * wl.T + t_min, (b + 1) * wl.T) for b in range(wl.B)])
+    assert rel_l2(got["x"][rows], ref) <= GRAD_REL_L2
+    for k_, v in got.items():
+        if v is not None:
+            assert np.isfinite(v).all(), k_

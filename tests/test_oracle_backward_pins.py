@@ -214,3 +214,18 @@ def test_planted_router_backward_mistake_is_caught(name, mistake, monkeypatch):
     monkeypatch.setattr(go, name, mistake)
     with pytest.raises(AssertionError):
         test_backward_matches_torch_autograd(0)
+
+
+@pytest.mark.parametrize("variant,N,G,k", [("gqe", 6, 3, 1), ("weighted_concat", 6, 3, 1),
+                                           ("hard_concat", 6, 3, 1), ("gqe", 8, 2, 2)])
+def test_backward_x_rows_equals_the_full_backward(variant, N, G, k):
+    """The row-restricted input gradient (queries at positions >= t_min only) equals those
+    rows of the full backward's dx: causally, nothing earlier reaches them."""
+    layer = go.Layer(dim=12, N=N, G=G, k=k, d_h=4, shared=True, variant=variant)
+    rng = np.random.default_rng(31)
+    B, T, t_min = 2, 23, 15
+    x, W_r, W_q, W_k, W_v, W_s, W_o, dy = rand_case(rng, layer, B, T)
+    full = go.backward(layer, x, B, T, W_r, W_q, W_k, W_v, W_s, W_o, dy, 0.3)
+    part = go.backward_x_rows(layer, x, B, T, W_r, W_q, W_k, W_v, W_s, W_o, dy, 0.3, t_min)
+    rows = np.concatenate([np.arange(b * T + t_min, (b + 1) * T) for b in range(B)])
+    np.testing.assert_allclose(part, full.x[rows], rtol=1e-10, atol=1e-12)

@@ -102,6 +102,7 @@ FULL = {
     "wide_k2_weighted": dict(variant="weighted_concat"),
     "wide_k2_hard": dict(variant="hard_concat"),
     "large_skew": {},
+    "long_t64k": {},
 }
 
 
