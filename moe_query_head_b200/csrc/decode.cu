@@ -353,13 +353,14 @@ int launch_dh(const DecParams& P, cudaStream_t st) {
 
 }  // namespace
 
-// Chunks per (sequence, group): enough CTAs for eight per SM, about two waves of the five
-// resident at d_h = 48 (measured at 64 sequences of 8192 cached tokens: 232 us with one chunk
-// per (sequence, group), 195 us with two, 182 us with three), at least one tile each, and
-// partial slots within the workspace's kDecodeSlots.
+// Chunks per (sequence, group): enough CTAs for sixteen per SM, about three waves of the
+// five resident at d_h = 48 (measured at 64 sequences of 8192 cached tokens: 232 us with one
+// chunk per (sequence, group), 195 us with two, 182 us with three, 169 us with five, 167 us
+// with seven), at least one tile each, and partial slots within the workspace's
+// kDecodeSlots.
 int decode_chunks(const gqe_ctx* h, int B, int L_max) {
   const int64_t bg = (int64_t)B * h->G;
-  int64_t nc = (8 * (int64_t)h->num_sms + bg - 1) / bg;
+  int64_t nc = (16 * (int64_t)h->num_sms + bg - 1) / bg;
   const int64_t max_by_len = ((int64_t)L_max + TKD - 1) / TKD;
   if (nc > max_by_len) nc = max_by_len;
   while (nc > 1 && bg * nc > kDecodeSlots) --nc;
