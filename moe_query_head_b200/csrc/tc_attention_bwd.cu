@@ -10,22 +10,24 @@
 //   dV = sum over the head's streams of P^T dO.
 //
 // Two kernels, neither with atomics (every output row is written by one CTA, so the result
-// is the same from run to run):
-//   attn_bwd_dq_kernel    work item = (sequence, stream, 128-query tile); for each key tile
+// is the same from run to run), each at two CTAs per SM (256 TMEM columns each; warpgroup 0
+// gives registers to the softmax warpgroup):
+//   attn_bwd_dq_kernel    work item = (sequence, stream, 128-query tile); per 64-key step
 //                         S = Q K^T and dP = dO V^T (both operands from shared memory) into
 //                         TMEM, the softmax warpgroup forms dS in bf16 in TMEM, and
 //                         dQ += dS K (A from TMEM, K as an MN-major shared-memory operand)
 //                         accumulates in TMEM. The routed stream (g, r) of token t lands in
 //                         row t of dQ_exp [M, N d_h] at the column block of its expert
 //                         g E + sel[t, g, r]; the shared stream in dQ_sh [M, d_h].
-//   attn_bwd_dkdv_kernel  work item = (sequence, KV head, 128-key tile); for each query tile
-//                         of each stream that reads the head, S^T = K Q^T and dP^T = V dO^T
-//                         into TMEM, the softmax warpgroup (one key per thread) forms P^T
-//                         and dS^T in bf16 in TMEM, and dV += P^T dO, dK += dS^T Q
-//                         accumulate in TMEM over all of the head's streams. dK, dV land
-//                         token-major in [M, G d_h] (head g at column g d_h).
-// Warps: 0 TMA loads, 1 TMEM owner and MMA issue, 2-3 idle, 4-7 softmax and epilogue. One
-// CTA per SM (TMEM: 512 columns), persistent, heaviest items first. Head dims up to 64.
+//   attn_bwd_dkdv_kernel  work item = (sequence, KV head, 128-key tile); per job (a stream
+//                         that reads the head, a tile of 48 queries, 32 at d_h = 64),
+//                         S^T = K Q^T and dP^T = V dO^T into TMEM, the softmax warpgroup
+//                         (one key per thread) forms P^T and dS^T in bf16 in TMEM, and
+//                         dV += P^T dO, dK += dS^T Q accumulate in TMEM over all of the
+//                         head's streams. dK, dV land token-major in [M, G d_h].
+// Warps: 0 TMA loads, 1 TMEM owner and MMA issue, 2-3 idle, 4-7 softmax and epilogue; the
+// next tile's S and dP are issued as soon as the softmax warps hold the current ones in
+// registers. Persistent CTAs take items heaviest first. Head dims up to 64.
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
@@ -73,7 +75,7 @@ constexpr int K_S = 0, K_DP = 128, K_P = 256, K_DS = 320, K_DV = 384, K_DK = 448
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO [S M, d_h]; K, V [G M, d_h]; 128-row boxes
   CUtensorMap tm_k64, tm_v64;           // K, V with 64-row boxes (the dQ kernel)
-  CUtensorMap tm_q64, tm_do64;          // Q, dO with 64-row boxes (the dK / dV kernel)
+  CUtensorMap tm_qj, tm_doj;            // Q, dO with job-row boxes (the dK / dV kernel)
   const float* lse;     // [S, M]
   const float* dsum;    // [S, M] rowsum(dO * O)
   const int32_t* sel;   // [M, G, k]
@@ -81,7 +83,7 @@ struct BwdParams {
   __nv_bfloat16* dq_sh;   // [M, d_h]
   __nv_bfloat16* dk;      // [M, G d_h]
   __nv_bfloat16* dv;      // [M, G d_h]
-  int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, nq64, items, chunked;
+  int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, items, chunked;
   float scale_log2;  // log2(e) / sqrt(d_h)
   float scale;       // 1 / sqrt(d_h)
   int* counter;      // [2] item counter and exit counter (zero at launch; reset by the last CTA)
@@ -582,10 +584,82 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_co
 // most query tiles). Jobs of an item: every (stream reading g, query tile at or after the
 // key tile when causal).
 // ---------------------------------------------------------------------------------------
+// TMEM -> registers, N consecutive 32-bit columns per lane (N = 32 or 48), and the wait
+// for them in the same statement.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld48_wait(uint32_t taddr, uint32_t (&r)[48]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%49];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+        "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47])
+      : "r"(taddr), "r"(taddr + 32u)
+      : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_ldN_wait(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32) tmem_ld32_wait(taddr, r);
+  else tmem_ld48_wait(taddr, r);
+}
+// bf16 pairs of a packed row -> TMEM, N/2 columns (N = 32 or 48), 8 columns per store
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// The dK / dV kernel runs two CTAs per SM with jobs of TQJ queries (48 for head dims up to
+// 48, 32 for 64), small enough that S^T, dP^T, P^T, dS^T, dV and dK all have TMEM columns
+// of their own within 256: the next job's S^T and dP^T are issued as soon as the softmax
+// warps hold the current ones in registers, as in the dQ kernel.
+template <int DH>
+struct KCfg {
+  using C = BCfg<DH>;
+  static constexpr int TQJ = DH <= 48 ? 48 : 32;    // queries per job
+  static constexpr int QT_BYTES = TQJ * DH * 2;     // one Q or dO tile of the job
+  static constexpr int STAGES = 3;
+  static constexpr int WARP_STAGE = 4 * 2 * 2 * 48 * 4;  // per-warp lse / D buffers
+  static constexpr int SMEM =
+      2 * C::TILE_BYTES + STAGES * 2 * QT_BYTES + 1024 + 512 + 2048 + WARP_STAGE;
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int S_COL = 0, DP_COL = TQJ, P_COL = 2 * TQJ, DS_COL = 2 * TQJ + TQJ / 2;
+  static constexpr int DV_COL = 3 * TQJ, DK_COL = 3 * TQJ + DH;
+  static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
+  static_assert(DP_COL % 16 == 0 && DV_COL % 16 == 0 && DK_COL % 16 == 0, "accumulator columns");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+
 struct KItem {
   int b, g, kt, ns, qt0, nj;
 };
-// Jobs of an item: (stream si of the head, 64-query tile qt0 + r) for si < ns, r < per.
+// Jobs of an item: (stream si of the head, query tile qt0 + r of TQJ queries) for si < ns,
+// r < per; the first tile is the first one reaching a query at or after the key tile.
+template <int TQJ>
 __device__ __forceinline__ KItem decode_k(const BwdParams& P, int i) {
   KItem it;
   const int bg = P.B * P.G;
@@ -594,44 +668,32 @@ __device__ __forceinline__ KItem decode_k(const BwdParams& P, int i) {
   it.g = r % P.G;
   it.b = r / P.G;
   it.ns = P.k + ((it.g == 0 && P.has_shared) ? 1 : 0);
-  it.qt0 = P.causal ? 2 * it.kt : 0;  // 64-query tiles at or after the key tile
-  it.nj = it.ns * (P.nq64 - it.qt0);
+  const int nqj = (P.T + TQJ - 1) / TQJ;
+  it.qt0 = P.causal ? (it.kt * TK) / TQJ : 0;
+  it.nj = it.ns * (nqj - it.qt0);
   return it;
 }
+template <int TQJ>
 __device__ __forceinline__ void job_of(const BwdParams& P, const KItem& it, int j, int& s,
                                        int& qt) {
-  const int per = P.nq64 - it.qt0;
+  const int per = (P.T + TQJ - 1) / TQJ - it.qt0;
   const int si = j / per;
   qt = it.qt0 + j % per;
   s = si < P.k ? it.g * P.k + si : P.Sr;
 }
 
-// The dK / dV kernel runs two CTAs per SM with 64-query jobs: S^T and dP^T (64 columns
-// each) share their TMEM columns with P^T and dS^T, so the next job's S^T waits until the
-// current job's dV and dK products are done; the other CTA of the SM fills those gaps.
-template <int DH>
-struct KCfg {
-  using C = BCfg<DH>;
-  static constexpr int TQJ = 64;                    // queries per job
-  static constexpr int QT_BYTES = TQJ * DH * 2;     // one 64-row Q or dO tile
-  static constexpr int STAGES = 3;
-  static constexpr int SMEM = 2 * C::TILE_BYTES + STAGES * 2 * QT_BYTES + 1024 + 512 + 2048;
-  static constexpr int TMEM_COLS = 256;
-  // S^T (P^T in its first 32 columns once read), dP^T (dS^T likewise), dV, dK
-  static constexpr int S_COL = 0, DP_COL = 64, DV_COL = 128, DK_COL = 128 + DH;
-  static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
-  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
-};
-
 template <int DH>
 __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
   using C = BCfg<DH>;
   using K = KCfg<DH>;
+  constexpr int TQJ = K::TQJ;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t *sK, *sV, *sQ, *sdO;
   const Shared sh = carve(smem, C::TILE_BYTES, K::QT_BYTES, K::STAGES, sK, sV, sQ, sdO);
+  // per-warp lse / D buffers after the shared lse / D area (unused here)
+  float* wstage = sh.sD + 256;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) init_shared(sh, K::STAGES);
   if (warp == 1) {
@@ -639,10 +701,10 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&P.tm_q64);
+    prefetch_tmap(&P.tm_qj);
     prefetch_tmap(&P.tm_k);
     prefetch_tmap(&P.tm_v);
-    prefetch_tmap(&P.tm_do64);
+    prefetch_tmap(&P.tm_doj);
   }
   tc_fence_before();
   __syncthreads();
@@ -661,7 +723,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
       while (!*sh.abort_flag) {
         int i;
         if (!publish_item(sh, P, islot, iphase, i) || i < 0) break;
-        const KItem it = decode_k(P, i);
+        const KItem it = decode_k<TQJ>(P, i);
         if (!lane_wait(sh.q_empty, q_phase ^ 1, P, sh.abort_flag)) break;
         q_phase ^= 1;
         mbar_arrive_expect_tx(sh.q_full, 2 * C::TILE_BYTES);
@@ -670,12 +732,12 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
         load_tile<DH>(P, &P.tm_v, sV, krow, sh.q_full);
         for (int j = 0; j < it.nj; ++j) {
           int s, qt;
-          job_of(P, it, j, s, qt);
+          job_of<TQJ>(P, it, j, s, qt);
           if (!lane_wait(&sh.r_empty[st], r_phase ^ 1, P, sh.abort_flag)) break;
           mbar_arrive_expect_tx(&sh.r_full[st], 2 * K::QT_BYTES);
-          const int qrow = s * P.M + it.b * P.T + qt * K::TQJ;
-          load_tile<DH, K::TQJ>(P, &P.tm_q64, sQ + st * K::QT_BYTES, qrow, &sh.r_full[st]);
-          load_tile<DH, K::TQJ>(P, &P.tm_do64, sdO + st * K::QT_BYTES, qrow, &sh.r_full[st]);
+          const int qrow = s * P.M + it.b * P.T + qt * TQJ;
+          load_tile<DH, TQJ>(P, &P.tm_qj, sQ + st * K::QT_BYTES, qrow, &sh.r_full[st]);
+          load_tile<DH, TQJ>(P, &P.tm_doj, sdO + st * K::QT_BYTES, qrow, &sh.r_full[st]);
           if (++st == K::STAGES) {
             st = 0;
             r_phase ^= 1;
@@ -685,36 +747,65 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issue
-    const uint32_t idesc_s = idesc_bf16_f32(TK, K::TQJ);
+    const uint32_t idesc_s = idesc_bf16_f32(TK, TQJ);
     const uint32_t idesc_kv = idesc_bf16_f32(TK, DH) | (1u << 16);  // B (Q, dO) MN-major
     const uint64_t k_desc = smem_desc(smem_u32(sK), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t v_desc = smem_desc(smem_u32(sV), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t q_desc = smem_desc(smem_u32(sQ), 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t do_desc = smem_desc(smem_u32(sdO), 8 * C::ROW_BYTES, C::LAYOUT);
-    // Q and dO as MN-major B operands: 64-row chunks
+    // Q and dO as MN-major B operands: TQJ-row chunks
     const uint64_t qmn_desc =
-        smem_desc_mn(smem_u32(sQ), K::TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+        smem_desc_mn(smem_u32(sQ), TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
     const uint64_t domn_desc =
-        smem_desc_mn(smem_u32(sdO), K::TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
+        smem_desc_mn(smem_u32(sdO), TQJ * C::ROW_BYTES, 8 * C::ROW_BYTES, C::LAYOUT);
     constexpr uint32_t kStep = K::QT_BYTES >> 4;
     int st = 0, islot = 0;
     uint32_t r_phase = 0, q_phase = 0, iphase = 0;
-    uint32_t n_dr = 0, n_df = 0, n_items = 0;
+    uint32_t n_sf = 0, n_dr = 0, n_items = 0;
     bool ok = true;
+    // S^T = K Q^T and dP^T = V dO^T of the next job
+    auto issue_sdp = [&](int stage, uint32_t phase) -> bool {
+      if (!warp_wait(&sh.r_full[stage], phase, P, sh.abort_flag)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t qd = q_desc + (uint64_t)(stage * kStep);
+        const uint64_t dd = do_desc + (uint64_t)(stage * kStep);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          mma_ss(tmem + K::S_COL, k_desc + kmajor_off<DH>(kk), qd + kmajor_off<DH, TQJ>(kk),
+                 idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          mma_ss(tmem + K::DP_COL, v_desc + kmajor_off<DH>(kk), dd + kmajor_off<DH, TQJ>(kk),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(sh.sdp_full);
+      }
+      __syncwarp();
+      return true;
+    };
     while (ok && !*sh.abort_flag) {
       int i;
       if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
-      const KItem it = decode_k(P, i);
+      const KItem it = decode_k<TQJ>(P, i);
       if (!warp_wait(sh.q_full, q_phase, P, sh.abort_flag)) break;
       q_phase ^= 1;
+      int st_next = st;
+      uint32_t ph_next = r_phase;
+      if (!issue_sdp(st_next, ph_next)) break;
       for (int j = 0; j < it.nj; ++j) {
-        // S^T = K Q^T and dP^T = V dO^T of job j; their columns hold the previous job's
-        // P^T and dS^T until that job's products are done
-        if (!warp_wait(&sh.r_full[st], r_phase, P, sh.abort_flag)) { ok = false; break; }
-        if (n_df > 0 && !warp_wait(sh.d_free, (n_df - 1) & 1, P, sh.abort_flag)) {
-          ok = false;
-          break;
+        const int st_j = st_next;
+        if (++st_next == K::STAGES) {
+          st_next = 0;
+          ph_next ^= 1;
         }
+        if (j + 1 < it.nj) {
+          // the softmax warps hold S^T(j), dP^T(j) in registers: the next pair may be written
+          if (!warp_wait(sh.s_free, n_sf & 1, P, sh.abort_flag)) { ok = false; break; }
+          ++n_sf;
+          if (!issue_sdp(st_next, ph_next)) { ok = false; break; }
+        }
+        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
+        ++n_dr;
         if (j == 0 && n_items > 0 &&
             !warp_wait(sh.acc_free, (n_items - 1) & 1, P, sh.abort_flag)) {
           ok = false;
@@ -722,38 +813,21 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
         }
         tc_fence_after();
         if (elect_one()) {
-          const uint64_t qd = q_desc + (uint64_t)(st * kStep);
-          const uint64_t dd = do_desc + (uint64_t)(st * kStep);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            mma_ss(tmem + K::S_COL, k_desc + kmajor_off<DH>(kk), qd + kmajor_off<DH, K::TQJ>(kk),
-                   idesc_s, kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk)
-            mma_ss(tmem + K::DP_COL, v_desc + kmajor_off<DH>(kk),
-                   dd + kmajor_off<DH, K::TQJ>(kk), idesc_s, kk > 0 ? 1u : 0u);
-          mma_commit(sh.sdp_full);
-        }
-        __syncwarp();
-        if (!warp_wait(sh.d_ready, n_dr & 1, P, sh.abort_flag)) { ok = false; break; }
-        ++n_dr;
-        tc_fence_after();
-        if (elect_one()) {
-          const uint64_t dmn = domn_desc + (uint64_t)(st * kStep);
-          const uint64_t qmn = qmn_desc + (uint64_t)(st * kStep);
-          // dV (+)= P^T dO and dK (+)= dS^T Q: A from TMEM (keys x 64 queries), B = the
+          const uint64_t dmn = domn_desc + (uint64_t)(st_j * kStep);
+          const uint64_t qmn = qmn_desc + (uint64_t)(st_j * kStep);
+          // dV (+)= P^T dO and dK (+)= dS^T Q: A from TMEM (keys x TQJ queries), B = the
           // dO / Q tile (N = head dim, K = queries; MN-major)
 #pragma unroll
-          for (int kk = 0; kk < K::TQJ / 16; ++kk)
-            mma_ts(tmem + K::DV_COL, tmem + K::S_COL + kk * 8,
+          for (int kk = 0; kk < TQJ / 16; ++kk)
+            mma_ts(tmem + K::DV_COL, tmem + K::P_COL + kk * 8,
                    dmn + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
                    (j == 0 && kk == 0) ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < K::TQJ / 16; ++kk)
-            mma_ts(tmem + K::DK_COL, tmem + K::DP_COL + kk * 8,
+          for (int kk = 0; kk < TQJ / 16; ++kk)
+            mma_ts(tmem + K::DK_COL, tmem + K::DS_COL + kk * 8,
                    qmn + (uint64_t)((kk * 16 * C::ROW_BYTES) >> 4), idesc_kv,
                    (j == 0 && kk == 0) ? 0u : 1u);
-          mma_commit(&sh.r_empty[st]);
+          mma_commit(&sh.r_empty[st_j]);
           mma_commit(sh.d_free);
           if (j + 1 == it.nj) {
             mma_commit(sh.acc_full);
@@ -761,12 +835,9 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
           }
         }
         __syncwarp();
-        ++n_df;
-        if (++st == K::STAGES) {
-          st = 0;
-          r_phase ^= 1;
-        }
       }
+      st = st_next;
+      r_phase = ph_next;
       ++n_items;
     }
   }
@@ -775,59 +846,73 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
     setmaxnreg_inc<kQLargeRegs>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row of the tile (TMEM lane)
-    const int tid = threadIdx.x - 128;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_base = tmem + lane_off;
-    uint32_t n_sdp = 0, n_acc = 0, n_job = 0;
+    // this warp's lse / D buffers: [2][48] each
+    float* wL = wstage + quarter * (2 * 2 * 48);
+    float* wD = wL + 2 * 48;
+    uint32_t n_sdp = 0, n_pd = 0, n_acc = 0, n_job = 0;
     int islot = 0;
     uint32_t iphase = 0;
     const float c2 = P.scale_log2;
     while (!*sh.abort_flag) {
       int i;
       if (!next_item(sh, P, islot, iphase, i) || i < 0) break;
-      const KItem it = decode_k(P, i);
+      const KItem it = decode_k<TQJ>(P, i);
       const int u = it.kt * TK + row;  // key position
       const bool key_ok = u < P.T;
       bool ok = true;
-      // a job's per-query lse and D (threads 0..63 load one value of each), one job ahead
-      auto fetch = [&](int jj, float& lv, float& dv) {
+      // a job's lse and D: lane l loads queries l and l + 32 (< TQJ), one job ahead
+      auto fetch = [&](int jj, float (&lv)[2], float (&dv)[2]) {
         int ss, qq_t;
-        job_of(P, it, jj, ss, qq_t);
-        const int qq = qq_t * K::TQJ + (tid & 63);
-        const int64_t idx = (int64_t)ss * P.M + (int64_t)it.b * P.T + qq;
-        lv = qq < P.T ? P.lse[idx] : 0.f;
-        dv = qq < P.T ? P.dsum[idx] : 0.f;
+        job_of<TQJ>(P, it, jj, ss, qq_t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = lane + 32 * h;
+          const int qq = qq_t * TQJ + c;
+          const bool in = c < TQJ && qq < P.T;
+          const int64_t idx = (int64_t)ss * P.M + (int64_t)it.b * P.T + qq;
+          lv[h] = in ? P.lse[idx] : 0.f;
+          dv[h] = in ? P.dsum[idx] : 0.f;
+        }
       };
-      float nl = 0.f, nd = 0.f;
-      if (tid < 64) fetch(0, nl, nd);
+      float nl[2], nd[2];
+      fetch(0, nl, nd);
       for (int j = 0; j < it.nj; ++j, ++n_job) {
         int s, qt;
-        job_of(P, it, j, s, qt);
-        const int buf = n_job & 1;
-        float* sL = sh.sL + buf * 128;
-        float* sD = sh.sD + buf * 128;
-        if (tid < 64) {
-          sL[tid] = nl;
-          sD[tid] = nd;
-          if (j + 1 < it.nj) fetch(j + 1, nl, nd);
+        job_of<TQJ>(P, it, j, s, qt);
+        float* sL = wL + (n_job & 1) * 48;
+        float* sD = wD + (n_job & 1) * 48;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = lane + 32 * h;
+          if (c < TQJ) {
+            sL[c] = nl[h];
+            sD[c] = nd[h];
+          }
         }
-        mbar_arrive(&sh.l_bar[buf]);
-        if (!warp_wait(&sh.l_bar[buf], (n_job >> 1) & 1, P, sh.abort_flag)) { ok = false; break; }
+        __syncwarp();  // this warp's buffer is complete (the other buffer is two jobs old)
+        if (j + 1 < it.nj) fetch(j + 1, nl, nd);
         if (!warp_wait(sh.sdp_full, n_sdp & 1, P, sh.abort_flag)) { ok = false; break; }
         ++n_sdp;
         tc_fence_after();
-        const int q0 = qt * K::TQJ;
+        const int q0 = qt * TQJ;
         // live queries of this key: q < T, and q >= u when causal
         const int qlo = P.causal ? u : 0;
-        const bool all_live = key_ok && q0 >= qlo && q0 + K::TQJ <= P.T;
-        uint32_t pp[32], pd[32];
+        const bool all_live = key_ok && q0 >= qlo && q0 + TQJ <= P.T;
+        uint32_t pp[TQJ / 2], pd[TQJ / 2];
         {
-          uint32_t sr[64], dr[64];
-          tmem_ld64_wait(t_base + K::S_COL, sr);
-          tmem_ld64_wait(t_base + K::DP_COL, dr);
+          uint32_t sr[TQJ], dr[TQJ];
+          tmem_ldN_wait<TQJ>(t_base + K::S_COL, sr);
+          tmem_ldN_wait<TQJ>(t_base + K::DP_COL, dr);
+          if (j + 1 < it.nj) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sh.s_free);
+          }
           if (all_live) {
 #pragma unroll
-            for (int x4 = 0; x4 < 16; ++x4) {
+            for (int x4 = 0; x4 < TQJ / 4; ++x4) {
               const float4 L4 = reinterpret_cast<const float4*>(sL)[x4];
               const float4 D4 = reinterpret_cast<const float4*>(sD)[x4];
               const float p0 = fast_exp2(fmaf(__uint_as_float(sr[4 * x4]), c2, -L4.x));
@@ -843,7 +928,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
             }
           } else {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
+            for (int x = 0; x < TQJ / 2; ++x) {
               const int c = 2 * x;
               float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
               const int qa = q0 + c, qb = q0 + c + 1;
@@ -860,10 +945,17 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
             }
           }
         }
-        // P^T and dS^T over the columns just read (the MMA warp issues nothing into them
-        // until this job's products are done)
-        store_packed32(t_base + K::S_COL, pp);
-        store_packed32(t_base + K::DP_COL, pd);
+        // the previous job's products have read P^T and dS^T: they may be overwritten
+        if (n_pd > 0 && !warp_wait(sh.d_free, (n_pd - 1) & 1, P, sh.abort_flag)) {
+          ok = false;
+          break;
+        }
+        ++n_pd;
+#pragma unroll
+        for (int c0 = 0; c0 < TQJ / 2; c0 += 8) {
+          tmem_st8(t_base + K::P_COL + c0, pp + c0);
+          tmem_st8(t_base + K::DS_COL + c0, pd + c0);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -925,8 +1017,10 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
               tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
               tmap_bf16_chunked(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
               tmap_bf16_chunked(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
-              tmap_bf16_chunked(&P.tm_q64, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 64, sw) &&
-              tmap_bf16_chunked(&P.tm_do64, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 64, sw);
+              tmap_bf16_chunked(&P.tm_qj, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW,
+                                KCfg<DH>::TQJ, sw) &&
+              tmap_bf16_chunked(&P.tm_doj, bb.dO, DH, (uint64_t)S * M, DH, C::CW,
+                                KCfg<DH>::TQJ, sw);
   if (!P.chunked &&
       (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
        !tmap_bf16_2d_ext(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
@@ -934,8 +1028,10 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
        !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
        !tmap_bf16_2d_ext(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
        !tmap_bf16_2d_ext(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_q64, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 64, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_do64, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 64, sw)))
+       !tmap_bf16_2d_ext(&P.tm_qj, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, KCfg<DH>::TQJ,
+                         sw) ||
+       !tmap_bf16_2d_ext(&P.tm_doj, bb.dO, DH, (uint64_t)S * M, DH, C::CW, KCfg<DH>::TQJ,
+                         sw)))
     return -1;
   P.lse = h->ws.lse;
   P.dsum = bb.dsum;
@@ -956,7 +1052,6 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   P.has_shared = has_shared;
   P.causal = causal;
   P.nq = (T + TQ - 1) / TQ;
-  P.nq64 = (T + 63) / 64;
   P.scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
   P.scale = 1.f / sqrtf((float)DH);
   P.status = h->ws.status;
