@@ -1,5 +1,6 @@
-// C ABI of the GQE attention forward library: argument checks, the workspace, and the
-// launch sequence on the caller's stream. The layer it computes is the one described in
+// C ABI of the GQE attention library (forward, decode step, group range): argument checks,
+// the workspace, and the launch sequence on the caller's stream. The backward pass's entry
+// points are in backward.cu. The layer it computes is the one described in
 // "GQE: Grouped Query Experts" (FrontiersMindAI/GQE README, Algorithm Overview and
 // Parameters) with the output construction of the gist.science summary (Methodology,
 // Output Construction).

@@ -230,7 +230,9 @@ attention_kernel(const T* __restrict__ Q, const T* __restrict__ Kc, const T* __r
 }
 
 // Variant gqe: the renormalised slot rho_t = sum_s w[t, s] * O[t, s] over the routed
-// streams, read back from Z's routed blocks and written to Z's slot block.
+// streams, read back from Z's routed blocks and written to Z's slot block. The slot weights
+// are the whole layer's [M, w_stride]; a handle restricted to a group range reads its
+// streams' columns from w_off on, so the ranges' slots sum to the layer's.
 // One thread per 16 bytes of the slot (8 bf16 or 4 fp32 values): 16-byte loads of every
 // routed block, fp32 accumulation, one 16-byte store.
 template <typename T>

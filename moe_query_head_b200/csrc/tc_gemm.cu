@@ -9,6 +9,8 @@
 //                     selected (token, expert) pairs are projected (README, Algorithm
 //                     Overview: only the active query-head computation is reduced).
 //   output projection Z [M, D_o] times W_o [dim, D_o].
+// A handle restricted to a group range (gqe_set_group_range) projects only its heads' K / V
+// and its experts' buckets (still routing every group in the dense projection).
 //
 // One persistent kernel, two CTAs per SM (each CTA's pipeline hand-offs, fills and tail are
 // covered by the other CTA's work):
