@@ -154,7 +154,7 @@ def test_backward_unsupported_shapes():
     G.gqe_destroy(h)
 
 
-@pytest.mark.parametrize("name", ["long_t16k", "main_b8_t2048"])
+@pytest.mark.parametrize("name", ["long_t16k", "main_b8_t2048", "wide_k2"])
 def test_backward_full_size_last_rows(name):
     """At the benchmark's full sizes, in its launch configuration: the input gradient of the
     last 256 positions of every sequence against the oracle's row-restricted backward (which

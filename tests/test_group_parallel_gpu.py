@@ -70,3 +70,31 @@ def test_group_range_errors():
         GQ.gqe_set_group_range(h, 0, 2)
     assert e.value.status == GQ.GQE_ERR_UNSUPPORTED
     GQ.gqe_destroy(h)
+
+
+def test_group_shards_full_size_sampled():
+    """The long-context workload split over 2 ranks, at full size, on sampled rows of the
+    summed output against the oracle's rows (routing bit-exact on every rank)."""
+    from moe_query_head_b200 import gqe as GQ
+    from tests.gqe_testlib import oracle_rows, sample_rows
+    wl = W.WORKLOADS["long_t16k"]
+    inp = W.cached("long_t16k")
+    d = {n: to_device(inp, n) for n in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")}
+    rows = sample_rows(wl)
+    ref = oracle_rows(inp, rows)
+    total = torch.zeros((wl.M, wl.dim), dtype=torch.float32, device="cuda")
+    for g0, g1 in GP.group_ranges(wl.G, 2):
+        sh = GP.GroupShard(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, variant=wl.variant,
+                           causal=wl.causal, max_tokens=wl.M, g0=g0, g1=g1, W_r=d["W_r"],
+                           W_q=d["W_q"], W_k=d["W_k"], W_v=d["W_v"], W_shared=d["W_shared"],
+                           W_o=d["W_o"])
+        out = torch.empty((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+        sh.forward(d["x"], wl.B, wl.T, out)
+        assert GQ.gqe_check_device_status(sh.h) == GQ.GQE_OK
+        total += out.float()
+        counts = torch.empty((wl.N,), dtype=torch.int32, device="cuda")
+        GQ.gqe_get_routing(sh.h, counts=counts)
+        torch.cuda.synchronize()
+        assert np.array_equal(counts.cpu().numpy(), ref["routing"].counts.astype(np.int32))
+        sh.close()
+    check_output(total.cpu().numpy().astype(np.float64)[rows], ref["y"], "bf16")
