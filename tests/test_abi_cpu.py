@@ -63,6 +63,11 @@ def test_null_handle_paths():
         == G.GQE_ERR_INVALID_ARG
     assert G.lib.gqe_check_device_status(None, None) == G.GQE_ERR_INVALID_ARG
     assert G.lib.gqe_kernel_launches(None) == -1
+    assert G.lib.gqe_set_group_range(None, 0, 1) == G.GQE_ERR_INVALID_ARG
+    assert G.lib.gqe_enable_backward(None) == G.GQE_ERR_INVALID_ARG
+    assert G.lib.gqe_backward(None, z, 1, 1, z, z, z, z, z, z, 16, 8, 1, 48, 0, 1, z, 0.0, z, z,
+                              z, z, z, z, z, None) == G.GQE_ERR_INVALID_ARG
+    assert G.lib.gqe_backward_launches(None) == -1
     G.lib.gqe_destroy(None)
 
 
