@@ -12,8 +12,8 @@
 //
 // The work is HBM-bound (every cached K/V row is read once, shared by all query streams of
 // its group), so it runs on CUDA cores. CTA (chunk c, group g, sequence b) streams its key
-// range in tiles of 64 rows through a cp.async ring in shared memory (rows padded by 16
-// bytes). Each of the four warps takes 16 keys of every tile for all of the group's queries,
+// range in tiles of 64 rows through a two-stage cp.async ring in shared memory (rows padded
+// by 16 bytes). Each of the four warps takes 16 keys of every tile for all of the group's queries,
 // so the work is spread evenly however few queries a group has (two at k = 1 in group 0,
 // one elsewhere): a score per (key, half of the head dims) lane pair, the online softmax
 // over the warp's keys with shuffles, P V with each lane owning pairs of head dimensions.
@@ -33,7 +33,7 @@ using tc::smem_u32;
 constexpr int THREADS = 128;
 constexpr int WARPS = THREADS / 32;
 constexpr int TKD = 64;      // keys per tile
-constexpr int STAGES = 3;    // tiles in flight
+constexpr int STAGES = 2;    // tiles in flight (two: the smaller footprint fits more CTAs per SM)
 constexpr int MAXQ = kMaxTopK + 1;
 constexpr int KPW = TKD / WARPS;  // keys of a tile per warp
 
