@@ -151,8 +151,9 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
  * with loss.backward()): allocate its backward workspace (cudaMalloc, on the current device;
  * the gradients of dZ, of the stream outputs and of the query, key and value projections
  * for max_tokens tokens, and a cuBLAS handle with its 32 MiB workspace). The
- * handle owns it until gqe_destroy. bf16 handles with d_h <= 64 only (GQE_ERR_UNSUPPORTED
- * otherwise); GQE_ERR_CUDA if an allocation fails. Calling it again does nothing.
+ * handle owns it until gqe_destroy. bf16 handles only (every head dim they accept, 16 to 128;
+ * GQE_ERR_UNSUPPORTED for float32 handles); GQE_ERR_CUDA if an allocation fails. Calling it
+ * again does nothing.
  */
 gqe_status gqe_enable_backward(gqe_handle h);
 

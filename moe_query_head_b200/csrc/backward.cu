@@ -56,7 +56,8 @@ __device__ __forceinline__ float bf16_round(float v) {
 
 constexpr int kCombWarps = 8;
 
-// One warp per token; lane l holds head dims l and l + 32 (d_h <= 64).
+// One warp per token; lane l holds head dims l, l + 32, l + 64 and l + 96 (d_h <= 128).
+constexpr int kDimsPerLane = 4;
 __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const CombBwd P) {
   __shared__ float s_g[kCombWarps][kMaxExperts];  // per routed stream: dw (gqe) / dp (wc)
   pdl_wait();
@@ -65,51 +66,51 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
   const int64_t t = (int64_t)blockIdx.x * kCombWarps + wi;
   if (t >= P.M) return;
   const int DH = P.d_h;
-  const bool v0 = lane < DH, v1 = lane + 32 < DH;
+  bool v[kDimsPerLane];
+#pragma unroll
+  for (int h = 0; h < kDimsPerLane; ++h) v[h] = lane + 32 * h < DH;
   const float* dz = P.dZ + t * P.Do;
   const __nv_bfloat16* z = P.Z + t * P.Do;
   const bool gqe = P.variant == GQE_VARIANT_GQE;
   const bool wcat = P.variant == GQE_VARIANT_WEIGHTED_CONCAT;
-  float ds0 = 0.f, ds1 = 0.f;  // the slot's gradient
-  if (gqe) {
-    const int c = P.Sr * DH;
-    ds0 = v0 ? dz[c + lane] : 0.f;
-    ds1 = v1 ? dz[c + lane + 32] : 0.f;
-  }
+  float ds[kDimsPerLane];  // the slot's gradient
+#pragma unroll
+  for (int h = 0; h < kDimsPerLane; ++h)
+    ds[h] = (gqe && v[h]) ? dz[P.Sr * DH + lane + 32 * h] : 0.f;
   float* g = s_g[wi];
   // routed streams
   for (int s = 0; s < P.Sr; ++s) {
     const int c = s * DH;
-    float o0 = v0 ? __bfloat162float(z[c + lane]) : 0.f;
-    float o1 = v1 ? __bfloat162float(z[c + lane + 32]) : 0.f;
-    const float b0 = v0 ? dz[c + lane] : 0.f;
-    const float b1 = v1 ? dz[c + lane + 32] : 0.f;
-    float d0, d1, gs = 0.f;
-    if (wcat) {
-      // Z holds p O: O = Z / p; dO = p dZ; dp = <dZ, O>
-      const float p = P.psel[t * P.Sr + s];
-      o0 /= p;
-      o1 /= p;
-      d0 = p * b0;
-      d1 = p * b1;
-      gs = warp_sum(b0 * o0 + b1 * o1);
-    } else if (gqe) {
-      // dO = dZ + w dslot; dw = <dslot, O>
-      const float ww = P.w[t * P.Sr + s];
-      d0 = fmaf(ww, ds0, b0);
-      d1 = fmaf(ww, ds1, b1);
-      gs = warp_sum(ds0 * o0 + ds1 * o1);
-    } else {
-      d0 = b0;
-      d1 = b1;
+    float o[kDimsPerLane], d[kDimsPerLane];
+    float gs = 0.f, dd = 0.f;
+    const float p = wcat ? P.psel[t * P.Sr + s] : 1.f;
+    const float ww = gqe ? P.w[t * P.Sr + s] : 0.f;
+#pragma unroll
+    for (int h = 0; h < kDimsPerLane; ++h) {
+      o[h] = v[h] ? __bfloat162float(z[c + lane + 32 * h]) : 0.f;
+      const float b = v[h] ? dz[c + lane + 32 * h] : 0.f;
+      if (wcat) {
+        // Z holds p O: O = Z / p; dO = p dZ; dp = <dZ, O>
+        o[h] /= p;
+        d[h] = p * b;
+        gs += b * o[h];
+      } else if (gqe) {
+        // dO = dZ + w dslot; dw = <dslot, O>
+        d[h] = fmaf(ww, ds[h], b);
+        gs += ds[h] * o[h];
+      } else {
+        d[h] = b;
+      }
+      // D from the bf16 dO the attention backward reads
+      d[h] = bf16_round(d[h]);
+      dd += d[h] * o[h];
     }
-    // D from the bf16 dO the attention backward reads
-    d0 = bf16_round(d0);
-    d1 = bf16_round(d1);
-    const float D = warp_sum(d0 * o0 + d1 * o1);
+    gs = (wcat || gqe) ? warp_sum(gs) : 0.f;
+    const float D = warp_sum(dd);
     __nv_bfloat16* dst = P.dO + ((int64_t)s * P.M + t) * DH;
-    if (v0) dst[lane] = __float2bfloat16_rn(d0);
-    if (v1) dst[lane + 32] = __float2bfloat16_rn(d1);
+#pragma unroll
+    for (int h = 0; h < kDimsPerLane; ++h)
+      if (v[h]) dst[lane + 32 * h] = __float2bfloat16_rn(d[h]);
     if (lane == 0) {
       P.dsum[(int64_t)s * P.M + t] = D;
       g[s] = gs;
@@ -117,14 +118,18 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
   }
   if (P.has_shared) {
     const int c = P.shared_col;
-    const float o0 = v0 ? __bfloat162float(z[c + lane]) : 0.f;
-    const float o1 = v1 ? __bfloat162float(z[c + lane + 32]) : 0.f;
-    const float d0 = v0 ? bf16_round(dz[c + lane]) : 0.f;
-    const float d1 = v1 ? bf16_round(dz[c + lane + 32]) : 0.f;
-    const float D = warp_sum(d0 * o0 + d1 * o1);
+    float d[kDimsPerLane], dd = 0.f;
+#pragma unroll
+    for (int h = 0; h < kDimsPerLane; ++h) {
+      const float o = v[h] ? __bfloat162float(z[c + lane + 32 * h]) : 0.f;
+      d[h] = v[h] ? bf16_round(dz[c + lane + 32 * h]) : 0.f;
+      dd += d[h] * o;
+    }
+    const float D = warp_sum(dd);
     __nv_bfloat16* dst = P.dO + ((int64_t)P.Sr * P.M + t) * DH;
-    if (v0) dst[lane] = __float2bfloat16_rn(d0);
-    if (v1) dst[lane + 32] = __float2bfloat16_rn(d1);
+#pragma unroll
+    for (int h = 0; h < kDimsPerLane; ++h)
+      if (v[h]) dst[lane + 32 * h] = __float2bfloat16_rn(d[h]);
     if (lane == 0) P.dsum[(int64_t)P.Sr * P.M + t] = D;
   }
   __syncwarp();

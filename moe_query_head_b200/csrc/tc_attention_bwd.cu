@@ -10,8 +10,9 @@
 //   dV = sum over the head's streams of P^T dO.
 //
 // Two kernels, neither with atomics (every output row is written by one CTA, so the result
-// is the same from run to run), each at two CTAs per SM (256 TMEM columns each; warpgroup 0
-// gives registers to the softmax warpgroup):
+// is the same from run to run). Head dims up to 64 run two CTAs per SM (256 TMEM columns
+// each; warpgroup 0 gives registers to the softmax warpgroup), larger ones (80 to 128) one
+// CTA per SM with 512 columns and the whole register file:
 //   attn_bwd_dq_kernel    work item = (sequence, stream, 128-query tile); per 64-key step
 //                         S = Q K^T and dP = dO V^T (both operands from shared memory) into
 //                         TMEM, the softmax warpgroup forms dS in bf16 in TMEM, and
@@ -20,14 +21,15 @@
 //                         row t of dQ_exp [M, N d_h] at the column block of its expert
 //                         g E + sel[t, g, r]; the shared stream in dQ_sh [M, d_h].
 //   attn_bwd_dkdv_kernel  work item = (sequence, KV head, 128-key tile); per job (a stream
-//                         that reads the head, a tile of 48 queries, 32 at d_h = 64),
+//                         that reads the head, a tile of 48 queries; 32 at d_h = 64, 64
+//                         above),
 //                         S^T = K Q^T and dP^T = V dO^T into TMEM, the softmax warpgroup
 //                         (one key per thread) forms P^T and dS^T in bf16 in TMEM, and
 //                         dV += P^T dO, dK += dS^T Q accumulate in TMEM over all of the
 //                         head's streams. dK, dV land token-major in [M, G d_h].
 // Warps: 0 TMA loads, 1 TMEM owner and MMA issue, 2-3 idle, 4-7 softmax and epilogue; the
 // next tile's S and dP are issued as soon as the softmax warps hold the current ones in
-// registers. Persistent CTAs take items heaviest first. Head dims up to 64.
+// registers. Persistent CTAs take items heaviest first. Head dims 16 to 128.
 #include <cudaTypedefs.h>
 
 #include "gqe_common.cuh"
@@ -52,25 +54,19 @@ constexpr int TK = 128;  // key rows of a tile
 
 template <int DH>
 struct BCfg {
-  static_assert(DH % 16 == 0 && DH <= 64, "the backward kernels take head dims up to 64");
-  // the forward's chunking: 64-column chunks (128-byte swizzle) for 64, else 16-column
-  // chunks (32-byte swizzle)
+  static_assert(DH % 16 == 0 && DH <= 128, "the backward kernels take head dims up to 128");
+  // shared-memory chunking: 64-column chunks (128-byte swizzle) for multiples of 64, else
+  // 16-column chunks (32-byte swizzle)
   static constexpr int CW = (DH % 64 == 0) ? 64 : 16;
   static constexpr int NC = DH / CW;
   static constexpr uint32_t LAYOUT = CW == 64 ? kSwizzle128B : kSwizzle32B;
   static constexpr int ROW_BYTES = CW * 2;
   static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;
   static constexpr int TILE_BYTES = 128 * DH * 2;
-  static constexpr int STAGES = 2;  // ring of tile pairs
-  // two fixed tiles, the ring of pairs, alignment, barriers, lse / D buffers
-  static constexpr int SMEM = 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 512 + 2 * 2 * 128 * 4;
-  static constexpr int TMEM_COLS = 512;
+  // CTAs per SM: two while each CTA's TMEM fits in 256 columns
+  static constexpr int CTAS = DH <= 64 ? 2 : 1;
+  static constexpr int TMEM_COLS = CTAS == 2 ? 256 : 512;
 };
-
-// TMEM columns. dQ kernel: S, dP (fp32), dS (bf16 pairs), dQ (fp32).
-constexpr int Q_S = 0, Q_DP = 128, Q_DS = 256, Q_DQ = 320;
-// dK / dV kernel: S^T, dP^T (fp32), P^T, dS^T (bf16 pairs), dV, dK (fp32, up to 64 each).
-constexpr int K_S = 0, K_DP = 128, K_P = 256, K_DS = 320, K_DV = 384, K_DK = 448;
 
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // Q, dO [S M, d_h]; K, V [G M, d_h]; 128-row boxes
@@ -300,17 +296,19 @@ struct QCfg {
   static constexpr int KT_BYTES = TKD * DH * 2;      // one 64-row K or V tile
   static constexpr int STAGES = 3;
   static constexpr int SMEM = 2 * C::TILE_BYTES + STAGES * 2 * KT_BYTES + 1024 + 512 + 2048;
-  static constexpr int TMEM_COLS = 256;
+  static constexpr int CTAS = C::CTAS;
+  static constexpr int TMEM_COLS = C::TMEM_COLS;
   static constexpr int S_COL = 0, DP_COL = 64, DS_COL = 128, DQ_COL = 160;
   static_assert(DQ_COL + DH <= TMEM_COLS, "TMEM budget");
-  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
 };
 constexpr int kQSmallRegs = 48, kQLargeRegs = 208;
 static_assert(kQSmallRegs * 128 + kQLargeRegs * 128 == THREADS * (65536 / (2 * THREADS)),
               "register split must equal the launch allocation");
 
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
+__global__ void __launch_bounds__(THREADS, QCfg<DH>::CTAS)
+attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
   using C = BCfg<DH>;
   using Q = QCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
@@ -338,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_co
   pdl_allow_next();
 
   if (warp < 4) {
-  setmaxnreg_dec<kQSmallRegs>();
+  if constexpr (C::CTAS == 2) setmaxnreg_dec<kQSmallRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------------ loads
     if (lane == 0) {
@@ -462,7 +460,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_co
   }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    setmaxnreg_inc<kQLargeRegs>();
+    if constexpr (C::CTAS == 2) setmaxnreg_inc<kQLargeRegs>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -584,7 +582,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dq_kernel(const __grid_co
 // most query tiles). Jobs of an item: every (stream reading g, query tile at or after the
 // key tile when causal).
 // ---------------------------------------------------------------------------------------
-// TMEM -> registers, N consecutive 32-bit columns per lane (N = 32 or 48), and the wait
+// TMEM -> registers, N consecutive 32-bit columns per lane (N = 32, 48 or 64), and the wait
 // for them in the same statement.
 __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -622,10 +620,12 @@ __device__ __forceinline__ void tmem_ld48_wait(uint32_t taddr, uint32_t (&r)[48]
 }
 template <int N>
 __device__ __forceinline__ void tmem_ldN_wait(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N == 32 || N == 48 || N == 64, "TMEM row widths of a job");
   if constexpr (N == 32) tmem_ld32_wait(taddr, r);
-  else tmem_ld48_wait(taddr, r);
+  else if constexpr (N == 48) tmem_ld48_wait(taddr, r);
+  else tmem_ld64_wait(taddr, r);
 }
-// bf16 pairs of a packed row -> TMEM, N/2 columns (N = 32 or 48), 8 columns per store
+// bf16 pairs of a packed row -> TMEM, 8 columns per store
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
@@ -633,25 +633,28 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// The dK / dV kernel runs two CTAs per SM with jobs of TQJ queries (48 for head dims up to
-// 48, 32 for 64), small enough that S^T, dP^T, P^T, dS^T, dV and dK all have TMEM columns
-// of their own within 256: the next job's S^T and dP^T are issued as soon as the softmax
-// warps hold the current ones in registers, as in the dQ kernel.
+// The dK / dV kernel runs jobs of TQJ queries small enough that S^T, dP^T, P^T, dS^T, dV
+// and dK all have TMEM columns of their own: at two CTAs per SM (256 columns) 48 queries for
+// head dims up to 48 and 32 for 64; at one CTA per SM (512 columns, head dims above 64) 64.
+// The next job's S^T and dP^T are issued as soon as the softmax warps hold the current
+// ones in registers, as in the dQ kernel.
 template <int DH>
 struct KCfg {
   using C = BCfg<DH>;
-  static constexpr int TQJ = DH <= 48 ? 48 : 32;    // queries per job
+  static constexpr int TQJ = DH <= 48 ? 48 : (DH <= 64 ? 32 : 64);  // queries per job
   static constexpr int QT_BYTES = TQJ * DH * 2;     // one Q or dO tile of the job
   static constexpr int STAGES = 3;
-  static constexpr int WARP_STAGE = 4 * 2 * 2 * 48 * 4;  // per-warp lse / D buffers
+  static constexpr int WARP_STAGE = 4 * 2 * 2 * TQJ * 4;  // per-warp lse / D buffers
   static constexpr int SMEM =
       2 * C::TILE_BYTES + STAGES * 2 * QT_BYTES + 1024 + 512 + 2048 + WARP_STAGE;
-  static constexpr int TMEM_COLS = 256;
+  static constexpr int CTAS = C::CTAS;
+  static constexpr int TMEM_COLS = C::TMEM_COLS;
   static constexpr int S_COL = 0, DP_COL = TQJ, P_COL = 2 * TQJ, DS_COL = 2 * TQJ + TQJ / 2;
   static constexpr int DV_COL = 3 * TQJ, DK_COL = 3 * TQJ + DH;
+  static_assert(TQJ % 16 == 0 && TQJ <= 64, "a job's queries: two per lane at most");
   static_assert(DK_COL + DH <= TMEM_COLS, "TMEM budget");
   static_assert(DP_COL % 16 == 0 && DV_COL % 16 == 0 && DK_COL % 16 == 0, "accumulator columns");
-  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static_assert(CTAS * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
 };
 
 struct KItem {
@@ -683,7 +686,8 @@ __device__ __forceinline__ void job_of(const BwdParams& P, const KItem& it, int 
 }
 
 template <int DH>
-__global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
+__global__ void __launch_bounds__(THREADS, KCfg<DH>::CTAS)
+attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams P) {
   using C = BCfg<DH>;
   using K = KCfg<DH>;
   constexpr int TQJ = K::TQJ;
@@ -714,7 +718,7 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
   pdl_allow_next();
 
   if (warp < 4) {
-  setmaxnreg_dec<kQSmallRegs>();
+  if constexpr (C::CTAS == 2) setmaxnreg_dec<kQSmallRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------------ loads
     if (lane == 0) {
@@ -843,14 +847,14 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
   }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    setmaxnreg_inc<kQLargeRegs>();
+    if constexpr (C::CTAS == 2) setmaxnreg_inc<kQLargeRegs>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row of the tile (TMEM lane)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_base = tmem + lane_off;
-    // this warp's lse / D buffers: [2][48] each
-    float* wL = wstage + quarter * (2 * 2 * 48);
-    float* wD = wL + 2 * 48;
+    // this warp's lse / D buffers: [2][TQJ] each
+    float* wL = wstage + quarter * (2 * 2 * TQJ);
+    float* wD = wL + 2 * TQJ;
     uint32_t n_sdp = 0, n_pd = 0, n_acc = 0, n_job = 0;
     int islot = 0;
     uint32_t iphase = 0;
@@ -881,8 +885,8 @@ __global__ void __launch_bounds__(THREADS, 2) attn_bwd_dkdv_kernel(const __grid_
       for (int j = 0; j < it.nj; ++j, ++n_job) {
         int s, qt;
         job_of<TQJ>(P, it, j, s, qt);
-        float* sL = wL + (n_job & 1) * 48;
-        float* sD = wD + (n_job & 1) * 48;
+        float* sL = wL + (n_job & 1) * TQJ;
+        float* sD = wD + (n_job & 1) * TQJ;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int c = lane + 32 * h;
@@ -1059,14 +1063,15 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   P.counter = bb.counter;
   // dQ
   P.items = B * S * P.nq;
-  int grid = P.items < 2 * h->num_sms ? P.items : 2 * h->num_sms;  // two CTAs per SM
+  const int per_sm = C::CTAS * h->num_sms;  // persistent CTAs
+  int grid = P.items < per_sm ? P.items : per_sm;
   if (launch_pdl(attn_bwd_dq_kernel<DH>, dim3(grid), dim3(THREADS), QCfg<DH>::SMEM, st, P) !=
       cudaSuccess)
     return -1;
   // dK, dV
   P.items = B * h->G * P.nq;
   P.counter = bb.counter + 2;
-  grid = P.items < 2 * h->num_sms ? P.items : 2 * h->num_sms;  // two CTAs per SM
+  grid = P.items < per_sm ? P.items : per_sm;
   if (launch_pdl(attn_bwd_dkdv_kernel<DH>, dim3(grid), dim3(THREADS), KCfg<DH>::SMEM, st, P) !=
       cudaSuccess)
     return -1;
@@ -1076,7 +1081,7 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
 }  // namespace
 
 bool tc_backward_supported(const gqe_ctx* h) {
-  return h->dtype == GQE_BF16 && h->d_h <= 64;
+  return h->dtype == GQE_BF16 && h->d_h <= 128;
 }
 
 int launch_tc_attention_backward(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S,
@@ -1086,6 +1091,10 @@ int launch_tc_attention_backward(gqe_ctx* h, const BwdBuffers& bb, int B, int T,
     case 32: return launch_bwd_dh<32>(h, bb, B, T, S, has_shared, causal, st);
     case 48: return launch_bwd_dh<48>(h, bb, B, T, S, has_shared, causal, st);
     case 64: return launch_bwd_dh<64>(h, bb, B, T, S, has_shared, causal, st);
+    case 80: return launch_bwd_dh<80>(h, bb, B, T, S, has_shared, causal, st);
+    case 96: return launch_bwd_dh<96>(h, bb, B, T, S, has_shared, causal, st);
+    case 112: return launch_bwd_dh<112>(h, bb, B, T, S, has_shared, causal, st);
+    case 128: return launch_bwd_dh<128>(h, bb, B, T, S, has_shared, causal, st);
     default: return -1;
   }
 }

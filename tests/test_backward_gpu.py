@@ -11,7 +11,8 @@ cancel and raise the relative error; it gets the same bound, checked on the gqe 
 whose slot feeds it and on the aux term alone.
 
 Cases: several query and key tiles with a ragged tail, causal and not, the three variants,
-head dims 16 / 32 / 48 / 64, three experts per group, no shared head, and the aux loss's
+every head dim the bf16 path accepts (16 to 64 on the two-CTA-per-SM kernels, 80 to 128 on
+the one-CTA-per-SM ones), three experts per group, no shared head, and the aux loss's
 gradient alone (dy = 0)."""
 import numpy as np
 import pytest
@@ -91,6 +92,11 @@ CASES = {
     "experts_3_per_group": MAIN.with_(B=1, T=200, N=12, G=4, k=1),
     "dh16": MAIN.with_(B=1, T=200, d_h=16),
     "dh32": MAIN.with_(B=2, T=150, d_h=32),
+    "dh80": MAIN.with_(B=1, T=300, d_h=80),
+    "dh96_noncausal": MAIN.with_(B=2, T=150, d_h=96, causal=False),
+    "dh112_weighted": MAIN.with_(B=1, T=260, d_h=112, variant="weighted_concat"),
+    "dh128": MAIN.with_(B=1, T=300, d_h=128),
+    "dh128_noncausal_k2": WIDE.with_(dim=768, B=1, T=200, d_h=128, causal=False),
 }
 
 
@@ -146,15 +152,16 @@ def test_backward_deterministic_and_requires_matching_forward():
 
 
 def test_backward_unsupported_shapes():
+    """float32 handles (the CUDA-core path) have no backward."""
     from moe_query_head_b200 import gqe as G
-    h = G.gqe_create(768, 16, 8, 1, 128, G.GQE_BF16, 64)
+    h = G.gqe_create(64, 4, 2, 1, 16, G.GQE_F32, 64)
     with pytest.raises(G.GQEError) as e:
         G.gqe_enable_backward(h)
     assert e.value.status == G.GQE_ERR_UNSUPPORTED
     G.gqe_destroy(h)
 
 
-@pytest.mark.parametrize("name", ["long_t16k", "main_b8_t2048", "wide_k2"])
+@pytest.mark.parametrize("name", ["long_t16k", "main_b8_t2048", "wide_k2", "large_skew"])
 def test_backward_full_size_last_rows(name):
     """At the benchmark's full sizes, in its launch configuration: the input gradient of the
     last 256 positions of every sequence against the oracle's row-restricted backward (which
