@@ -106,6 +106,8 @@ WORKLOADS = {
     "long_t64k": Workload("long_t64k", dim=768, N=16, G=8, k=1, d_h=48, B=1, T=65536, seed=6),
     "long_t128k": Workload("long_t128k", dim=768, N=16, G=8, k=1, d_h=48, B=1, T=131072,
                            seed=7),
+    "long_t1m": Workload("long_t1m", dim=768, N=16, G=8, k=1, d_h=48, B=1, T=1048576,
+                         seed=8),
     # Large and skewed: 70% of tokens to expert 0 of each group.
     "large_skew": Workload("large_skew", dim=4096, N=32, G=8, k=1, d_h=128, B=1, T=32768,
                            seed=5, skew=0.70),

@@ -103,11 +103,18 @@ FULL = {
     "wide_k2_hard": dict(variant="hard_concat"),
     "large_skew": {},
     "long_t64k": {},
+    "long_t1m": {},
 }
+# host memory the oracle's float64 rows need at 1M tokens (x, K and V over every token)
+HOST_BYTES = {"long_t1m": 40 << 30}
 
 
 @pytest.mark.parametrize("case", list(FULL))
 def test_full_size_sampled(case):
+    if case in HOST_BYTES:
+        import psutil
+        if psutil.virtual_memory().available < HOST_BYTES[case]:
+            pytest.skip("not enough host memory for the oracle's float64 rows")
     name = case if case in W.WORKLOADS else "wide_k2"
     inp = W.cached(name, **FULL[case]) if FULL[case] else W.cached(name)
     wl = inp.wl
