@@ -149,6 +149,16 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def wait_first(self, timeout: float = 5.0):
+        """Returns once nvidia-smi has written its first sample (or after `timeout` s), so
+        the samples cover the timed region however slowly the tool starts."""
+        t_end = time.time() + timeout
+        while self.proc is not None and time.time() < t_end:
+            self.file.flush()
+            if os.path.getsize(self.file.name) > 0:
+                return
+            time.sleep(0.05)
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -341,7 +351,8 @@ def bench_ours(args, rank, world, dist):
         raise RuntimeError("device status after warm-up: " + G.status_str(st))
 
     sampler = ClockSampler(gpu_id)
-    time.sleep(0.3)
+    sampler.wait_first()
+    time.sleep(0.1)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -575,7 +586,8 @@ def bench_decode(args, rank, world, dist):
     if st != G.GQE_OK:
         raise RuntimeError("device status after warm-up: " + G.status_str(st))
     sampler = ClockSampler(gpu_id)
-    time.sleep(0.3)
+    sampler.wait_first()
+    time.sleep(0.1)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -710,7 +722,8 @@ def bench_backward(args, rank, world, dist):
     if G.gqe_check_device_status(h) != G.GQE_OK:
         raise RuntimeError("device status after warm-up")
     sampler = ClockSampler(gpu_id)
-    time.sleep(0.3)
+    sampler.wait_first()
+    time.sleep(0.1)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -801,7 +814,8 @@ def bench_groups(args, rank, world, dist):
     gpu_id = torch.cuda.get_device_properties(torch.cuda.current_device()).uuid
     gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id)
     sampler = ClockSampler(gpu_id)
-    time.sleep(0.3)
+    sampler.wait_first()
+    time.sleep(0.1)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()

@@ -187,8 +187,49 @@ gqe_status gqe_backward(gqe_handle h, const void* x, int B, int T, const void* W
                         const void* dy, float aux_grad, float* dx, float* dW_r, float* dW_q,
                         float* dW_k, float* dW_v, float* dW_shared, float* dW_o, void* stream);
 
-/* gqe_backward_launches — kernels of this library the last gqe_backward launched (the cuBLAS
- * GEMMs are not counted). */
+/*
+ * gqe_backward_begin / gqe_backward_finish — the backward pass in two phases, for a handle
+ * restricted to a group range (gqe_set_group_range) as well as for a whole layer; gqe_backward
+ * is the two in one call on a whole layer.
+ *
+ * The group-parallel split (one range per GPU, the layer's y the sum of the ranges' shares)
+ * keeps the backward local to each range except for one number per token: the gqe slot
+ * weights w = p_sel / P_t divide by the selected probabilities of ALL groups (gist.science
+ * summary, Output Construction), so the router gradient of every range needs
+ * <dslot, slot> = sum over all routed streams of w_s <dslot, O_s>. begin writes this range's
+ * share of it, the caller sums the shares over the ranges (an all-reduce of B*T floats, which
+ * may overlap begin's attention backward on another stream), and finish takes the sum.
+ *
+ * begin: the arguments of gqe_backward up to dy, then
+ *   slot_dot  [B*T] float32, device, 4-byte aligned: written (zero for the weighted_concat
+ *             and hard_concat variants, whose router gradient needs no exchange).
+ * finish: the same arguments, aux_grad, slot_dot (the sum over the ranges; for a whole layer
+ * begin's own output), then the gradients as gqe_backward, each this range's share, in the
+ * shapes of the weights this handle was given: dW_q [(g1-g0)*E*d_h, dim], dW_k, dW_v
+ * [(g1-g0)*d_h, dim], dW_shared (the range holding group 0, with W_shared), dW_o [dim, D_o of
+ * this range's Z], dW_r [N, dim] (zero outside the range's experts) and dx [B*T, dim]; the
+ * layer's gradients are the sums of the shares (dW_o's slot columns are a share of the
+ * slot's; every other block belongs to one range).
+ *
+ * finish must follow a successful begin on the same handle with the same arguments, with no
+ * gqe_forward or gqe_decode between them (GQE_ERR_INVALID_ARG otherwise). Both enqueue on
+ * `stream`, allocate nothing and do not synchronise. Errors as gqe_backward.
+ */
+gqe_status gqe_backward_begin(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                              const void* W_q, const void* W_k, const void* W_v,
+                              const void* W_shared, const void* W_o, int N, int G, int k,
+                              int d_h, int variant, int causal, const void* dy, float* slot_dot,
+                              void* stream);
+gqe_status gqe_backward_finish(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                               const void* W_q, const void* W_k, const void* W_v,
+                               const void* W_shared, const void* W_o, int N, int G, int k,
+                               int d_h, int variant, int causal, const void* dy, float aux_grad,
+                               const float* slot_dot, float* dx, float* dW_r, float* dW_q,
+                               float* dW_k, float* dW_v, float* dW_shared, float* dW_o,
+                               void* stream);
+
+/* gqe_backward_launches — kernels of this library the last gqe_backward (or begin and finish)
+ * launched (the cuBLAS GEMMs are not counted). */
 int gqe_backward_launches(gqe_handle h);
 
 /*
@@ -237,8 +278,9 @@ gqe_status gqe_check_device_status(gqe_handle h, void* stream);
  * all-reduce or reduce-scatter over the ranks). K, V, the query streams and Z of
  * gqe_get_tensor hold the range's heads only. bf16 handles whose routing runs in the dense
  * projection (N a power of two up to 32) only, else GQE_ERR_UNSUPPORTED; gqe_decode and
- * gqe_backward return GQE_ERR_UNSUPPORTED unless the range is the whole layer
- * (gqe_set_group_range(h, 0, G) restores it). GQE_ERR_INVALID_ARG unless 0 <= g0 < g1 <= G.
+ * the one-call gqe_backward return GQE_ERR_UNSUPPORTED unless the range is the whole layer
+ * (gqe_set_group_range(h, 0, G) restores it); a range trains with gqe_backward_begin /
+ * gqe_backward_finish. GQE_ERR_INVALID_ARG unless 0 <= g0 < g1 <= G.
  */
 gqe_status gqe_set_group_range(gqe_handle h, int g0, int g1);
 

@@ -269,6 +269,9 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   h->last_variant = variant;
   h->last_causal = causal;
   h->last_shared = has_shared;
+  h->last_g0 = h->g0;
+  h->last_g1 = h->g1;
+  h->bwd_begun = 0;
   return ok ? GQE_OK : GQE_ERR_CUDA;
 }
 
@@ -332,6 +335,7 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
   h->last_Do = Do;
   h->last_launches = launches;
   h->last_kind = ok ? 2 : 0;
+  h->bwd_begun = 0;
   return ok ? GQE_OK : GQE_ERR_CUDA;
 }
 

@@ -1,21 +1,33 @@
-// Backward pass of one GQE attention layer: gqe_enable_backward and gqe_backward.
+// Backward pass of one GQE attention layer: gqe_enable_backward, gqe_backward and its two
+// phases gqe_backward_begin / gqe_backward_finish.
 //
 // Training adds the load-balancing loss to the task loss and back-propagates through the
 // layer ("GQE: Grouped Query Experts" README, Usage); the renormalised slot gives the router
 // a differentiable path (gist.science summary, Output Construction). Given dy = dF/dy and the
 // aux coefficient dA, the gradients of F = <dy, y> + dA L are formed in this order:
-//   1. dZ = dy W_o and dW_o = dy^T Z                         (plain GEMMs, cuBLAS)
+//   phase 1 (begin)
+//   1. dZ = dy W_o                                              (plain GEMM, cuBLAS)
 //   2. combine_bwd_kernel, one warp per token: the stream gradients dO from dZ by variant
-//      (routed blocks, the slot's share w dslot, the shared block), D = rowsum(dO * O), the
-//      selected probabilities' gradients (slot weights with their denominator, or the raw p
-//      of weighted_concat), the aux term dA (E/G) f / M on every p, and the per-group
-//      softmax Jacobian: the router logits' gradient dl [M, N]
+//      (routed blocks, the slot's share w dslot, the shared block), D = rowsum(dO * O), and
+//      per routed stream dw = <dslot, O> (gqe) or dp = <dZ, O> (weighted_concat); for gqe
+//      also <dslot, slot> = sum over the streams of w dw
 //   3. the attention backward (tc_attention_bwd.cu): dQ into dQ_exp [M, N d_h] (each routed
 //      row at the column block of its expert, zero elsewhere) and dQ_sh, dK and dV [M, G d_h]
-//   4. the weight gradients dW = (gradient)^T x and dx = sum of (gradient) W over the router,
-//      the N query heads (dQ_exp: the unselected heads' blocks are zero, so one dense GEMM
-//      serves every expert), the K, V and shared projections (plain GEMMs, cuBLAS)
+//   phase 2 (finish)
+//   4. router_bwd_kernel, one warp per token: the selected probabilities' gradients (for gqe
+//      the slot weights w = p_sel / P_t differentiated with their denominator:
+//      dp_sel = (dw - <dslot, slot>) / P_t), the aux term dA (E/G) f / M on every p, and the
+//      per-group softmax Jacobian: the router logits' gradient dl [M, N]
+//   5. dW_o = dy^T Z, the weight gradients dW = (gradient)^T x and dx = sum of (gradient) W
+//      over the router, the query heads (dQ_exp: the unselected heads' blocks are zero, so one
+//      dense GEMM serves every expert), the K, V and shared projections (plain GEMMs, cuBLAS)
 // The top-k selection is held constant (its sets are the forward's).
+//
+// A handle restricted to groups [g0, g1) (gqe_set_group_range) computes its share: every
+// step above is local to its groups except <dslot, slot>, which sums over all of the
+// layer's streams; phase 1 writes this handle's share of it, the caller sums the shares over
+// the ranges, and phase 2 takes the sum. The router gradient of the other groups is zero
+// here, so the layer's gradients are the sums of the ranges' shares.
 #include <cublas_v2.h>
 #include <string.h>
 
@@ -26,17 +38,23 @@ namespace gqe {
 namespace {
 
 struct CombBwd {
-  const float* dZ;          // [M, Do]
+  const float* dZ;          // [M, Do] this handle's Z columns
   const __nv_bfloat16* Z;   // [M, Do]
-  const float* psel;        // [M, G k]
-  const float* w;           // [M, G k]
-  const int32_t* sel;       // [M, G k]
+  const float* psel;        // [M, gk] the layer's routing (every group)
+  const float* w;           // [M, gk]
+  const int32_t* sel;       // [M, gk]
   const float* logits;      // [M, N]
   const int32_t* counts;    // [N]
-  __nv_bfloat16* dO;        // [S, M, d_h]
+  __nv_bfloat16* dO;        // [S, M, d_h] this handle's streams
   float* dsum;              // [S, M]
+  float* dgs;               // [M, Sr] per routed stream of this handle: dw (gqe), dp (weighted)
+  float* slot_dot;          // [M] phase 1: this handle's share of <dslot, slot>
+  const float* slot_dot_in; // [M] phase 2: the sum over the layer's ranges
   __nv_bfloat16* dl;        // [M, N]
-  int M, N, G, E, k, Sr, d_h, Do, variant, has_shared, shared_col;
+  int M, N, G, E, k, d_h, Do, variant, has_shared, shared_col;
+  int gk;                   // G k: row stride of the routing arrays
+  int g0, g1;               // this handle's groups
+  int Sr;                   // its routed streams, (g1 - g0) k, numbered from group g0
   float dA;
 };
 
@@ -56,10 +74,10 @@ __device__ __forceinline__ float bf16_round(float v) {
 
 constexpr int kCombWarps = 8;
 
-// One warp per token; lane l holds head dims l, l + 32, l + 64 and l + 96 (d_h <= 128).
+// Phase 1, one warp per token; lane l holds head dims l, l + 32, l + 64 and l + 96
+// (d_h <= 128).
 constexpr int kDimsPerLane = 4;
 __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const CombBwd P) {
-  __shared__ float s_g[kCombWarps][kMaxExperts];  // per routed stream: dw (gqe) / dp (wc)
   pdl_wait();
   pdl_allow_next();
   const int wi = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -73,18 +91,19 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
   const __nv_bfloat16* z = P.Z + t * P.Do;
   const bool gqe = P.variant == GQE_VARIANT_GQE;
   const bool wcat = P.variant == GQE_VARIANT_WEIGHTED_CONCAT;
+  const int64_t rt = t * P.gk + (int64_t)P.g0 * P.k;  // this handle's first stream's routing
   float ds[kDimsPerLane];  // the slot's gradient
 #pragma unroll
   for (int h = 0; h < kDimsPerLane; ++h)
     ds[h] = (gqe && v[h]) ? dz[P.Sr * DH + lane + 32 * h] : 0.f;
-  float* g = s_g[wi];
+  float dot = 0.f;  // <dslot, slot> over this handle's streams: sum of w dw
   // routed streams
   for (int s = 0; s < P.Sr; ++s) {
     const int c = s * DH;
     float o[kDimsPerLane], d[kDimsPerLane];
     float gs = 0.f, dd = 0.f;
-    const float p = wcat ? P.psel[t * P.Sr + s] : 1.f;
-    const float ww = gqe ? P.w[t * P.Sr + s] : 0.f;
+    const float p = wcat ? P.psel[rt + s] : 1.f;
+    const float ww = gqe ? P.w[rt + s] : 0.f;
 #pragma unroll
     for (int h = 0; h < kDimsPerLane; ++h) {
       o[h] = v[h] ? __bfloat162float(z[c + lane + 32 * h]) : 0.f;
@@ -106,6 +125,7 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
       dd += d[h] * o[h];
     }
     gs = (wcat || gqe) ? warp_sum(gs) : 0.f;
+    dot = fmaf(gs, ww, dot);
     const float D = warp_sum(dd);
     __nv_bfloat16* dst = P.dO + ((int64_t)s * P.M + t) * DH;
 #pragma unroll
@@ -113,9 +133,10 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
       if (v[h]) dst[lane + 32 * h] = __float2bfloat16_rn(d[h]);
     if (lane == 0) {
       P.dsum[(int64_t)s * P.M + t] = D;
-      g[s] = gs;
+      P.dgs[t * P.Sr + s] = gs;
     }
   }
+  if (lane == 0) P.slot_dot[t] = dot;
   if (P.has_shared) {
     const int c = P.shared_col;
     float d[kDimsPerLane], dd = 0.f;
@@ -132,22 +153,30 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
       if (v[h]) dst[lane + 32 * h] = __float2bfloat16_rn(d[h]);
     if (lane == 0) P.dsum[(int64_t)P.Sr * P.M + t] = D;
   }
-  __syncwarp();
-  // gradients of the selected probabilities
+}
+
+// Phase 2, one warp per token: the router logits' gradient of this handle's groups (zero
+// for the others).
+__global__ void __launch_bounds__(kCombWarps * 32) router_bwd_kernel(const CombBwd P) {
+  __shared__ float s_g[kCombWarps][kMaxExperts];  // per routed stream: dp_sel
+  pdl_wait();
+  pdl_allow_next();
+  const int wi = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t t = (int64_t)blockIdx.x * kCombWarps + wi;
+  if (t >= P.M) return;
+  const bool gqe = P.variant == GQE_VARIANT_GQE;
+  const bool wcat = P.variant == GQE_VARIANT_WEIGHTED_CONCAT;
+  float* g = s_g[wi];
   if (gqe) {
-    // w = p_sel / P_t: dp_sel = (dw - sum(dw w)) / P_t
-    float pt = 0.f, dww = 0.f;
-    for (int s = lane; s < P.Sr; s += 32) {
-      const float ww = P.w[t * P.Sr + s];
-      pt += P.psel[t * P.Sr + s];
-      dww += g[s] * ww;
-    }
+    // w = p_sel / P_t over the layer's G k selections: dp_sel = (dw - sum(dw w)) / P_t,
+    // sum(dw w) = <dslot, slot>
+    float pt = 0.f;
+    for (int s = lane; s < P.gk; s += 32) pt += P.psel[t * P.gk + s];
     pt = warp_sum(pt);
-    dww = warp_sum(dww);
-    __syncwarp();
-    for (int s = lane; s < P.Sr; s += 32) g[s] = (g[s] - dww) / pt;
-  } else if (!wcat) {
-    for (int s = lane; s < P.Sr; s += 32) g[s] = 0.f;
+    const float dot = P.slot_dot_in[t];
+    for (int s = lane; s < P.Sr; s += 32) g[s] = (P.dgs[t * P.Sr + s] - dot) / pt;
+  } else {
+    for (int s = lane; s < P.Sr; s += 32) g[s] = wcat ? P.dgs[t * P.Sr + s] : 0.f;
   }
   __syncwarp();
   // router logits: dp on every p of the group (selected terms and the aux term), then the
@@ -155,6 +184,13 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
   const float aux_c = P.dA * (float)P.E / (float)P.G / ((float)P.M * (float)P.k * (float)P.M);
   for (int gg = 0; gg < P.G; ++gg) {
     const int e0 = gg * P.E;
+    if (gg < P.g0 || gg >= P.g1) {
+      // another range's group
+      for (int j = lane; j < P.E; j += 32) P.dl[t * P.N + e0 + j] = __float2bfloat16_rn(0.f);
+      continue;
+    }
+    const int32_t* sl = P.sel + t * P.gk + gg * P.k;  // the group's selections
+    const float* gsel = g + (gg - P.g0) * P.k;          // and their dp_sel
     for (int jb = 0; jb < P.E; jb += 32) {
       const int j = jb + lane;
       const bool in = j < P.E;
@@ -169,7 +205,7 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
       const float p = in ? expf(l - mx) / den : 0.f;
       float dp = in ? aux_c * (float)P.counts[e0 + j] : 0.f;
       for (int r = 0; r < P.k; ++r)
-        if (in && P.sel[t * P.Sr + gg * P.k + r] == j) dp += g[gg * P.k + r];
+        if (in && sl[r] == j) dp += gsel[r];
       // sum over the group of p dp
       float spd = 0.f;
       for (int jj = lane; jj < P.E; jj += 32) {
@@ -177,7 +213,7 @@ __global__ void __launch_bounds__(kCombWarps * 32) combine_bwd_kernel(const Comb
         const float pj = expf(lj - mx) / den;
         float dpj = aux_c * (float)P.counts[e0 + jj];
         for (int r = 0; r < P.k; ++r)
-          if (P.sel[t * P.Sr + gg * P.k + r] == jj) dpj += g[gg * P.k + r];
+          if (sl[r] == jj) dpj += gsel[r];
         spd += pj * dpj;
       }
       spd = warp_sum(spd);
@@ -220,12 +256,166 @@ size_t bwd_layout(BwdBuffers& b, char* base, const gqe_ctx* h) {
   b.dq_sh = (__nv_bfloat16*)take((size_t)M * h->d_h * 2);
   b.dk = (__nv_bfloat16*)take((size_t)M * h->G * h->d_h * 2);
   b.dv = (__nv_bfloat16*)take((size_t)M * h->G * h->d_h * 2);
+  b.dgs = (float*)take((size_t)M * h->G * h->k * 4);
+  b.slot_dot = (float*)take((size_t)M * 4);
   b.counter = (int*)take(16 * sizeof(int));
   b.cublas_ws = take(kCublasWorkspace);
   return off;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Sizes of one backward call on this handle's groups.
+struct BwdCall {
+  int M, S, Do, Sr, Gl, Nl, has_shared;
+};
+
+// The arguments both phases take: checked against the handle and its last forward (which
+// must be a gqe_forward with the same x, weights, B, T, variant, causal, presence of W_shared
+// and group range).
+gqe_status check_call(const gqe_ctx* h, const void* x, int B, int T, const void* W_r,
+                      const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
+                      const void* W_o, int N, int G, int k, int d_h, int variant, int causal,
+                      const void* dy, BwdCall& c) {
+  if (!h->bwd_base) return GQE_ERR_INVALID_ARG;  // gqe_enable_backward first
+  if (N != h->N || G != h->G || k != h->k || d_h != h->d_h) return GQE_ERR_INVALID_ARG;
+  if (B < 1 || T < 1) return GQE_ERR_INVALID_ARG;
+  if (variant < GQE_VARIANT_GQE || variant > GQE_VARIANT_HARD_CONCAT) return GQE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return GQE_ERR_INVALID_ARG;
+  if (!x || !W_r || !W_q || !W_k || !W_v || !W_o || !dy) return GQE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_r, W_q, W_k, W_v, W_o, dy};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return GQE_ERR_INVALID_ARG;
+  if (W_shared && !aligned16(W_shared)) return GQE_ERR_INVALID_ARG;
+  const int64_t M64 = (int64_t)B * T;
+  if (M64 > h->max_tokens) return GQE_ERR_WORKSPACE;
+  c.M = (int)M64;
+  c.has_shared = W_shared != nullptr;
+  // the saved state must be this layer's last forward, on the same groups
+  if (h->last_kind != 1 || h->last_M != c.M || h->last_B != B || h->last_T != T ||
+      h->last_variant != variant || h->last_causal != causal ||
+      h->last_shared != c.has_shared || h->last_g0 != h->g0 || h->last_g1 != h->g1)
+    return GQE_ERR_INVALID_ARG;
+  c.Gl = h->g1 - h->g0;
+  c.Sr = c.Gl * k;
+  c.Nl = c.Gl * h->E;
+  c.S = c.Sr + c.has_shared;
+  c.Do = (c.Sr + (variant == GQE_VARIANT_GQE ? 1 : 0) + c.has_shared) * d_h;
+  return GQE_OK;
+}
+
+CombBwd comb_args(const gqe_ctx* h, const BwdCall& c, int variant, float aux_grad) {
+  const BwdBuffers& b = h->bwd;
+  CombBwd a;
+  memset(&a, 0, sizeof(a));
+  a.dZ = b.dZ;
+  a.Z = static_cast<const __nv_bfloat16*>(h->ws.Z);
+  a.psel = h->ws.psel;
+  a.w = h->ws.w;
+  a.sel = h->ws.sel;
+  a.logits = h->ws.logits;
+  a.counts = h->ws.counts;
+  a.dO = b.dO;
+  a.dsum = b.dsum;
+  a.dgs = b.dgs;
+  a.dl = b.dl;
+  a.M = c.M;
+  a.N = h->N;
+  a.G = h->G;
+  a.E = h->E;
+  a.k = h->k;
+  a.d_h = h->d_h;
+  a.Do = c.Do;
+  a.variant = variant;
+  a.has_shared = c.has_shared;
+  a.shared_col = (c.Sr + (variant == GQE_VARIANT_GQE ? 1 : 0)) * h->d_h;
+  a.gk = h->G * h->k;
+  a.g0 = h->g0;
+  a.g1 = h->g1;
+  a.Sr = c.Sr;
+  a.dA = aux_grad;
+  return a;
+}
+
+// Phase 1: dZ, the stream gradients and this handle's share of <dslot, slot> (slot_dot
+// [M], device), the attention backward.
+gqe_status phase1(gqe_ctx* h, const BwdCall& c, int B, int T, const void* W_o, int variant,
+                  int causal, const void* dy, float* slot_dot, cudaStream_t st) {
+  cublasHandle_t hb = static_cast<cublasHandle_t>(h->cublas);
+  if (cublasSetStream(hb, st) != CUBLAS_STATUS_SUCCESS) return GQE_ERR_CUDA;
+  const BwdBuffers& b = h->bwd;
+  const int dim = h->dim, d_h = h->d_h;
+  int launches = 0;
+  bool ok = gemm_rm(hb, false, false, c.M, c.Do, dim, dy, dim, W_o, c.Do, b.dZ, c.Do, 0.f);
+  // dQ_exp is zero outside the selected heads' blocks
+  ok = ok && cudaMemsetAsync(b.dq_exp, 0, (size_t)c.M * c.Nl * d_h * 2, st) == cudaSuccess;
+  if (ok) {
+    CombBwd a = comb_args(h, c, variant, 0.f);
+    a.slot_dot = slot_dot;
+    combine_bwd_kernel<<<(c.M + kCombWarps - 1) / kCombWarps, kCombWarps * 32, 0, st>>>(a);
+    ok = cudaGetLastError() == cudaSuccess;
+    ++launches;
+  }
+  if (ok) {
+    const int n = launch_tc_attention_backward(h, b, B, T, c.S, c.has_shared, causal, st);
+    ok = n >= 0;
+    launches += n > 0 ? n : 0;
+  }
+  h->last_bwd_launches = launches;
+  h->bwd_begun = ok ? 1 : 0;
+  h->bwd_M = c.M;
+  h->bwd_variant = variant;
+  return ok ? GQE_OK : GQE_ERR_CUDA;
+}
+
+// Phase 2: the router backward with <dslot, slot> summed over the layer (slot_dot_in [M],
+// device), dW_o, the weight gradients and dx.
+gqe_status phase2(gqe_ctx* h, const BwdCall& c, const void* x, const void* W_r,
+                  const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
+                  int variant, const void* dy, float aux_grad, const float* slot_dot_in,
+                  float* dx, float* dW_r, float* dW_q, float* dW_k, float* dW_v,
+                  float* dW_shared, float* dW_o, cudaStream_t st) {
+  if (!h->bwd_begun || h->bwd_M != c.M || h->bwd_variant != variant) return GQE_ERR_INVALID_ARG;
+  h->bwd_begun = 0;
+  cublasHandle_t hb = static_cast<cublasHandle_t>(h->cublas);
+  if (cublasSetStream(hb, st) != CUBLAS_STATUS_SUCCESS) return GQE_ERR_CUDA;
+  const BwdBuffers& b = h->bwd;
+  const int dim = h->dim, d_h = h->d_h, N = h->N, M = c.M;
+  bool ok = true;
+  {
+    CombBwd a = comb_args(h, c, variant, aux_grad);
+    a.slot_dot_in = slot_dot_in;
+    router_bwd_kernel<<<(M + kCombWarps - 1) / kCombWarps, kCombWarps * 32, 0, st>>>(a);
+    ok = cudaGetLastError() == cudaSuccess;
+    ++h->last_bwd_launches;
+  }
+  const int Nd = c.Nl * d_h, Gd = c.Gl * d_h;
+  ok = ok && gemm_rm(hb, true, false, dim, c.Do, M, dy, dim, h->ws.Z, c.Do, dW_o, c.Do, 0.f);
+  ok = ok && gemm_rm(hb, true, false, Nd, dim, M, b.dq_exp, Nd, x, dim, dW_q, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dk, Gd, x, dim, dW_k, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dv, Gd, x, dim, dW_v, dim, 0.f);
+  ok = ok && gemm_rm(hb, true, false, N, dim, M, b.dl, N, x, dim, dW_r, dim, 0.f);
+  if (c.has_shared)
+    ok = ok && gemm_rm(hb, true, false, d_h, dim, M, b.dq_sh, d_h, x, dim, dW_shared, dim, 0.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Nd, b.dq_exp, Nd, W_q, dim, dx, dim, 0.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dk, Gd, W_k, dim, dx, dim, 1.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dv, Gd, W_v, dim, dx, dim, 1.f);
+  ok = ok && gemm_rm(hb, false, false, M, dim, N, b.dl, N, W_r, dim, dx, dim, 1.f);
+  if (c.has_shared)
+    ok = ok && gemm_rm(hb, false, false, M, dim, d_h, b.dq_sh, d_h, W_shared, dim, dx, dim, 1.f);
+  return ok ? GQE_OK : GQE_ERR_CUDA;
+}
+
+bool outputs_ok(const void* W_shared, const float* dx, const float* dW_r, const float* dW_q,
+                const float* dW_k, const float* dW_v, const float* dW_shared,
+                const float* dW_o) {
+  if (!dx || !dW_r || !dW_q || !dW_k || !dW_v || !dW_o) return false;
+  if ((W_shared == nullptr) != (dW_shared == nullptr)) return false;
+  const void* outs[] = {dx, dW_r, dW_q, dW_k, dW_v, dW_o};
+  for (const void* p : outs)
+    if (!aligned16(p)) return false;
+  return !dW_shared || aligned16(dW_shared);
+}
 
 }  // namespace
 
@@ -279,92 +469,53 @@ gqe_status gqe_backward(gqe_handle h, const void* x, int B, int T, const void* W
                         const void* dy, float aux_grad, float* dx, float* dW_r, float* dW_q,
                         float* dW_k, float* dW_v, float* dW_shared, float* dW_o, void* stream) {
   if (!h) return GQE_ERR_INVALID_ARG;
-  if (!h->bwd_base) return GQE_ERR_INVALID_ARG;  // gqe_enable_backward first
-  if (h->g0 != 0 || h->g1 != h->G) return GQE_ERR_UNSUPPORTED;  // whole layers only
-  if (N != h->N || G != h->G || k != h->k || d_h != h->d_h) return GQE_ERR_INVALID_ARG;
-  if (B < 1 || T < 1) return GQE_ERR_INVALID_ARG;
-  if (variant < GQE_VARIANT_GQE || variant > GQE_VARIANT_HARD_CONCAT) return GQE_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return GQE_ERR_INVALID_ARG;
-  if (!x || !W_r || !W_q || !W_k || !W_v || !W_o || !dy || !dx || !dW_r || !dW_q || !dW_k ||
-      !dW_v || !dW_o)
+  // a part of the layer needs the sum of <dslot, slot> over the parts: the two phases
+  if (h->g0 != 0 || h->g1 != h->G) return GQE_ERR_UNSUPPORTED;
+  BwdCall c;
+  gqe_status r = check_call(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h,
+                            variant, causal, dy, c);
+  if (r != GQE_OK) return r;
+  if (!outputs_ok(W_shared, dx, dW_r, dW_q, dW_k, dW_v, dW_shared, dW_o))
     return GQE_ERR_INVALID_ARG;
-  if ((W_shared == nullptr) != (dW_shared == nullptr)) return GQE_ERR_INVALID_ARG;
-  const void* ptrs[] = {x, W_r, W_q, W_k, W_v, W_o, dy, dx, dW_r, dW_q, dW_k, dW_v, dW_o};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return GQE_ERR_INVALID_ARG;
-  if (W_shared && (!aligned16(W_shared) || !aligned16(dW_shared))) return GQE_ERR_INVALID_ARG;
-  const int64_t M64 = (int64_t)B * T;
-  if (M64 > h->max_tokens) return GQE_ERR_WORKSPACE;
-  const int M = (int)M64;
-  const int has_shared = W_shared != nullptr;
-  // the saved state must be this layer's last forward
-  if (h->last_kind != 1 || h->last_M != M || h->last_B != B || h->last_T != T ||
-      h->last_variant != variant || h->last_causal != causal || h->last_shared != has_shared)
-    return GQE_ERR_INVALID_ARG;
-  const int S = G * k + has_shared;
-  const int Do = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
-  const int dim = h->dim;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cublasHandle_t hb = static_cast<cublasHandle_t>(h->cublas);
-  if (cublasSetStream(hb, st) != CUBLAS_STATUS_SUCCESS) return GQE_ERR_CUDA;
-  const BwdBuffers& b = h->bwd;
-  int launches = 0;
-  bool ok = true;
-  // 1. dZ = dy W_o; dW_o = dy^T Z
-  ok = ok && gemm_rm(hb, false, false, M, Do, dim, dy, dim, W_o, Do, b.dZ, Do, 0.f);
-  ok = ok && gemm_rm(hb, true, false, dim, Do, M, dy, dim, h->ws.Z, Do, dW_o, Do, 0.f);
-  // 2. dQ_exp is zero outside the selected heads' blocks
-  ok = ok && cudaMemsetAsync(b.dq_exp, 0, (size_t)M * N * d_h * 2, st) == cudaSuccess;
-  if (ok) {
-    CombBwd c;
-    c.dZ = b.dZ;
-    c.Z = static_cast<const __nv_bfloat16*>(h->ws.Z);
-    c.psel = h->ws.psel;
-    c.w = h->ws.w;
-    c.sel = h->ws.sel;
-    c.logits = h->ws.logits;
-    c.counts = h->ws.counts;
-    c.dO = b.dO;
-    c.dsum = b.dsum;
-    c.dl = b.dl;
-    c.M = M;
-    c.N = N;
-    c.G = G;
-    c.E = h->E;
-    c.k = k;
-    c.Sr = G * k;
-    c.d_h = d_h;
-    c.Do = Do;
-    c.variant = variant;
-    c.has_shared = has_shared;
-    c.shared_col = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0)) * d_h;
-    c.dA = aux_grad;
-    combine_bwd_kernel<<<(M + kCombWarps - 1) / kCombWarps, kCombWarps * 32, 0, st>>>(c);
-    ok = cudaGetLastError() == cudaSuccess;
-    ++launches;
-  }
-  // 3. attention backward
-  if (ok) {
-    const int n = launch_tc_attention_backward(h, b, B, T, S, has_shared, causal, st);
-    ok = n >= 0;
-    launches += n > 0 ? n : 0;
-  }
-  // 4. weight gradients and dx
-  const int Nd = N * d_h, Gd = G * d_h;
-  ok = ok && gemm_rm(hb, true, false, Nd, dim, M, b.dq_exp, Nd, x, dim, dW_q, dim, 0.f);
-  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dk, Gd, x, dim, dW_k, dim, 0.f);
-  ok = ok && gemm_rm(hb, true, false, Gd, dim, M, b.dv, Gd, x, dim, dW_v, dim, 0.f);
-  ok = ok && gemm_rm(hb, true, false, N, dim, M, b.dl, N, x, dim, dW_r, dim, 0.f);
-  if (has_shared)
-    ok = ok && gemm_rm(hb, true, false, d_h, dim, M, b.dq_sh, d_h, x, dim, dW_shared, dim, 0.f);
-  ok = ok && gemm_rm(hb, false, false, M, dim, Nd, b.dq_exp, Nd, W_q, dim, dx, dim, 0.f);
-  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dk, Gd, W_k, dim, dx, dim, 1.f);
-  ok = ok && gemm_rm(hb, false, false, M, dim, Gd, b.dv, Gd, W_v, dim, dx, dim, 1.f);
-  ok = ok && gemm_rm(hb, false, false, M, dim, N, b.dl, N, W_r, dim, dx, dim, 1.f);
-  if (has_shared)
-    ok = ok && gemm_rm(hb, false, false, M, dim, d_h, b.dq_sh, d_h, W_shared, dim, dx, dim, 1.f);
-  h->last_bwd_launches = launches;
-  return ok ? GQE_OK : GQE_ERR_CUDA;
+  r = phase1(h, c, B, T, W_o, variant, causal, dy, h->bwd.slot_dot, st);
+  if (r != GQE_OK) return r;
+  return phase2(h, c, x, W_r, W_q, W_k, W_v, W_shared, variant, dy, aux_grad, h->bwd.slot_dot,
+                dx, dW_r, dW_q, dW_k, dW_v, dW_shared, dW_o, st);
+}
+
+gqe_status gqe_backward_begin(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                              const void* W_q, const void* W_k, const void* W_v,
+                              const void* W_shared, const void* W_o, int N, int G, int k,
+                              int d_h, int variant, int causal, const void* dy, float* slot_dot,
+                              void* stream) {
+  if (!h) return GQE_ERR_INVALID_ARG;
+  h->bwd_begun = 0;
+  BwdCall c;
+  const gqe_status r = check_call(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h,
+                                  variant, causal, dy, c);
+  if (r != GQE_OK) return r;
+  if (!slot_dot || (reinterpret_cast<uintptr_t>(slot_dot) & 3u)) return GQE_ERR_INVALID_ARG;
+  return phase1(h, c, B, T, W_o, variant, causal, dy, slot_dot, static_cast<cudaStream_t>(stream));
+}
+
+gqe_status gqe_backward_finish(gqe_handle h, const void* x, int B, int T, const void* W_r,
+                               const void* W_q, const void* W_k, const void* W_v,
+                               const void* W_shared, const void* W_o, int N, int G, int k,
+                               int d_h, int variant, int causal, const void* dy, float aux_grad,
+                               const float* slot_dot, float* dx, float* dW_r, float* dW_q,
+                               float* dW_k, float* dW_v, float* dW_shared, float* dW_o,
+                               void* stream) {
+  if (!h) return GQE_ERR_INVALID_ARG;
+  BwdCall c;
+  const gqe_status r = check_call(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h,
+                                  variant, causal, dy, c);
+  if (r != GQE_OK) return r;
+  if (!slot_dot || (reinterpret_cast<uintptr_t>(slot_dot) & 3u)) return GQE_ERR_INVALID_ARG;
+  if (!outputs_ok(W_shared, dx, dW_r, dW_q, dW_k, dW_v, dW_shared, dW_o))
+    return GQE_ERR_INVALID_ARG;
+  return phase2(h, c, x, W_r, W_q, W_k, W_v, W_shared, variant, dy, aux_grad, slot_dot, dx,
+                dW_r, dW_q, dW_k, dW_v, dW_shared, dW_o, static_cast<cudaStream_t>(stream));
 }
 
 int gqe_backward_launches(gqe_handle h) { return h ? h->last_bwd_launches : -1; }

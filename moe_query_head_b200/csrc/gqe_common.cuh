@@ -143,6 +143,8 @@ struct BwdBuffers {
   __nv_bfloat16* dq_sh = nullptr;     // [M, d_h] shared-head query gradient
   __nv_bfloat16* dk = nullptr;        // [M, G d_h] key gradients, token-major
   __nv_bfloat16* dv = nullptr;        // [M, G d_h] value gradients, token-major
+  float* dgs = nullptr;               // [M, G k] per routed stream: dw (gqe), dp (weighted)
+  float* slot_dot = nullptr;          // [M] <dslot, slot> of a whole-layer backward
   int* counter = nullptr;             // [4] work counters of the two attention kernels
   void* cublas_ws = nullptr;          // cuBLAS workspace
 };
@@ -168,7 +170,7 @@ struct gqe_ctx {
   // what the last call was (1 gqe_forward, 2 gqe_decode) and its arguments, which a
   // gqe_backward must repeat
   int last_kind = 0, last_B = 0, last_T = 0, last_variant = -1, last_causal = -1,
-      last_shared = -1;
+      last_shared = -1, last_g0 = -1, last_g1 = -1;
   int route_set = 0;  // the dense-projection routing's cursor set for the next call
   // backward pass (gqe_enable_backward)
   void* bwd_base = nullptr;
@@ -176,6 +178,9 @@ struct gqe_ctx {
   void* cublas = nullptr;  // cublasHandle_t
   gqe::BwdBuffers bwd;
   int last_bwd_launches = 0;
+  // the last gqe_backward_begin (checked by gqe_backward_finish): M, variant, and 1 once
+  // it succeeded
+  int bwd_begun = 0, bwd_M = 0, bwd_variant = -1;
 };
 
 namespace gqe {

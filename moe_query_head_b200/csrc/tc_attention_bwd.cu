@@ -74,12 +74,15 @@ struct BwdParams {
   CUtensorMap tm_qj, tm_doj;            // Q, dO with job-row boxes (the dK / dV kernel)
   const float* lse;     // [S, M]
   const float* dsum;    // [S, M] rowsum(dO * O)
-  const int32_t* sel;   // [M, G, k]
+  const int32_t* sel;   // [M, sel_stride]: stream s's selection at column sel_off + s
   __nv_bfloat16* dq_exp;  // [M, N d_h]
   __nv_bfloat16* dq_sh;   // [M, d_h]
   __nv_bfloat16* dk;      // [M, G d_h]
   __nv_bfloat16* dv;      // [M, G d_h]
+  // S, Sr, G, N: this handle's streams, routed streams, KV heads and experts (a group range
+  // counts from its first group)
   int M, T, B, S, Sr, k, G, E, N, has_shared, causal, nq, items, chunked;
+  int sel_stride, sel_off;
   float scale_log2;  // log2(e) / sqrt(d_h)
   float scale;       // 1 / sqrt(d_h)
   int* counter;      // [2] item counter and exit counter (zero at launch; reset by the last CTA)
@@ -544,7 +547,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams P) {
       if (valid) {
         if (it.s < P.Sr) {
           const int g = it.s / P.k;
-          const int e = g * P.E + P.sel[tok * (int64_t)P.Sr + it.s];
+          const int e = g * P.E + P.sel[tok * (int64_t)P.sel_stride + P.sel_off + it.s];
           dst = P.dq_exp + tok * (int64_t)P.N * DH + (int64_t)e * DH;
         } else {
           dst = P.dq_sh + tok * DH;
@@ -1011,16 +1014,18 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   if (!set_smem_limit_once<attn_bwd_dq_kernel<DH>>(QCfg<DH>::SMEM)) return -1;
   if (!set_smem_limit_once<attn_bwd_dkdv_kernel<DH>>(KCfg<DH>::SMEM)) return -1;
   const int M = B * T;
+  const int Gl = h->g1 - h->g0;  // this handle's KV heads
+  const uint64_t kv_rows = (uint64_t)Gl * M;
   BwdParams P;
   memset(&P, 0, sizeof(P));
   const CUtensorMapSwizzle sw = C::CW == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B;
   P.chunked = C::NC > 1 &&
               tmap_bf16_chunked(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
               tmap_bf16_chunked(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) &&
-              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
-              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) &&
-              tmap_bf16_chunked(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
-              tmap_bf16_chunked(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) &&
+              tmap_bf16_chunked(&P.tm_k, h->ws.K, DH, kv_rows, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_v, h->ws.V, DH, kv_rows, DH, C::CW, 128, sw) &&
+              tmap_bf16_chunked(&P.tm_k64, h->ws.K, DH, kv_rows, DH, C::CW, 64, sw) &&
+              tmap_bf16_chunked(&P.tm_v64, h->ws.V, DH, kv_rows, DH, C::CW, 64, sw) &&
               tmap_bf16_chunked(&P.tm_qj, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW,
                                 KCfg<DH>::TQJ, sw) &&
               tmap_bf16_chunked(&P.tm_doj, bb.dO, DH, (uint64_t)S * M, DH, C::CW,
@@ -1028,10 +1033,10 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   if (!P.chunked &&
       (!tmap_bf16_2d_ext(&P.tm_q, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
        !tmap_bf16_2d_ext(&P.tm_do, bb.dO, DH, (uint64_t)S * M, DH, C::CW, 128, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 128, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_k64, h->ws.K, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
-       !tmap_bf16_2d_ext(&P.tm_v64, h->ws.V, DH, (uint64_t)h->G * M, DH, C::CW, 64, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_k, h->ws.K, DH, kv_rows, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v, h->ws.V, DH, kv_rows, DH, C::CW, 128, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_k64, h->ws.K, DH, kv_rows, DH, C::CW, 64, sw) ||
+       !tmap_bf16_2d_ext(&P.tm_v64, h->ws.V, DH, kv_rows, DH, C::CW, 64, sw) ||
        !tmap_bf16_2d_ext(&P.tm_qj, h->ws.Q, DH, (uint64_t)S * M, DH, C::CW, KCfg<DH>::TQJ,
                          sw) ||
        !tmap_bf16_2d_ext(&P.tm_doj, bb.dO, DH, (uint64_t)S * M, DH, C::CW, KCfg<DH>::TQJ,
@@ -1048,11 +1053,13 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
   P.T = T;
   P.B = B;
   P.S = S;
-  P.Sr = h->G * h->k;
+  P.Sr = Gl * h->k;
   P.k = h->k;
-  P.G = h->G;
+  P.G = Gl;
   P.E = h->E;
-  P.N = h->N;
+  P.N = Gl * h->E;
+  P.sel_stride = h->G * h->k;
+  P.sel_off = h->g0 * h->k;
   P.has_shared = has_shared;
   P.causal = causal;
   P.nq = (T + TQ - 1) / TQ;
@@ -1069,7 +1076,7 @@ int launch_bwd_dh(gqe_ctx* h, const BwdBuffers& bb, int B, int T, int S, int has
       cudaSuccess)
     return -1;
   // dK, dV
-  P.items = B * h->G * P.nq;
+  P.items = B * Gl * P.nq;
   P.counter = bb.counter + 2;
   grid = P.items < per_sm ? P.items : per_sm;
   if (launch_pdl(attn_bwd_dkdv_kernel<DH>, dim3(grid), dim3(THREADS), KCfg<DH>::SMEM, st, P) !=

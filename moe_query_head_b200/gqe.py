@@ -25,7 +25,7 @@ EXPORTED = ("gqe_create", "gqe_forward", "gqe_get_routing", "gqe_get_tensor",
             "gqe_workspace_bytes", "gqe_kernel_launches", "gqe_set_stage_events",
             "gqe_stage_name", "gqe_route_static", "gqe_exp2_fma", "gqe_selftest_timeout",
             "gqe_decode", "gqe_enable_backward", "gqe_backward", "gqe_backward_launches",
-            "gqe_set_group_range")
+            "gqe_set_group_range", "gqe_backward_begin", "gqe_backward_finish")
 GQE_NUM_STAGES = 6
 
 
@@ -81,6 +81,11 @@ def _load() -> ctypes.CDLL:
     lib.gqe_backward.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P,
                                  ctypes.c_float, P, P, P, P, P, P, P, P]
     lib.gqe_backward.restype = I
+    lib.gqe_backward_begin.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.gqe_backward_begin.restype = I
+    lib.gqe_backward_finish.argtypes = [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P,
+                                        ctypes.c_float, P, P, P, P, P, P, P, P, P]
+    lib.gqe_backward_finish.restype = I
     lib.gqe_backward_launches.argtypes = [P]
     lib.gqe_backward_launches.restype = I
     return lib
@@ -153,6 +158,28 @@ def gqe_backward(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, va
                             float(aux_grad), _ptr(dx), _ptr(dW_r), _ptr(dW_q), _ptr(dW_k),
                             _ptr(dW_v), _ptr(dW_shared), _ptr(dW_o), _stream(stream)),
            "gqe_backward")
+
+
+def gqe_backward_begin(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, variant,
+                       causal, dy, slot_dot, stream=None) -> None:
+    """Phase 1 of the backward of a handle's last gqe_forward: writes this handle's share of
+    <dslot, slot> per token to slot_dot (float32 [B*T], device; see include/gqe.h)."""
+    _check(lib.gqe_backward_begin(h, _ptr(x), B, T, _ptr(W_r), _ptr(W_q), _ptr(W_k), _ptr(W_v),
+                                  _ptr(W_shared), _ptr(W_o), N, G, k, d_h, variant, causal,
+                                  _ptr(dy), _ptr(slot_dot), _stream(stream)),
+           "gqe_backward_begin")
+
+
+def gqe_backward_finish(h, x, B, T, W_r, W_q, W_k, W_v, W_shared, W_o, N, G, k, d_h, variant,
+                        causal, dy, aux_grad, slot_dot, dx, dW_r, dW_q, dW_k, dW_v, dW_shared,
+                        dW_o, stream=None) -> None:
+    """Phase 2: the gradients, given <dslot, slot> summed over the layer's group ranges."""
+    _check(lib.gqe_backward_finish(h, _ptr(x), B, T, _ptr(W_r), _ptr(W_q), _ptr(W_k),
+                                   _ptr(W_v), _ptr(W_shared), _ptr(W_o), N, G, k, d_h, variant,
+                                   causal, _ptr(dy), float(aux_grad), _ptr(slot_dot), _ptr(dx),
+                                   _ptr(dW_r), _ptr(dW_q), _ptr(dW_k), _ptr(dW_v),
+                                   _ptr(dW_shared), _ptr(dW_o), _stream(stream)),
+           "gqe_backward_finish")
 
 
 def gqe_backward_launches(h) -> int:

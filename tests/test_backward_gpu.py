@@ -151,6 +151,33 @@ def test_backward_deterministic_and_requires_matching_forward():
     run.close()
 
 
+def test_backward_two_phases_equal_one_call():
+    """On a whole layer, gqe_backward_begin with its own <dslot, slot> fed to
+    gqe_backward_finish gives exactly the one-call gqe_backward's gradients."""
+    from moe_query_head_b200 import gqe as G
+    wl = WIDE.with_(B=1, T=300)
+    inp = W.generate(wl)
+    dy = W.grad_output(wl)
+    run = GpuRun(inp).forward()
+    a = _gpu_backward(run, dy, 0.01)
+    d = run.dev
+    f32 = lambda *s: torch.full(s, float("nan"), dtype=torch.float32, device="cuda")  # noqa
+    g = dict(x=f32(wl.M, wl.dim), W_r=f32(wl.N, wl.dim), W_q=f32(wl.N * wl.d_h, wl.dim),
+             W_k=f32(wl.G * wl.d_h, wl.dim), W_v=f32(wl.G * wl.d_h, wl.dim),
+             W_shared=f32(wl.d_h, wl.dim), W_o=f32(wl.dim, wl.D_o))
+    sd = f32(wl.M)
+    args = (run.h, d["x"], wl.B, wl.T, d["W_r"], d["W_q"], d["W_k"], d["W_v"], d["W_shared"],
+            d["W_o"], wl.N, wl.G, wl.k, wl.d_h, W.VARIANT_IDS[wl.variant], int(wl.causal),
+            _bf16(dy))
+    G.gqe_backward_begin(*args, sd)
+    G.gqe_backward_finish(*args, 0.01, sd, g["x"], g["W_r"], g["W_q"], g["W_k"], g["W_v"],
+                          g["W_shared"], g["W_o"])
+    assert G.gqe_check_device_status(run.h) == G.GQE_OK
+    for k_, v in g.items():
+        assert np.array_equal(v.cpu().numpy().astype(np.float64), a[k_]), k_
+    run.close()
+
+
 def test_backward_unsupported_shapes():
     """float32 handles (the CUDA-core path) have no backward."""
     from moe_query_head_b200 import gqe as G

@@ -92,3 +92,45 @@ def test_shares_sum_to_the_layer_over_gloo(wl_name):
         p.join(timeout=60)
         assert p.exitcode == 0
     assert max(errs) < 1e-12, errs
+
+
+@pytest.mark.parametrize("variant", ["gqe", "weighted_concat", "hard_concat"])
+@pytest.mark.parametrize("shared", [True, False])
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_full_gradients_place_the_shares(variant, shared, world):
+    """A rank's gradient shares come in the shapes of its weight slices; full_gradients puts
+    them back at the rows and columns rank_weights took them from, zero elsewhere, so the
+    sum over the ranks of the slices of a full array rebuilds it (W_o's slot columns once per
+    rank: every rank holds a share of the slot's gradient)."""
+    N, G, k, d_h, dim = 16, 8, 2, 4, 6
+    E = N // G
+    D_o = (G * k + (variant == "gqe") + shared) * d_h
+    rng = np.random.default_rng(1)
+    A = {"W_q": rng.standard_normal((N * d_h, dim)), "W_k": rng.standard_normal((G * d_h, dim)),
+         "W_v": rng.standard_normal((G * d_h, dim)),
+         "W_shared": rng.standard_normal((d_h, dim)) if shared else None,
+         "W_o": rng.standard_normal((dim, D_o))}
+    x = rng.standard_normal((5, dim))
+    total = None
+    for g0, g1 in GP.group_ranges(G, world):
+        s = GP.rank_weights(A["W_q"], A["W_k"], A["W_v"], A["W_shared"], A["W_o"], N=N, G=G,
+                            k=k, d_h=d_h, variant=variant, g0=g0, g1=g1)
+        assert s["W_q"].shape == ((g1 - g0) * E * d_h, dim)
+        s = dict(s, x=x, W_r=np.zeros((N, dim)))
+        f = GP.full_gradients(s, N=N, G=G, k=k, d_h=d_h, variant=variant, shared=shared,
+                              D_o=D_o, g0=g0, g1=g1)
+        # zero outside the rank's rows
+        mask = np.ones(N * d_h, bool)
+        mask[g0 * E * d_h:g1 * E * d_h] = False
+        assert not f["W_q"][mask].any()
+        total = f if total is None else {n: (None if v is None else v + f[n])
+                                         for n, v in total.items()}
+    for n in ("W_q", "W_k", "W_v"):
+        assert np.array_equal(total[n], A[n]), n
+    if shared:
+        assert np.array_equal(total["W_shared"], A["W_shared"])
+    times = np.ones(D_o)
+    if variant == "gqe":
+        times[G * k * d_h:(G * k + 1) * d_h] = world
+    assert np.allclose(total["W_o"], A["W_o"] * times[None, :])
+    assert np.array_equal(total["x"], world * x)

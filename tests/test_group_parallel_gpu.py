@@ -4,7 +4,9 @@ run one after another, and their sum is checked against the float64 oracle's who
 y at the bf16 tolerances. Every share's routing and aux loss are the whole layer's
 (bit-exact routing, aux within 1e-4 relative). The shares run as separate launches with no
 waits between ranks, so one GPU can run them in turn; the multi-process sum itself is the
-NCCL all-reduce that group_parallel.GroupShard.forward_allreduce issues."""
+NCCL all-reduce that group_parallel.GroupShard.forward_allreduce issues. The backward on the
+split (gqe_backward_begin / gqe_backward_finish with the ranks' <dslot, slot> summed in
+between) is checked the same way against the oracle's whole-layer gradients."""
 import numpy as np
 import pytest
 import torch
@@ -98,3 +100,112 @@ def test_group_shards_full_size_sampled():
         assert np.array_equal(counts.cpu().numpy(), ref["routing"].counts.astype(np.int32))
         sh.close()
     check_output(total.cpu().numpy().astype(np.float64)[rows], ref["y"], "bf16")
+
+
+MAIN = W.WORKLOADS["main_b8_t2048"]
+WIDE = W.WORKLOADS["wide_k2"]
+BWD_CASES = {
+    "main_2_ranks": (MAIN.with_(B=1, T=300), 2),
+    "main_3_ranks_uneven": (MAIN.with_(B=2, T=150), 3),
+    "main_8_ranks_noncausal": (MAIN.with_(B=1, T=200, causal=False), 8),
+    "wide_gqe_2_ranks": (WIDE.with_(B=1, T=260), 2),
+    "wide_weighted_4_ranks": (WIDE.with_(B=1, T=200, variant="weighted_concat"), 4),
+    "main_hard_no_shared_2_ranks": (MAIN.with_(B=1, T=200, shared=False,
+                                               variant="hard_concat"), 2),
+    "dh128_2_ranks": (MAIN.with_(B=1, T=200, d_h=128), 2),
+}
+GRAD_REL_L2 = 1e-2  # as the whole-layer backward tests: bf16 dO, dQ, dK, dV and dl
+
+
+@pytest.mark.parametrize("case", list(BWD_CASES))
+def test_group_shards_backward_sums_to_the_layer(case):
+    """Training on the split: every rank's forward, then phase 1 on every rank, the ranks'
+    <dslot, slot> summed (what the all-reduce of GroupShard.backward_allreduce does), phase
+    2 on every rank; the ranks' gradient shares placed in the layer's shapes and summed give
+    the float64 oracle's gradients of <dy, y> + 0.01 aux for x and every weight."""
+    import oracle
+    from moe_query_head_b200 import gqe as GQ
+    from tests.gqe_testlib import rel_l2
+    wl, world = BWD_CASES[case]
+    inp = W.generate(wl)
+    d = {n: to_device(inp, n) for n in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")}
+    dy_h = W.grad_output(wl)
+    dy = torch.from_numpy(W.f32_to_bf16_bits(dy_h).view(np.int16)).view(torch.bfloat16).cuda()
+    f = inp.f64
+    layer = oracle.Layer(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, shared=wl.shared,
+                         variant=wl.variant, causal=wl.causal)
+    ref = oracle.backward(layer, f("x"), wl.B, wl.T, f("W_r"), f("W_q"), f("W_k"), f("W_v"),
+                          f("W_shared"), f("W_o"), dy_h.astype(np.float64), 0.01)
+    shards = []
+    for g0, g1 in GP.group_ranges(wl.G, world):
+        sh = GP.GroupShard(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, variant=wl.variant,
+                           causal=wl.causal, max_tokens=wl.M, g0=g0, g1=g1, W_r=d["W_r"],
+                           W_q=d["W_q"], W_k=d["W_k"], W_v=d["W_v"],
+                           W_shared=d["W_shared"] if wl.shared else None, W_o=d["W_o"])
+        sh.enable_backward()
+        out = torch.empty((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+        sh.forward(d["x"], wl.B, wl.T, out)
+        shards.append(sh)
+    slot_dot = torch.zeros(wl.M, dtype=torch.float32, device="cuda")
+    for sh in shards:
+        part = torch.full((wl.M,), float("nan"), dtype=torch.float32, device="cuda")
+        sh.backward_begin(d["x"], wl.B, wl.T, dy, part)
+        slot_dot += part
+    total = None
+    for sh in shards:
+        g = sh.backward_finish(d["x"], wl.B, wl.T, dy, 0.01, slot_dot)
+        assert GQ.gqe_check_device_status(sh.h) == GQ.GQE_OK
+        full = GP.full_gradients(g, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, variant=wl.variant,
+                                 shared=wl.shared, D_o=wl.D_o, g0=sh.g0, g1=sh.g1)
+        total = full if total is None else {n: (None if v is None else v + full[n])
+                                            for n, v in total.items()}
+    for sh in shards:
+        sh.close()
+    errs = {}
+    for name in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o"):
+        r = getattr(ref, name)
+        if r is None:
+            assert total[name] is None
+            continue
+        got = total[name].cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all(), name
+        errs[name] = rel_l2(got, r)
+    bad = {n: e for n, e in errs.items() if not e <= GRAD_REL_L2}
+    assert not bad, (errs, bad)
+
+
+def test_backward_phases_need_a_begin():
+    """finish without a successful begin after the last forward is refused, as is the
+    one-call backward on a group range."""
+    from moe_query_head_b200 import gqe as GQ
+    wl = MAIN.with_(B=1, T=130)
+    inp = W.generate(wl)
+    d = {n: to_device(inp, n) for n in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")}
+    dy = torch.zeros((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+    sh = GP.GroupShard(dim=wl.dim, N=wl.N, G=wl.G, k=wl.k, d_h=wl.d_h, variant=wl.variant,
+                       causal=wl.causal, max_tokens=wl.M, g0=0, g1=4, W_r=d["W_r"],
+                       W_q=d["W_q"], W_k=d["W_k"], W_v=d["W_v"], W_shared=d["W_shared"],
+                       W_o=d["W_o"])
+    sh.enable_backward()
+    out = torch.empty((wl.M, wl.dim), dtype=torch.bfloat16, device="cuda")
+    sh.forward(d["x"], wl.B, wl.T, out)
+    sd = torch.zeros(wl.M, dtype=torch.float32, device="cuda")
+    with pytest.raises(GQ.GQEError) as e:
+        sh.backward_finish(d["x"], wl.B, wl.T, dy, 0.01, sd)
+    assert e.value.status == GQ.GQE_ERR_INVALID_ARG
+    w = sh.w
+    z = lambda *s: torch.zeros(s, dtype=torch.float32, device="cuda")  # noqa: E731
+    with pytest.raises(GQ.GQEError) as e:
+        GQ.gqe_backward(sh.h, d["x"], wl.B, wl.T, d["W_r"], w["W_q"], w["W_k"], w["W_v"],
+                        w["W_shared"], w["W_o"], wl.N, wl.G, wl.k, wl.d_h, 0, 1, dy, 0.01,
+                        z(wl.M, wl.dim), z(wl.N, wl.dim), z(*w["W_q"].shape),
+                        z(*w["W_k"].shape), z(*w["W_v"].shape), z(wl.d_h, wl.dim),
+                        z(*w["W_o"].shape))
+    assert e.value.status == GQ.GQE_ERR_UNSUPPORTED
+    # begin then finish works; a second finish is refused
+    sh.backward_begin(d["x"], wl.B, wl.T, dy, sd)
+    sh.backward_finish(d["x"], wl.B, wl.T, dy, 0.01, sd)
+    with pytest.raises(GQ.GQEError) as e:
+        sh.backward_finish(d["x"], wl.B, wl.T, dy, 0.01, sd)
+    assert e.value.status == GQ.GQE_ERR_INVALID_ARG
+    sh.close()
