@@ -84,6 +84,11 @@ for _dh in (16, 32, 48, 64, 80, 96, 112, 128):
     SMALL[f"dh{_dh}_causal"] = dict(base="main_b8_t2048", B=2, T=300, d_h=_dh)
     SMALL[f"dh{_dh}_noncausal"] = dict(base="main_b8_t2048", B=1, T=200, d_h=_dh,
                                        causal=False)
+# head dims above 64 (one CTA per SM, 512 TMEM columns): more query tiles, a ragged last
+# tile, weighted_concat
+SMALL["dh128_long"] = dict(base="main_b8_t2048", B=2, T=1000, d_h=128)
+SMALL["dh96_long_weighted"] = dict(base="main_b8_t2048", B=1, T=700, d_h=96,
+                                   variant="weighted_concat")
 
 
 @pytest.mark.parametrize("case", sorted(SMALL))
