@@ -64,7 +64,11 @@ __device__ __forceinline__ float ex2(float x) {
 
 template <int DH>
 struct DecCfg {
-  static constexpr int ROWB = DH * 2 + 16;        // padded row bytes
+  // Dense rows where two lanes per key (key = lane / 2, half = lane % 2) read them without
+  // bank conflicts (d_h an odd multiple of 16: the 16-byte reads of eight lanes fall on
+  // distinct banks); else rows padded by 16 bytes with a lane per key and half.
+  static constexpr bool DENSE = DH % 32 == 16;
+  static constexpr int ROWB = DENSE ? DH * 2 : DH * 2 + 16;  // row bytes in the ring
   static constexpr int TILE = TKD * ROWB;         // one K or V tile
   static constexpr int CHUNKS = DH / 8;           // 16-byte pieces per row
   static constexpr int NP = (DH / 2 + 31) / 32;   // dim pairs per lane
@@ -80,8 +84,11 @@ __device__ __forceinline__ int stream_of(const DecParams& P, int g, int i) {
 
 // QMAX: the most queries a group can have at this launch (k, plus the shared head in group
 // 0): 2, 4 or 9, a compile-time count so the per-query state stays in registers.
+// With at most two queries per group and d_h <= 48 the state fits 64 registers, so eight
+// CTAs share an SM (the work is bound by the bytes in flight: more CTAs, more of them).
 template <int DH, int QMAX>
-__global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P) {
+__global__ void __launch_bounds__(THREADS, (DH <= 48 && QMAX <= 2) ? 8 : 1)
+decode_attn_kernel(const DecParams P) {
   using C = DecCfg<DH>;
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* sK = smem;
@@ -149,9 +156,12 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
   }
   // Every warp takes a quarter of each tile (keys 16 w .. 16 w + 15) for every query, with
   // its own online-softmax state; the four states are merged after the last tile. Score:
-  // lane = key (lane & 15) x half of the head dims (lane >> 4), halves summed by a shuffle.
+  // one key and one half of the head dims per lane (key = lane / 2, half = lane % 2 on dense
+  // rows; key = lane % 16, half = lane / 16 on padded ones), halves summed by a shuffle.
   // P V: lanes own dimension pairs and loop over the warp's 16 keys.
-  const int kq = lane & 15, half = lane >> 4;
+  const int kq = C::DENSE ? lane >> 1 : lane & 15, half = C::DENSE ? lane & 1 : lane >> 4;
+  constexpr int kHalfXor = C::DENSE ? 1 : 16;  // the lane holding the key's other half
+  constexpr int kKeyLane = C::DENSE ? 2 : 1;   // lane stride between keys
   const int krow = warp * KPW + kq;
   float m[QMAX], l[QMAX];
   float2 o[QMAX][C::NP];
@@ -195,11 +205,12 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
       float acc = 0.f;
 #pragma unroll
       for (int d = 0; d < DH / 2; ++d) acc = fmaf(q[d], kf[d], acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+      acc += __shfl_xor_sync(0xffffffffu, acc, kHalfXor);
       const float sc = key_ok ? acc : -INFINITY;
       float mt = sc;
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      for (int off = 8 * kKeyLane; off >= kKeyLane; off >>= 1)
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
       const float m_new = fmaxf(m[a], mt);
       // a warp whose keys are all masked so far keeps m = -inf, l = 0, O = 0
       const float m_ref = m_new == -INFINITY ? 0.f : m_new;
@@ -207,7 +218,8 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
       const float pk = ex2(sc - m_ref);       // 0 for a masked key
       float ps = pk;
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      for (int off = 8 * kKeyLane; off >= kKeyLane; off >>= 1)
+        ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l[a] = l[a] * alpha + ps;
       m[a] = m_new;
 #pragma unroll
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(THREADS) decode_attn_kernel(const DecParams P)
       }
 #pragma unroll
       for (int j = 0; j < KPW; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, pk, j);
+        const float pj = __shfl_sync(0xffffffffu, pk, j * kKeyLane);
         const uint8_t* row = vt + (warp * KPW + j) * C::ROWB;
 #pragma unroll
         for (int p = 0; p < C::NP; ++p) {
