@@ -79,31 +79,50 @@ def parse_args():
 
 
 ATTENTION_SOURCES = ("tc_attention.cu", "exp2_fma.cuh", "tc_ptx.cuh", "gqe_common.cuh")
+DECODE_SOURCES = ("decode.cu", "gqe_common.cuh", "tc_ptx.cuh")
 
 
-def attention_source_sha() -> str:
-    """sha256 over the attention kernel's translation unit and the headers it includes."""
+def source_sha(names) -> str:
+    """sha256 over a kernel's translation unit and the headers it includes (in csrc/)."""
     import hashlib
     h = hashlib.sha256()
-    for name in ATTENTION_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "moe_query_head_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def attention_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu capture, if that capture was
-    taken on this workload and on the current attention sources; else None."""
-    rec_path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+def attention_source_sha() -> str:
+    return source_sha(ATTENTION_SOURCES)
+
+
+def decode_source_sha() -> str:
+    return source_sha(DECODE_SOURCES)
+
+
+def kernel_traffic(record: str, workload: str, sha_fn):
+    """DRAM bytes per launch from a committed ncu capture (profiles/<record>), if that
+    capture was taken on this workload and on the kernel's current sources; else None."""
+    rec_path = os.path.join(ROOT, "profiles", record)
     try:
         with open(rec_path) as f:
             rec = json.load(f)
-        sha = attention_source_sha()
+        sha = sha_fn()
     except OSError:
         return None
     if rec.get("sources_sha256") != sha or rec.get("workload") != workload:
         return None
     return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
+
+
+def attention_traffic(workload: str):
+    """The attention kernel's DRAM bytes per launch (profiles/attn_traffic.json)."""
+    return kernel_traffic("attn_traffic.json", workload, attention_source_sha)
+
+
+def decode_traffic(workload: str):
+    """The decode cache attention's DRAM bytes per launch (profiles/decode_traffic.json)."""
+    return kernel_traffic("decode_traffic.json", workload, decode_source_sha)
 
 
 def reduce_max_over_ranks(values, dist, device):
@@ -649,7 +668,8 @@ def bench_decode(args, rank, world, dist):
                       for i in range(G.GQE_NUM_STAGES)},
         "roofline": {"kernel": "decode attention (cache read, merge)", "bound": "hbm",
                      "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                     "peak_source": f"{peak_src} HBM copy", "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy",
+                     "traffic": decode_traffic(f"decode_b{B}_l{L}"),
                      "algorithmic_bytes": kv_bytes},
         "e2e": {"value": B * world / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * 2),

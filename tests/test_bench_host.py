@@ -1,6 +1,7 @@
-"""Host logic of bench.py that needs no GPU: the DRAM traffic of the attention is reported
-only for the profiled workload and only while the attention kernel's sources hash to the
-value recorded with the ncu capture; the decode workload's shapes."""
+"""Host logic of bench.py that needs no GPU: the DRAM traffic of the attention and of the
+decode cache attention is reported only for the profiled workload and only while the
+kernel's sources hash to the value recorded with the ncu capture; the decode workload's
+shapes."""
 import json
 import os
 
@@ -20,6 +21,19 @@ def test_traffic_withheld_for_other_workloads_and_changed_sources(monkeypatch):
     assert bench.attention_traffic("main_b8_t2048") is None
     monkeypatch.setattr(bench, "attention_source_sha", lambda: "0" * 64)
     assert bench.attention_traffic("long_t16k") is None
+
+
+def test_decode_traffic_reported_only_for_the_profiled_sources(monkeypatch):
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "decode_traffic.json")))
+    assert [os.path.basename(p) for p in rec["sources"]] == list(bench.DECODE_SOURCES)
+    got = bench.decode_traffic(rec["workload"])
+    if rec["sources_sha256"] == bench.decode_source_sha():
+        assert got == rec["dram_read_bytes"] + rec["dram_write_bytes"]
+    else:
+        assert got is None
+    assert bench.decode_traffic("decode_b80_l8192") is None
+    monkeypatch.setattr(bench, "decode_source_sha", lambda: "0" * 64)
+    assert bench.decode_traffic(rec["workload"]) is None
 
 
 def test_decode_workload_is_the_papers_layer():
