@@ -133,6 +133,10 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
  *   W_*, N, G, k, d_h, variant, out [B, dim], aux_loss, stream: as gqe_forward (the aux loss
  *                                    is the Switch loss over the B new tokens).
  *
+ * A handle restricted to groups [g0, g1) (gqe_set_group_range) takes the weights as its
+ * gqe_forward does and caches of its heads only, [(g1-g0), B, L_max, d_h]; `out` receives its
+ * share of the new tokens' y (the layer's is the sum over the ranges).
+ *
  * bf16 handles only (GQE_ERR_UNSUPPORTED for fp32, or for B > 65535). Requires
  * B <= max_tokens (GQE_ERR_WORKSPACE). Allocates nothing and does not synchronise; the routing and tensors
  * of the step are available through gqe_get_routing / gqe_get_tensor (M = B). A position
@@ -277,10 +281,11 @@ gqe_status gqe_check_device_status(gqe_handle h, void* stream);
  * `out` then receives this range's share of y; the layer's y is the sum over ranges (one
  * all-reduce or reduce-scatter over the ranks). K, V, the query streams and Z of
  * gqe_get_tensor hold the range's heads only. bf16 handles whose routing runs in the dense
- * projection (N a power of two up to 32) only, else GQE_ERR_UNSUPPORTED; gqe_decode and
- * the one-call gqe_backward return GQE_ERR_UNSUPPORTED unless the range is the whole layer
- * (gqe_set_group_range(h, 0, G) restores it); a range trains with gqe_backward_begin /
- * gqe_backward_finish. GQE_ERR_INVALID_ARG unless 0 <= g0 < g1 <= G.
+ * projection (N a power of two up to 32) only, else GQE_ERR_UNSUPPORTED. gqe_decode takes
+ * the range's caches and gives its share of y; the one-call gqe_backward returns
+ * GQE_ERR_UNSUPPORTED unless the range is the whole layer (gqe_set_group_range(h, 0, G)
+ * restores it): a range trains with gqe_backward_begin / gqe_backward_finish.
+ * GQE_ERR_INVALID_ARG unless 0 <= g0 < g1 <= G.
  */
 gqe_status gqe_set_group_range(gqe_handle h, int g0, int g1);
 

@@ -293,13 +293,15 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
   if (reinterpret_cast<uintptr_t>(lengths) & 3u) return GQE_ERR_INVALID_ARG;
   if (aux_loss && (reinterpret_cast<uintptr_t>(aux_loss) & 3u)) return GQE_ERR_INVALID_ARG;
   if (h->dtype != GQE_BF16) return GQE_ERR_UNSUPPORTED;
-  if (h->g0 != 0 || h->g1 != h->G) return GQE_ERR_UNSUPPORTED;  // whole layers only
+  // the shared head reads KV head 0: only the group range that holds group 0 computes it
+  if (W_shared && h->g0 != 0) return GQE_ERR_INVALID_ARG;
   if (B > 65535) return GQE_ERR_UNSUPPORTED;  // one grid row per sequence
   if (B > h->max_tokens) return GQE_ERR_WORKSPACE;
   const int M = B;
   const int has_shared = W_shared != nullptr;
-  const int S = G * k + has_shared;
-  const int Do = (G * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
+  const int Gl = h->g1 - h->g0;  // the groups this handle computes (their caches)
+  const int S = Gl * k + has_shared;
+  const int Do = (Gl * k + (variant == GQE_VARIANT_GQE ? 1 : 0) + has_shared) * d_h;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   int launches = 0;

@@ -45,10 +45,13 @@ struct DecParams {
   __nv_bfloat16* vc;
   const int32_t* lengths;     // [B]
   __nv_bfloat16* Z;           // [B, Do]
-  const float* psel;          // [B, G*k]
+  const float* psel;          // [B, psel_stride]: stream s's p at column psel_off + s
   float* part;                // [B, G, nc, k+1, d_h + 2] partial (m, l, O) per chunk
   int32_t* status;
+  // G, S, Sr: this handle's KV heads, streams and routed streams (a group range counts
+  // from its first group; the caches hold its heads only)
   int B, G, k, S, Sr, has_shared, Do, shared_col, weighted, L_max, nc, chunk;
+  int psel_stride, psel_off;
   float scale_log2;
 };
 
@@ -288,7 +291,7 @@ decode_attn_kernel(const DecParams P) {
       int col;
       if (s < P.Sr) {
         col = s * DH;
-        if (P.weighted) scale *= P.psel[(size_t)b * P.Sr + s];
+        if (P.weighted) scale *= P.psel[(size_t)b * P.psel_stride + P.psel_off + s];
       } else {
         col = P.shared_col;
       }
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(THREADS) decode_merge_kernel(const DecParams P
     int col;
     if (s < P.Sr) {
       col = s * DH;
-      if (P.weighted) scale *= P.psel[(size_t)b * P.Sr + s];
+      if (P.weighted) scale *= P.psel[(size_t)b * P.psel_stride + P.psel_off + s];
     } else {
       col = P.shared_col;
     }
@@ -371,7 +374,7 @@ int launch_dh(const DecParams& P, cudaStream_t st) {
 // with seven), at least one tile each, and partial slots within the workspace's
 // kDecodeSlots.
 int decode_chunks(const gqe_ctx* h, int B, int L_max) {
-  const int64_t bg = (int64_t)B * h->G;
+  const int64_t bg = (int64_t)B * (h->g1 - h->g0);  // (sequence, KV head) pairs
   int64_t nc = (16 * (int64_t)h->num_sms + bg - 1) / bg;
   const int64_t max_by_len = ((int64_t)L_max + TKD - 1) / TKD;
   if (nc > max_by_len) nc = max_by_len;
@@ -396,10 +399,12 @@ int launch_tc_decode_attention(gqe_ctx* h, int B, int S, int has_shared, int var
   P.part = h->ws.dec_part;
   P.status = h->ws.status;
   P.B = B;
-  P.G = h->G;
+  P.G = h->g1 - h->g0;
   P.k = h->k;
   P.S = S;
-  P.Sr = h->G * h->k;
+  P.Sr = P.G * h->k;
+  P.psel_stride = h->G * h->k;
+  P.psel_off = h->g0 * h->k;
   P.has_shared = has_shared;
   P.Do = Do;
   P.shared_col = (P.Sr + (variant == GQE_VARIANT_GQE ? 1 : 0)) * d_h;

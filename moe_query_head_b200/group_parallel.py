@@ -82,6 +82,15 @@ def rank_weights(W_q, W_k, W_v, W_shared, W_o, *, N: int, G: int, k: int, d_h: i
     }
 
 
+def rank_caches(k_cache, v_cache, g0: int, g1: int):
+    """The KV caches [G, B, L_max, d_h] of groups g0 .. g1-1: a rank's own caches for the
+    decode step (contiguous copies; the rank keeps them and its steps append to them)."""
+    def part(c):
+        r = c[g0:g1]
+        return r.contiguous() if hasattr(r, "contiguous") else np.ascontiguousarray(r)
+    return part(k_cache), part(v_cache)
+
+
 def full_gradients(shares: dict, *, N: int, G: int, k: int, d_h: int, variant: str,
                    shared: bool, D_o: int, g0: int, g1: int) -> dict:
     """A rank's gradient shares (the shapes of its weight slices, as rank_weights gives them)
@@ -147,6 +156,22 @@ class GroupShard:
 
     def forward_allreduce(self, x, B, T, out, dist, group=None):
         self.forward(x, B, T, out)
+        dist.all_reduce(out, group=group)
+        return out
+
+    def decode(self, x, B, k_cache, v_cache, L_max, lengths, out, stream=None):
+        """One decode step on this rank's groups: k_cache / v_cache hold its heads only,
+        [(g1-g0), B, L_max, d_h] (rank_caches of the layer's caches); `out` receives the
+        rank's share of the new tokens' y, and the new K / V are written into its caches."""
+        from .workloads import VARIANT_IDS
+        w = self.w
+        self.GQ.gqe_decode(self.h, x, B, k_cache, v_cache, L_max, lengths, self.W_r, w["W_q"],
+                           w["W_k"], w["W_v"], w["W_shared"], w["W_o"], self.N, self.G, self.k,
+                           self.d_h, VARIANT_IDS[self.variant], out, self.aux, stream)
+        return out
+
+    def decode_allreduce(self, x, B, k_cache, v_cache, L_max, lengths, out, dist, group=None):
+        self.decode(x, B, k_cache, v_cache, L_max, lengths, out)
         dist.all_reduce(out, group=group)
         return out
 

@@ -13,7 +13,7 @@ import torch
 
 from moe_query_head_b200 import group_parallel as GP
 from moe_query_head_b200 import workloads as W
-from tests.gqe_testlib import AUX_REL, check_output, oracle_forward, to_device
+from tests.gqe_testlib import AUX_REL, check_output, oracle_forward, to_device, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -209,3 +209,54 @@ def test_backward_phases_need_a_begin():
         sh.backward_finish(d["x"], wl.B, wl.T, dy, 0.01, sd)
     assert e.value.status == GQ.GQE_ERR_INVALID_ARG
     sh.close()
+
+
+DEC_CASES = {
+    "main_2_ranks": (MAIN, [0, 5, 63, 64, 200, 511], 512, 2),
+    "main_3_ranks_uneven": (MAIN, [3, 130, 300], 320, 3),
+    "wide_weighted_4_ranks": (WIDE.with_(variant="weighted_concat"), [10, 257, 70], 260, 4),
+    "main_hard_no_shared_8_ranks": (MAIN.with_(shared=False, variant="hard_concat"),
+                                    [1, 100], 128, 8),
+}
+
+
+@pytest.mark.parametrize("case", list(DEC_CASES))
+def test_group_shards_decode_sums_to_the_layer(case):
+    """A decode step on the split: every rank holds its heads' caches and computes its share;
+    the shares sum to the float64 oracle's step (y at the bf16 tolerances, routing bit-exact
+    on every rank), and each rank writes its heads' new K / V at the new positions and no
+    other cache row."""
+    from moe_query_head_b200 import gqe as GQ
+    from tests.test_decode_gpu import _dev_bf16, oracle_decode
+    wl, lengths, L_max, world = DEC_CASES[case]
+    d = W.generate_decode(wl, lengths, L_max)
+    ref = oracle_decode(d)
+    inp = d.inp
+    dev = {n: to_device(inp, n) for n in ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")}
+    kc, vc = _dev_bf16(d.k_cache), _dev_bf16(d.v_cache)
+    lens = torch.from_numpy(d.lengths.astype(np.int32)).cuda()
+    B = len(lengths)
+    total = torch.zeros((B, inp.wl.dim), dtype=torch.float32, device="cuda")
+    for g0, g1 in GP.group_ranges(inp.wl.G, world):
+        sh = GP.GroupShard(dim=inp.wl.dim, N=inp.wl.N, G=inp.wl.G, k=inp.wl.k, d_h=inp.wl.d_h,
+                           variant=inp.wl.variant, causal=True, max_tokens=B, g0=g0, g1=g1,
+                           W_r=dev["W_r"], W_q=dev["W_q"], W_k=dev["W_k"], W_v=dev["W_v"],
+                           W_shared=dev["W_shared"] if inp.wl.shared else None, W_o=dev["W_o"])
+        kr, vr = GP.rank_caches(kc, vc, g0, g1)
+        k0, v0 = kr.clone(), vr.clone()
+        out = torch.full((B, inp.wl.dim), float("nan"), dtype=torch.bfloat16, device="cuda")
+        sh.decode(dev["x"], B, kr, vr, L_max, lens, out)
+        assert GQ.gqe_check_device_status(sh.h) == GQ.GQE_OK
+        total += out.float()
+        sel = torch.empty((B, inp.wl.G, inp.wl.k), dtype=torch.int32, device="cuda")
+        GQ.gqe_get_routing(sh.h, sel=sel)
+        torch.cuda.synchronize()
+        assert np.array_equal(sel.cpu().numpy(), ref.routing.sel.astype(np.int32))
+        keep = torch.ones(kr.shape[:3], dtype=torch.bool, device="cuda")
+        for b, L in enumerate(d.lengths.tolist()):
+            keep[:, b, L] = False
+        assert torch.equal(kr[keep], k0[keep]) and torch.equal(vr[keep], v0[keep])
+        rows = torch.stack([kr[:, b, L] for b, L in enumerate(d.lengths.tolist())], dim=1)
+        np.testing.assert_allclose(to_host_f64(rows), ref.K_new[g0:g1], rtol=1e-2, atol=1e-2)
+        sh.close()
+    check_output(total.cpu().numpy().astype(np.float64), ref.y, "bf16")
