@@ -243,56 +243,3 @@ def gqe_set_stage_events(h, events) -> None:
         return
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(lib.gqe_set_stage_events(h, arr, len(events)), "gqe_set_stage_events")
-
-
-class GQEAttention:
-    """One GQE attention layer shape on the current CUDA device.
-
-    The constructor arguments follow the module of the "GQE: Grouped Query Experts" README
-    (Usage, Parameters): dim, num_query_experts, num_kv_heads, top_k, head_dim (default
-    dim // num_query_experts), variant. Weights are passed to `forward` by the caller.
-    """
-
-    def __init__(self, dim, num_query_experts=16, num_kv_heads=8, top_k=1, head_dim=None,
-                 variant="gqe", dtype=torch.bfloat16, max_tokens=65536, shared=True,
-                 causal=True):
-        if num_query_experts % num_kv_heads != 0:
-            raise ValueError("num_query_experts must be divisible by num_kv_heads")
-        self.dim, self.N, self.G, self.k = dim, num_query_experts, num_kv_heads, top_k
-        self.d_h = head_dim if head_dim is not None else dim // num_query_experts
-        self.variant = variant
-        self.dtype = dtype
-        self.shared = shared
-        self.causal = causal
-        self.max_tokens = max_tokens
-        code = GQE_F32 if dtype == torch.float32 else GQE_BF16
-        self.handle = gqe_create(dim, self.N, self.G, self.k, self.d_h, code, max_tokens)
-        self.aux = torch.zeros(1, dtype=torch.float32, device="cuda")
-
-    @property
-    def D_o(self) -> int:
-        return (self.G * self.k + (self.variant == "gqe") + self.shared) * self.d_h
-
-    def forward(self, x, W_r, W_q, W_k, W_v, W_shared, W_o, B, T, out=None, stream=None):
-        if out is None:
-            out = torch.empty((B * T, self.dim), dtype=self.dtype, device=x.device)
-        gqe_forward(self.handle, x, B, T, W_r, W_q, W_k, W_v, W_shared if self.shared else None,
-                    W_o, self.N, self.G, self.k, self.d_h, VARIANTS[self.variant],
-                    int(self.causal), out, self.aux, stream)
-        return out
-
-    def collect_aux_loss(self):
-        """The load-balancing loss of the last forward, as a device scalar (the README's
-        collect_aux_loss; the caller applies its 0.01 coefficient)."""
-        return self.aux[0]
-
-    def close(self):
-        if self.handle:
-            gqe_destroy(self.handle)
-            self.handle = None
-
-    def __del__(self):
-        try:
-            self.close()
-        except Exception:
-            pass

@@ -134,3 +134,18 @@ def test_full_gradients_place_the_shares(variant, shared, world):
         times[G * k * d_h:(G * k + 1) * d_h] = world
     assert np.allclose(total["W_o"], A["W_o"] * times[None, :])
     assert np.array_equal(total["x"], world * x)
+
+
+def test_module_constructor_follows_the_readme():
+    """GQEAttention's constructor (no GPU needed until the first call): head_dim defaults to
+    dim // num_query_experts, the experts must split evenly over the KV heads, the weights
+    have nn.Linear's [out, in] shapes."""
+    from moe_query_head_b200.module import GQEAttention
+    m = GQEAttention(768)
+    assert (m.N, m.G, m.k, m.d_h, m.variant) == (16, 8, 1, 48, "gqe")
+    assert tuple(m.W_q.shape) == (16 * 48, 768) and tuple(m.W_o.shape) == (768, 10 * 48)
+    assert GQEAttention(768, variant="hard_concat", shared=False).W_o.shape[1] == 8 * 48
+    with pytest.raises(ValueError):
+        GQEAttention(768, num_query_experts=12, num_kv_heads=8)
+    with pytest.raises(ValueError):
+        GQEAttention(768, variant="sum")
