@@ -130,6 +130,32 @@ class GQEAttention(nn.Module):
         self._aux = aux
         return y
 
+    def allocate_cache(self, B: int, L_max: int, device=None):
+        """Empty KV caches for generation: k_cache, v_cache [G, B, L_max, d_h] in bf16."""
+        shape = (self.G, B, L_max, self.d_h)
+        dev = device if device is not None else self.W_r.device
+        return (torch.zeros(shape, dtype=torch.bfloat16, device=dev),
+                torch.zeros(shape, dtype=torch.bfloat16, device=dev))
+
+    @torch.no_grad()
+    def decode_step(self, x_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    lengths: torch.Tensor) -> torch.Tensor:
+        """One generation step (gqe_decode): x_new [B, dim], one new token per sequence at
+        position lengths[b] (int32, on the device); its K / V are written into the caches at
+        that row and y_new [B, dim] (bf16) is returned. The caller advances `lengths`."""
+        B = x_new.shape[0]
+        bf = torch.bfloat16
+        h = self._handle_for(B)
+        w = [W.to(bf).contiguous() for W in (self.W_r, self.W_q, self.W_k, self.W_v)]
+        ws = self.W_shared.to(bf).contiguous() if self.W_shared is not None else None
+        out = torch.empty((B, self.dim), dtype=bf, device=x_new.device)
+        aux = torch.zeros(1, dtype=torch.float32, device=x_new.device)
+        G.gqe_decode(h, x_new.to(bf).contiguous(), B, k_cache, v_cache, k_cache.shape[2],
+                     lengths, w[0], w[1], w[2], w[3], ws, self.W_o.to(bf).contiguous(), self.N,
+                     self.G, self.k, self.d_h, G.VARIANTS[self.variant], out, aux)
+        self._calls += 1  # the handle's saved state is no longer a forward's
+        return out
+
     def aux_loss(self) -> torch.Tensor | None:
         """The Switch load-balancing loss of the last call (a differentiable scalar)."""
         return self._aux

@@ -108,3 +108,22 @@ def test_collect_aux_loss_sums_the_layers():
     assert torch.allclose(a, m1.aux_loss() + m2.aux_loss())
     ref_aux = oracle_forward(inp).aux
     assert abs(float(m1.aux_loss().detach()) - ref_aux) <= 1e-4 * ref_aux
+
+
+def test_module_decode_step_matches_the_oracle():
+    """GQEAttention.decode_step over caches filled for a few sequences: y_new at the bf16
+    tolerances against the oracle's decode step, the new K / V written at the positions."""
+    from tests.test_decode_gpu import _dev_bf16, oracle_decode
+    wl = MAIN
+    d = W.generate_decode(wl, [0, 37, 200], 256)
+    inp = d.inp
+    m = _module(inp.wl, inp)
+    kc, vc = _dev_bf16(d.k_cache), _dev_bf16(d.v_cache)
+    lens = torch.from_numpy(d.lengths.astype(np.int32)).cuda()
+    x_new = torch.from_numpy(inp.f64("x")).float().cuda()
+    y = m.decode_step(x_new, kc, vc, lens)
+    ref = oracle_decode(d)
+    check_output(y.double().cpu().numpy(), ref.y, "bf16")
+    for b, L in enumerate(d.lengths.tolist()):
+        np.testing.assert_allclose(kc[:, b, L].double().cpu().numpy(), ref.K_new[:, b],
+                                   rtol=1e-2, atol=1e-2)
