@@ -68,6 +68,12 @@ def test_null_handle_paths():
     assert G.lib.gqe_backward(None, z, 1, 1, z, z, z, z, z, z, 16, 8, 1, 48, 0, 1, z, 0.0, z, z,
                               z, z, z, z, z, None) == G.GQE_ERR_INVALID_ARG
     assert G.lib.gqe_backward_launches(None) == -1
+    assert G.lib.gqe_backward_begin(None, z, 1, 1, z, z, z, z, z, z, 16, 8, 1, 48, 0, 1, z, z,
+                                    None) == G.GQE_ERR_INVALID_ARG
+    assert G.lib.gqe_backward_finish(None, z, 1, 1, z, z, z, z, z, z, 16, 8, 1, 48, 0, 1, z,
+                                     0.0, z, z, z, z, z, z, z, z, None) == G.GQE_ERR_INVALID_ARG
+    assert G.lib.gqe_decode(None, z, 1, z, z, 8, z, z, z, z, z, z, z, 16, 8, 1, 48, 0, z, z,
+                            None) == G.GQE_ERR_INVALID_ARG
     G.lib.gqe_destroy(None)
 
 
