@@ -109,6 +109,13 @@ gqe_status gqe_create(gqe_handle* h, int dim, int N, int G, int k, int d_h, gqe_
  * index. Allocates nothing and does not synchronise. Returns GQE_ERR_WORKSPACE if
  * B*T > max_tokens, GQE_ERR_INVALID_ARG for null required pointers, pointers not 16-byte
  * aligned, B < 1, T < 1, or N/G/k/d_h different from the handle's.
+ *
+ * CUDA graphs: a call (gqe_forward or gqe_decode) may be captured on `stream` and the graph
+ * replayed any number of times, interleaved with eager calls on the same handle in stream
+ * order; every per-call state the kernels keep (the routing cursors' two alternating sets
+ * and their set flag, the attention's work counter) lives in the handle's device workspace
+ * and is advanced by the kernels themselves. The replay reads the pointers and sizes of the
+ * captured call. Two captured graphs of one handle must not run concurrently.
  */
 gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_r,
                        const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
@@ -258,7 +265,9 @@ gqe_status gqe_get_tensor(gqe_handle h, int which, void* dst, size_t bytes, void
  * gqe_check_device_status — synchronise `stream`, then read and clear the handle's device
  * status word. Returns GQE_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
  * check (its output is then invalid), GQE_ERR_INVALID_ARG if a gqe_decode met a position
- * outside its cache, GQE_ERR_CUDA if the stream reports an error, else GQE_OK.
+ * outside its cache, GQE_ERR_CUDA if the stream reports an error or the routed projection
+ * found its routing cursors out of range (a state no sequence of calls should reach: the
+ * bucket reads were clamped and the output is invalid), else GQE_OK.
  */
 gqe_status gqe_check_device_status(gqe_handle h, void* stream);
 

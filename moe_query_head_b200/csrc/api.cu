@@ -68,7 +68,7 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
   w.tile_count = (int32_t*)take(16);
   w.attn_counter = (int32_t*)take(16);
   w.cursor = (int32_t*)take((kMaxExperts + 4) * 4);
-  w.rcur = (int32_t*)take(2 * kMaxExperts * 4);
+  w.rcur = (int32_t*)take((kRouteFlag + 2) * 4);
   w.rpsum = (unsigned long long*)take(2 * kMaxExperts * 8);
   w.dec_part = (float*)take((size_t)kDecodeSlots * (k + 1) * (d_h + 2) * 4);
   w.status = (int32_t*)take(16);
@@ -77,6 +77,14 @@ size_t layout(Workspace& w, char* base, int dim, int N, int G, int k, int d_h, i
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A call that launched the dense projection's routing but not the routed projection leaves
+// a cursor set written and the set flag unflipped: both sets and the flag go back to zero so
+// the next call starts clean.
+void reset_route_sets(gqe_ctx* h, cudaStream_t st) {
+  cudaMemsetAsync(h->ws.rcur, 0, (kRouteFlag + 2) * sizeof(int32_t), st);
+  cudaMemsetAsync(h->ws.rpsum, 0, 2 * kMaxExperts * sizeof(unsigned long long), st);
+}
 
 }  // namespace
 
@@ -241,24 +249,23 @@ gqe_status gqe_forward(gqe_handle h, const void* x, int B, int T, const void* W_
   // bf16: tensor-core (tcgen05) kernels for the projections; fp32: CUDA-core kernels.
   const bool tc = h->dtype == GQE_BF16;
   // bf16 with N a power of two up to 32: the routing runs in the dense projection's router
-  // tiles, and the routed projection schedules from its cursors (set `rs`, alternating)
+  // tiles, and the routed projection schedules from its cursors (the two cursor sets
+  // alternate between calls on a flag the kernels keep in device memory, so the call can be
+  // captured in a CUDA graph and replayed)
   const bool fused = tc && tc_dense_routes(h);
-  const int rs = h->route_set;
   int dense = -1;
   bool ok = mark() &&
-            add(dense = tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, rs, st)
+            add(dense = tc ? launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)
                            : launch_simt_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
             add(fused ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
-            add(tc ? launch_tc_qproj(h, x, M, W_q, fused ? rs : -1, aux_loss, st)
+            add(tc ? launch_tc_qproj(h, x, M, W_q, fused, aux_loss, st)
                    : launch_simt_qproj(h, x, M, W_q, st)) &&
             add(tc ? launch_tc_attention(h, B, T, S, has_shared, variant, causal, Do, st)
                    : launch_simt_attention(h, B, T, S, has_shared, variant, causal, Do, st)) &&
             add(launch_combine(h, M, variant, Do, st)) &&
             add(tc ? launch_tc_oproj(h, M, Do, W_o, out, st)
                    : launch_simt_oproj(h, M, Do, W_o, out, st));
-  // once the dense projection has run, this call's cursor set is in use and the other one
-  // cleared: the next call takes the other one
-  if (fused && dense >= 0) h->route_set ^= 1;
+  if (fused && dense >= 0 && !ok) reset_route_sets(h, st);
   h->last_M = M;
   h->last_S = S;
   h->last_Do = Do;
@@ -321,17 +328,16 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
   // the forward's stages on the B new tokens, with the cache attention in place of the
   // prefill attention
   const bool fused = tc_dense_routes(h);
-  const int rs = h->route_set;
   int dense = -1;
   bool ok = mark() &&
-            add(dense = launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, rs, st)) &&
+            add(dense = launch_tc_dense_proj(h, x, M, W_r, W_k, W_v, W_shared, st)) &&
             add(fused ? 0 : launch_route_fused(h, M, aux_loss, st)) &&
-            add(launch_tc_qproj(h, x, M, W_q, fused ? rs : -1, aux_loss, st)) &&
+            add(launch_tc_qproj(h, x, M, W_q, fused, aux_loss, st)) &&
             add(launch_tc_decode_attention(h, B, S, has_shared, variant, Do, k_cache, v_cache,
                                            L_max, lengths, st)) &&
             add(launch_combine(h, M, variant, Do, st)) &&
             add(launch_tc_oproj(h, M, Do, W_o, out, st));
-  if (fused && dense >= 0) h->route_set ^= 1;
+  if (fused && dense >= 0 && !ok) reset_route_sets(h, st);
   h->last_M = M;
   h->last_S = S;
   h->last_Do = Do;
@@ -390,7 +396,9 @@ gqe_status gqe_check_device_status(gqe_handle h, void* stream) {
   if (cudaMemcpy(&v, h->ws.status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return GQE_ERR_CUDA;
   if (v != kStatusOk) {
     cudaMemset(h->ws.status, 0, 4);
-    return v == kStatusBadInput ? GQE_ERR_INVALID_ARG : GQE_ERR_TIMEOUT;
+    return v == kStatusBadInput ? GQE_ERR_INVALID_ARG
+           : v == kStatusBadState ? GQE_ERR_CUDA
+                                  : GQE_ERR_TIMEOUT;
   }
   return GQE_OK;
 }

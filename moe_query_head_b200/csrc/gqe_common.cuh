@@ -16,11 +16,15 @@ constexpr int kRouteBlock = 128;
 // Maximum sizes this build supports.
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
+// The dense projection's routing keeps its bucket cursors in two sets that alternate between
+// calls; the set of the next call is a flag in device memory after them (see tc_gemm.cu).
+constexpr int kRouteFlag = 2 * kMaxExperts;
 
 // Device status word values (written by kernels whose bounded waits give up).
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusBadInput = 2;  // a decode position outside its cache
+constexpr int kStatusBadState = 3;  // routing cursors out of range (never expected)
 
 // Partial-result slots of the decode attention: (sequence, group, key chunk) triples whose
 // (m, l, O) are merged by a second kernel. Bounded independently of the cache length (the
@@ -123,7 +127,8 @@ struct Workspace {
   int32_t* attn_counter = nullptr; // attention work-item counter
   // dense-projection routing: two sets (alternate calls) of bucket cursors and
   // fixed-point probability sums; a call's set is zero when it starts
-  int32_t* rcur = nullptr;                // [2, kMaxExperts]
+  int32_t* rcur = nullptr;                // [2, kMaxExperts] cursors, then the set flag and an
+                                          // exit counter (kRouteFlag, kRouteFlag + 1)
   unsigned long long* rpsum = nullptr;    // [2, kMaxExperts]
   int32_t* cursor = nullptr;       // [kMaxExperts] bucket cursors, then the routing ticket
                                    // (zero between calls)
@@ -171,7 +176,6 @@ struct gqe_ctx {
   // gqe_backward must repeat
   int last_kind = 0, last_B = 0, last_T = 0, last_variant = -1, last_causal = -1,
       last_shared = -1, last_g0 = -1, last_g1 = -1;
-  int route_set = 0;  // the dense-projection routing's cursor set for the next call
   // backward pass (gqe_enable_backward)
   void* bwd_base = nullptr;
   size_t bwd_bytes = 0;
@@ -214,10 +218,9 @@ int launch_combine(gqe_ctx* h, int M, int variant, int Do, cudaStream_t st);
 int launch_simt_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 // tcgen05 paths (bf16)
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, int route_set,
-                         cudaStream_t st);
+                         const void* W_v, const void* W_shared, cudaStream_t st);
 bool tc_dense_routes(const gqe_ctx* h);  // launch_tc_dense_proj also routes
-int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route_set,
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, bool from_cursors,
                     float* aux_out, cudaStream_t st);
 int launch_tc_oproj(gqe_ctx* h, int M, int Do, const void* W_o, void* out, cudaStream_t st);
 int launch_tc_attention(gqe_ctx* h, int B, int T, int S, int has_shared, int variant,

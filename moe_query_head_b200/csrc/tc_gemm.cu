@@ -71,19 +71,20 @@ struct Problem {
 };
 
 // Outputs of the routing done in the dense projection's router tiles (see route_rows). The
-// cursors and probability sums come in two sets used by alternate calls: this call's set
-// is zero when it starts (the previous call's dense projection cleared it), and this call
-// clears the other one, whose last reader (the previous call's routed projection) is done.
+// cursors and probability sums come in two sets used by alternate calls, chosen on the
+// device by a flag that the routed projection's last CTA flips when it is done with its set
+// (so a captured graph alternates as its calls would): this call's set is zero when it
+// starts (the previous call's dense projection cleared it), and this call clears the other
+// one, whose last reader (the previous call's routed projection) is done.
 struct RouteOut {
   float* logits_out;     // [M, N] problem 0's output (router logits, fp32)
   int32_t* sel;          // [M, G, k]
   float* psel;           // [M, G, k]
   float* gates;          // [M, G, k]
   float* wslot;          // [M, G, k]
-  unsigned long long* psum_fx;  // [kMaxExperts] probability sums, fixed point
-  int32_t* cursor;       // [kMaxExperts] bucket cursors
-  unsigned long long* clear_psum;  // the other set, zeroed here
-  int32_t* clear_cursor;
+  unsigned long long* psum_fx;  // [2][kMaxExperts] probability sums, fixed point
+  int32_t* cursor;       // [2][kMaxExperts] bucket cursors
+  const int32_t* set_flag;  // the set of this call (0 or 1)
   int32_t* bucket;       // [N * M]
 };
 
@@ -119,9 +120,12 @@ struct Params {
   const int2* tile_list;                // (expert | rows << 8, first bucket slot) per tile
   const int32_t* tile_count;            // number of tiles (device)
   // scheduling from the dense projection's cursors instead of the tile list (rc non-null):
-  // expert e's bucket holds rc[e] entries; CTA 0 also writes the statistics
-  const int32_t* rc;
-  const unsigned long long* rpsum;      // probability sums, fixed point
+  // expert e's bucket holds rc[set][e] entries for the call's set (*set_flag); CTA 0 also
+  // writes the statistics; the last CTA to finish flips *set_flag
+  const int32_t* rc;                    // [2][kMaxExperts]
+  const unsigned long long* rpsum;      // [2][kMaxExperts] probability sums, fixed point
+  int32_t* set_flag;
+  int32_t* exit_counter;                // zero between calls
   int nexp;
   // experts whose buckets this projection computes: [e_lo, e_hi) (a group range of the
   // layer, see gqe_set_group_range); W_q holds their rows only and their query streams
@@ -215,7 +219,7 @@ constexpr double kProbFix = 4294967296.0;  // 2^32
 // The only memory round trip on this path is that atomic.
 template <int N, int E>
 __device__ void route_rows(const Params& P, uint32_t t_row, int t, bool valid, int lane,
-                           uint64_t* acc_empty) {
+                           uint64_t* acc_empty, int cset) {
   constexpr int G = N / E;
   constexpr unsigned all = 0xffffffffu;
   const RouteOut& R = P.ro;
@@ -321,8 +325,9 @@ __device__ void route_rows(const Params& P, uint32_t t_row, int t, bool valid, i
   }
   int my_base = 0;
   if (lane < N) {
-    if (my_cnt) my_base = atomicAdd(&R.cursor[lane], my_cnt);
-    atomicAdd(&R.psum_fx[lane], (unsigned long long)__double2ll_rn((double)my_sum * kProbFix));
+    if (my_cnt) my_base = atomicAdd(&R.cursor[cset + lane], my_cnt);
+    atomicAdd(&R.psum_fx[cset + lane],
+              (unsigned long long)__double2ll_rn((double)my_sum * kProbFix));
   }
   const unsigned below = (1u << lane) - 1u;
 #pragma unroll
@@ -339,26 +344,26 @@ __device__ void route_rows(const Params& P, uint32_t t_row, int t, bool valid, i
 
 template <int N>
 __device__ void route_rows_e(const Params& P, uint32_t t_row, int t, bool valid, int lane,
-                             uint64_t* bar) {
+                             uint64_t* bar, int cset) {
   switch (N / P.G) {
-    case 1: route_rows<N, 1>(P, t_row, t, valid, lane, bar); break;
-    case 2: if constexpr (N >= 2) route_rows<N, (N >= 2 ? 2 : 1)>(P, t_row, t, valid, lane, bar); break;
-    case 4: if constexpr (N >= 4) route_rows<N, (N >= 4 ? 4 : 1)>(P, t_row, t, valid, lane, bar); break;
-    case 8: if constexpr (N >= 8) route_rows<N, (N >= 8 ? 8 : 1)>(P, t_row, t, valid, lane, bar); break;
-    case 16: if constexpr (N >= 16) route_rows<N, (N >= 16 ? 16 : 1)>(P, t_row, t, valid, lane, bar); break;
-    default: if constexpr (N >= 32) route_rows<N, (N >= 32 ? 32 : 1)>(P, t_row, t, valid, lane, bar); break;
+    case 1: route_rows<N, 1>(P, t_row, t, valid, lane, bar, cset); break;
+    case 2: if constexpr (N >= 2) route_rows<N, (N >= 2 ? 2 : 1)>(P, t_row, t, valid, lane, bar, cset); break;
+    case 4: if constexpr (N >= 4) route_rows<N, (N >= 4 ? 4 : 1)>(P, t_row, t, valid, lane, bar, cset); break;
+    case 8: if constexpr (N >= 8) route_rows<N, (N >= 8 ? 8 : 1)>(P, t_row, t, valid, lane, bar, cset); break;
+    case 16: if constexpr (N >= 16) route_rows<N, (N >= 16 ? 16 : 1)>(P, t_row, t, valid, lane, bar, cset); break;
+    default: if constexpr (N >= 32) route_rows<N, (N >= 32 ? 32 : 1)>(P, t_row, t, valid, lane, bar, cset); break;
   }
 }
 
 __device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool valid, int lane,
-                               uint64_t* bar) {
+                               uint64_t* bar, int cset) {
   switch (P.prob[0].N) {
-    case 1: route_rows_e<1>(P, t_row, t, valid, lane, bar); break;
-    case 2: route_rows_e<2>(P, t_row, t, valid, lane, bar); break;
-    case 4: route_rows_e<4>(P, t_row, t, valid, lane, bar); break;
-    case 8: route_rows_e<8>(P, t_row, t, valid, lane, bar); break;
-    case 16: route_rows_e<16>(P, t_row, t, valid, lane, bar); break;
-    default: route_rows_e<32>(P, t_row, t, valid, lane, bar); break;
+    case 1: route_rows_e<1>(P, t_row, t, valid, lane, bar, cset); break;
+    case 2: route_rows_e<2>(P, t_row, t, valid, lane, bar, cset); break;
+    case 4: route_rows_e<4>(P, t_row, t, valid, lane, bar, cset); break;
+    case 8: route_rows_e<8>(P, t_row, t, valid, lane, bar, cset); break;
+    case 16: route_rows_e<16>(P, t_row, t, valid, lane, bar, cset); break;
+    default: route_rows_e<32>(P, t_row, t, valid, lane, bar, cset); break;
   }
 }
 
@@ -368,10 +373,16 @@ __device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool vali
 // writes the routing statistics ("GQE" README, Algorithm Overview; the Switch-style
 // load-balancing loss): counts, mean_prob (fixed-point sum / M), offsets (e M) and
 //   L = (1/G) sum_e E f_e Pbar_e,  f = count / (M k),  Pbar = prob_sum / M.
-__device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0) {
+__device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0, int cset) {
   const int N = P.nexp, M = P.M;
   const int tid = threadIdx.x;
-  if (tid < N) s_cnt[tid] = __ldcg(P.rc + tid);
+  if (tid < N) {
+    // a count above M would mean a cursor set that was not cleared: never reached, but the
+    // bucket reads stay inside expert e's M slots whatever the cursors hold
+    const int c = __ldcg(P.rc + cset + tid);
+    s_cnt[tid] = min(max(c, 0), M);
+    if (c < 0 || c > M) atomicExch(P.status, kStatusBadState);
+  }
   __syncthreads();
   if (tid == 0) {
     int nt = 0;
@@ -385,7 +396,8 @@ __device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0) {
     const StatsOut& S = P.so;
     const int G = N / P.E;
     if (tid < N) {
-      const double ps = (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + tid) / kProbFix;
+      const double ps =
+          (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + cset + tid) / kProbFix;
       S.counts[tid] = s_cnt[tid];
       S.offsets[tid] = tid * M;
       S.mean_prob[tid] = (float)(ps / M);
@@ -395,7 +407,7 @@ __device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0) {
       double L = 0.0;
       for (int x = 0; x < N; ++x) {
         const double ps =
-            (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + x) / kProbFix;
+            (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + cset + x) / kProbFix;
         L += (double)P.E * ((double)s_cnt[x] / ((double)M * P.k)) * (ps / M);
       }
       if (S.aux) S.aux[0] = (float)(L / G);
@@ -464,16 +476,20 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   int* s_cnt = reinterpret_cast<int*>(scratch);         // [kMaxExperts] routed schedule
   int* s_t0 = s_cnt + kMaxExperts;                      // [kMaxExperts + 1]
   int total = P.total_tiles;
+  int cset = 0;  // this call's cursor set, as an offset into the two sets
   if constexpr (ROUTE) {
     // this call's cursor set is zero; the other one (the previous call's) is cleared here
+    cset = (__ldcg(P.ro.set_flag) & 1) * kMaxExperts;
     if (blockIdx.x == 0 && threadIdx.x < kMaxExperts) {
-      P.ro.clear_cursor[threadIdx.x] = 0;
-      P.ro.clear_psum[threadIdx.x] = 0ull;
+      const int other = kMaxExperts - cset;
+      P.ro.cursor[other + threadIdx.x] = 0;
+      P.ro.psum_fx[other + threadIdx.x] = 0ull;
     }
   }
   if constexpr (GATHER) {
     if (P.rc != nullptr) {
-      routed_schedule(P, s_cnt, s_t0);  // block-wide
+      cset = (__ldcg(P.set_flag) & 1) * kMaxExperts;
+      routed_schedule(P, s_cnt, s_t0, cset);  // block-wide
       total = s_t0[P.nexp];
     } else {
       total = *P.tile_count;
@@ -700,7 +716,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
       } else if (ROUTE && ti.p == 0) {
         // router tile: the logits stay in registers for the routing, which also releases
         // the accumulator and stores the logits
-        route_rows_any(P, t_row, ti.m0 + row, valid, lane, &acc_empty[acc]);
+        route_rows_any(P, t_row, ti.m0 + row, valid, lane, &acc_empty[acc], cset);
       } else {
         const Problem& pr = P.prob[ti.p];
         const OutMap& o = pr.out;
@@ -754,6 +770,13 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   if (warp == L::MMA) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  // routed projection scheduled from the cursors: once every CTA has read this call's set,
+  // the next call takes the other one
+  if (GATHER && P.rc != nullptr && threadIdx.x == 0 &&
+      atomicAdd(P.exit_counter, 1) == (int)gridDim.x - 1) {
+    *P.set_flag ^= 1;
+    *P.exit_counter = 0;
   }
 }
 
@@ -870,8 +893,7 @@ bool tc_dense_routes(const gqe_ctx* h) { return h->N <= 32 && (h->N & (h->N - 1)
 // fills the buckets, and the last CTA forms the statistics, the aux loss (if aux_out) and
 // the routed-projection tiles.
 int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, const void* W_k,
-                         const void* W_v, const void* W_shared, int route_set,
-                         cudaStream_t st) {
+                         const void* W_v, const void* W_shared, cudaStream_t st) {
   const int d_h = h->d_h, G = h->g1 - h->g0, dim = h->dim;  // this handle's KV heads
   const int S = G * h->k + (W_shared ? 1 : 0);
   Params P;
@@ -905,18 +927,16 @@ int launch_tc_dense_proj(gqe_ctx* h, const void* x, int M, const void* W_r, cons
   P.G = h->G;  // routing covers every group
   P.k = h->k;
   const Workspace& w = h->ws;
-  const int cur = route_set & 1, other = cur ^ 1;
-  P.ro = RouteOut{w.logits, w.sel, w.psel, w.gates, w.w,
-                  w.rpsum + cur * kMaxExperts, w.rcur + cur * kMaxExperts,
-                  w.rpsum + other * kMaxExperts, w.rcur + other * kMaxExperts, w.bucket};
+  P.ro = RouteOut{w.logits, w.sel, w.psel, w.gates, w.w, w.rpsum, w.rcur,
+                  w.rcur + kRouteFlag, w.bucket};
   const int grid = min(P.total_tiles, CTAS_PER_SM * h->num_sms);
   return route ? launch<false, true>(h, P, grid, st) : launch<false>(h, P, grid, st);
 }
 
 // The tile list (expert | rows << 8, first bucket slot) and its length come from the routing.
-// route_set >= 0: schedule from the dense projection's cursor set route_set and write the
+// from_cursors: schedule from the dense projection's cursors (the call's set) and write the
 // routing statistics (aux_out if non-null); otherwise from the routing kernel's tile list.
-int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route_set,
+int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, bool from_cursors,
                     float* aux_out, cudaStream_t st) {
   Params P;
   memset(&P, 0, sizeof(P));
@@ -936,9 +956,11 @@ int launch_tc_qproj(gqe_ctx* h, const void* x, int M, const void* W_q, int route
   P.bucket = h->ws.bucket;
   P.tile_list = h->ws.tile_list;
   P.tile_count = h->ws.tile_count;
-  if (route_set >= 0) {
-    P.rc = h->ws.rcur + (route_set & 1) * kMaxExperts;
-    P.rpsum = h->ws.rpsum + (route_set & 1) * kMaxExperts;
+  if (from_cursors) {
+    P.rc = h->ws.rcur;
+    P.rpsum = h->ws.rpsum;
+    P.set_flag = h->ws.rcur + kRouteFlag;
+    P.exit_counter = h->ws.rcur + kRouteFlag + 1;
     P.so = StatsOut{h->ws.counts, h->ws.mean_prob, h->ws.offsets, aux_out, h->ws.tile_count};
   }
   P.nexp = h->N;
