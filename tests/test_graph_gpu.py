@@ -1,4 +1,5 @@
-"""CUDA-graph capture and replay of gqe_forward and gqe_decode through the C ABI.
+"""CUDA-graph capture and replay through the C ABI: gqe_forward, gqe_decode, and a training
+step (gqe_forward + gqe_backward) captured as one graph.
 
 A captured call is replayed several times with new inputs copied into its static buffers,
 with eager calls on the same handle in between; every replay must give exactly the eager
@@ -12,7 +13,8 @@ import pytest
 import torch
 
 from moe_query_head_b200 import workloads as W
-from tests.gqe_testlib import GpuRun, check_output, oracle_forward, to_device, to_host_f64
+from tests.gqe_testlib import (GpuRun, check_output, oracle_forward, rel_l2, to_device,
+                               to_host_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -133,3 +135,59 @@ def test_decode_graph_replays_match_eager():
     del g
     G.gqe_destroy(he)
     G.gqe_destroy(hg)
+
+
+def test_training_step_graph_replays_match_eager():
+    """gqe_forward + gqe_backward captured together (the backward's GEMMs run in cuBLAS with
+    the handle's preset workspace) and replayed with new x and dy: y bit-identical to the
+    eager step's, every gradient equal to the eager step's within rel-L2 1e-6 (the same
+    kernels; a library GEMM may pick another reduction order under capture)."""
+    from moe_query_head_b200 import gqe as G
+    wl = MAIN.with_(B=1, T=300)
+    inp = W.generate(wl)
+    xs = [to_device(inp, "x"), to_device(W.generate(wl.with_(seed=wl.seed + 5)), "x")]
+    dys = [_dev_bf16(W.grad_output(wl)), _dev_bf16(W.grad_output(wl, seed_offset=1))]
+    names = ("x", "W_r", "W_q", "W_k", "W_v", "W_shared", "W_o")
+    shapes = dict(x=(wl.M, wl.dim), W_r=(wl.N, wl.dim), W_q=(wl.N * wl.d_h, wl.dim),
+                  W_k=(wl.G * wl.d_h, wl.dim), W_v=(wl.G * wl.d_h, wl.dim),
+                  W_shared=(wl.d_h, wl.dim), W_o=(wl.dim, wl.D_o))
+
+    def make():
+        run = GpuRun(inp)
+        G.gqe_enable_backward(run.h)
+        run.dy = dys[0].clone()
+        run.g = {n: torch.zeros(shapes[n], dtype=torch.float32, device="cuda") for n in names}
+        return run
+
+    def train_step(run):
+        _fwd(run)
+        d, g = run.dev, run.g
+        G.gqe_backward(run.h, d["x"], wl.B, wl.T, d["W_r"], d["W_q"], d["W_k"], d["W_v"],
+                       d["W_shared"], d["W_o"], wl.N, wl.G, wl.k, wl.d_h,
+                       W.VARIANT_IDS[wl.variant], int(wl.causal), run.dy, 0.01, g["x"],
+                       g["W_r"], g["W_q"], g["W_k"], g["W_v"], g["W_shared"], g["W_o"])
+
+    eager = make()
+    ref = []
+    for x, dy in zip(xs, dys):
+        eager.dev["x"], eager.dy = x, dy
+        train_step(eager)
+        assert G.gqe_check_device_status(eager.h) == G.GQE_OK
+        ref.append((eager.out.clone(), {n: eager.g[n].clone() for n in names}))
+    eager.close()
+
+    run = make()
+    run.dev["x"] = xs[0].clone()
+    g = _capture(lambda: train_step(run))
+    for step, i in enumerate([1, 0, 1]):
+        run.dev["x"].copy_(xs[i])
+        run.dy.copy_(dys[i])
+        g.replay()
+        torch.cuda.synchronize()
+        assert G.gqe_check_device_status(run.h) == G.GQE_OK, step
+        assert torch.equal(run.out, ref[i][0]), f"replay {step}: y differs"
+        for n in names:
+            err = rel_l2(run.g[n].cpu().numpy(), ref[i][1][n].cpu().numpy())
+            assert err <= 1e-6, (step, n, err)
+    del g
+    run.close()
