@@ -335,7 +335,7 @@ gqe_status gqe_decode(gqe_handle h, const void* x, int B, void* k_cache, void* v
             add(launch_tc_qproj(h, x, M, W_q, fused, aux_loss, st)) &&
             add(launch_tc_decode_attention(h, B, S, has_shared, variant, Do, k_cache, v_cache,
                                            L_max, lengths, st)) &&
-            add(launch_combine(h, M, variant, Do, st)) &&
+            add(0) &&  // the combine (gqe slot) runs in the cache attention's finish kernel
             add(launch_tc_oproj(h, M, Do, W_o, out, st));
   if (fused && dense >= 0 && !ok) reset_route_sets(h, st);
   h->last_M = M;

@@ -19,7 +19,10 @@
 // over the warp's keys with shuffles, P V with each lane owning pairs of head dimensions.
 // After the last tile the four warps' (m, l, O) are merged in shared memory. With one chunk
 // per sequence and group the CTA writes Z directly; otherwise it writes (m, l, O) to a
-// partial slot and decode_merge_kernel combines the chunks.
+// partial slot. decode_finish_kernel, one CTA per sequence, then combines the chunks of
+// every (group, query) and, for the gqe variant, forms the sequence's renormalised slot from
+// the Z blocks it has just written (gist.science summary, Output Construction), in the order
+// and precision of the forward's slot kernel.
 #include <string.h>
 
 #include "gqe_common.cuh"
@@ -47,11 +50,13 @@ struct DecParams {
   __nv_bfloat16* Z;           // [B, Do]
   const float* psel;          // [B, psel_stride]: stream s's p at column psel_off + s
   float* part;                // [B, G, nc, k+1, d_h + 2] partial (m, l, O) per chunk
+  const float* wslot;         // [B, w_stride] slot weights: stream s's at column w_off + s
   int32_t* status;
   // G, S, Sr: this handle's KV heads, streams and routed streams (a group range counts
   // from its first group; the caches hold its heads only)
   int B, G, k, S, Sr, has_shared, Do, shared_col, weighted, L_max, nc, chunk;
   int psel_stride, psel_off;
+  int slot, w_stride, w_off;  // slot: form the gqe slot at column Sr d_h
   float scale_log2;
 };
 
@@ -307,38 +312,57 @@ decode_attn_kernel(const DecParams P) {
   }
 }
 
-// Combines the chunks' (m, l, O) of every (sequence, group, query) and writes Z.
-__global__ void __launch_bounds__(THREADS) decode_merge_kernel(const DecParams P, int DH) {
-  const int g = blockIdx.x, b = blockIdx.y;
+// One CTA per sequence: combines the key chunks' (m, l, O) of every (group, query) of the
+// sequence and writes Z (when keys are split), then forms the gqe slot from Z's routed
+// blocks (a fixed order: stream 0 first, fp32 fused multiply-adds of the bf16 values).
+constexpr int FINISH_THREADS = 512;
+__global__ void __launch_bounds__(FINISH_THREADS) decode_finish_kernel(const DecParams P,
+                                                                       int DH) {
+  const int b = blockIdx.x;
   pdl_wait();
   pdl_allow_next();
   const int L = P.lengths[b];
   if (L < 0 || L >= P.L_max) return;  // flagged by the attention kernel
-  const int nq = P.k + ((g == 0 && P.has_shared) ? 1 : 0);
-  for (int e = threadIdx.x; e < nq * DH; e += THREADS) {
-    const int i = e / DH, d = e % DH;
-    const float* base = P.part + (((size_t)b * P.G + g) * P.nc * (P.k + 1) + i) * (DH + 2);
+  if (P.nc > 1) {
+    // queries: k per group, then the shared one (group 0, query index k)
+    const int nqs = P.G * P.k + P.has_shared;
     const size_t cstride = (size_t)(P.k + 1) * (DH + 2);
-    float mx = -INFINITY;
-    for (int c = 0; c < P.nc; ++c) mx = fmaxf(mx, base[c * cstride]);
-    float l = 0.f, o = 0.f;
-    for (int c = 0; c < P.nc; ++c) {
-      const float* sl = base + c * cstride;
-      if (sl[0] == -INFINITY) continue;  // a chunk past the sequence's last position
-      const float w = ex2(sl[0] - mx);
-      l += w * sl[1];
-      o += w * sl[2 + d];
+    for (int e = threadIdx.x; e < nqs * DH; e += FINISH_THREADS) {
+      const int q = e / DH, d = e % DH;
+      const int g = q < P.G * P.k ? q / P.k : 0;
+      const int i = q < P.G * P.k ? q % P.k : P.k;
+      const float* base = P.part + (((size_t)b * P.G + g) * P.nc * (P.k + 1) + i) * (DH + 2);
+      float mx = -INFINITY;
+      for (int c = 0; c < P.nc; ++c) mx = fmaxf(mx, base[c * cstride]);
+      float l = 0.f, o = 0.f;
+      for (int c = 0; c < P.nc; ++c) {
+        const float* sl = base + c * cstride;
+        if (sl[0] == -INFINITY) continue;  // a chunk past the sequence's last position
+        const float w = ex2(sl[0] - mx);
+        l += w * sl[1];
+        o += w * sl[2 + d];
+      }
+      const int s = stream_of(P, g, i);
+      float scale = 1.f / l;
+      int col;
+      if (s < P.Sr) {
+        col = s * DH;
+        if (P.weighted) scale *= P.psel[(size_t)b * P.psel_stride + P.psel_off + s];
+      } else {
+        col = P.shared_col;
+      }
+      P.Z[(size_t)b * P.Do + col + d] = __float2bfloat16_rn(o * scale);
     }
-    const int s = stream_of(P, g, i);
-    float scale = 1.f / l;
-    int col;
-    if (s < P.Sr) {
-      col = s * DH;
-      if (P.weighted) scale *= P.psel[(size_t)b * P.psel_stride + P.psel_off + s];
-    } else {
-      col = P.shared_col;
+    __syncthreads();  // the sequence's routed blocks of Z are written
+  }
+  if (P.slot) {
+    const float* w = P.wslot + (size_t)b * P.w_stride + P.w_off;
+    __nv_bfloat16* z = P.Z + (size_t)b * P.Do;
+    for (int d = threadIdx.x; d < DH; d += FINISH_THREADS) {
+      float acc = 0.f;
+      for (int s = 0; s < P.Sr; ++s) acc = fmaf(w[s], __bfloat162float(z[s * DH + d]), acc);
+      z[(size_t)P.Sr * DH + d] = __float2bfloat16_rn(acc);
     }
-    P.Z[(size_t)b * P.Do + col + d] = __float2bfloat16_rn(o * scale);
   }
 }
 
@@ -359,8 +383,8 @@ int launch_dh(const DecParams& P, cudaStream_t st) {
                 : nq_max <= 4 ? launch_attn<DH, 4>(P, st)
                               : launch_attn<DH, MAXQ>(P, st);
   if (r < 0) return -1;
-  if (P.nc == 1) return 1;
-  return launch_pdl(decode_merge_kernel, dim3(P.G, P.B), dim3(THREADS), 0, st, P, DH) ==
+  if (P.nc == 1 && !P.slot) return 1;
+  return launch_pdl(decode_finish_kernel, dim3(P.B), dim3(FINISH_THREADS), 0, st, P, DH) ==
                  cudaSuccess
              ? 2
              : -1;
@@ -397,6 +421,7 @@ int launch_tc_decode_attention(gqe_ctx* h, int B, int S, int has_shared, int var
   P.Z = static_cast<__nv_bfloat16*>(h->ws.Z);
   P.psel = h->ws.psel;
   P.part = h->ws.dec_part;
+  P.wslot = h->ws.w;
   P.status = h->ws.status;
   P.B = B;
   P.G = h->g1 - h->g0;
@@ -409,6 +434,9 @@ int launch_tc_decode_attention(gqe_ctx* h, int B, int S, int has_shared, int var
   P.Do = Do;
   P.shared_col = (P.Sr + (variant == GQE_VARIANT_GQE ? 1 : 0)) * d_h;
   P.weighted = variant == GQE_VARIANT_WEIGHTED_CONCAT;
+  P.slot = variant == GQE_VARIANT_GQE;
+  P.w_stride = h->G * h->k;  // the slot weights are the whole layer's
+  P.w_off = h->g0 * h->k;
   P.L_max = L_max;
   P.nc = decode_chunks(h, B, L_max);
   // keys per chunk: a multiple of the tile, covering positions 0 .. L_max - 1

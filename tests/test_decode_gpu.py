@@ -4,9 +4,12 @@ tolerances (rel-L2 1e-2, max-abs 3e-2); aux loss within 1e-4 relative; the new t
 written at its position (equal to the step's own projection, and to the oracle's within bf16
 rounding) and every other cache row left bit-identical.
 
-Cases cover both ways the attention runs (one CTA per sequence and group writing Z
-directly when there are at least four such pairs per SM, and split key chunks merged by a
-second kernel), ragged positions (0, tile edges, long), the three variants, every head dim the ABI accepts,
+Cases cover both ways the attention runs: one CTA per (sequence, group) writing Z directly
+(a single 64-key tile, or at least sixteen such pairs per SM of a B200), and split key
+chunks combined by the per-sequence finish kernel, which also forms the gqe slot (with one
+chunk it forms only the slot; weighted_concat and hard_concat with one chunk launch no
+finish kernel). Also: ragged positions (0, tile edges, long), the three variants, every
+head dim the ABI accepts,
 one to three queries per warp (k up to 8), a layer without the shared head, and the
 consistency of a decode step with the GPU prefill row at the same position."""
 import numpy as np
@@ -113,9 +116,15 @@ LARGE = W.WORKLOADS["large_skew"].with_(skew=None)
 CASES = {
     # B * G = 56, far fewer than four per SM: many key chunks per pair, merged
     "main_split_ragged": (MAIN, [0, 1, 63, 64, 65, 700, 1023], 1024),
-    # B * G = 640 (at least four CTAs per SM of a B200 without splitting): one CTA per
-    # (sequence, group), Z written directly
-    "main_direct_batch80": (MAIN, list(np.random.default_rng(3).integers(0, 300, 80)), 320),
+    # B * G = 640: four key chunks per (sequence, group) on a B200
+    "main_split4_batch80": (MAIN, list(np.random.default_rng(3).integers(0, 300, 80)), 320),
+    # one 64-key tile per sequence: one CTA per (sequence, group) writes Z; the finish
+    # kernel forms only the slot
+    "main_direct_short": (MAIN, [0, 5, 31, 63, 17], 64),
+    # B * G = 2560, at least sixteen CTAs per SM of a B200 without splitting
+    "main_direct_batch320": (MAIN, list(np.random.default_rng(7).integers(0, 200, 320)), 256),
+    # one chunk and no slot: no finish kernel
+    "wide_weighted_direct": (WIDE.with_(variant="weighted_concat"), [0, 40, 63], 64),
     # B * G = 320: two key chunks per (sequence, group), merged
     "main_split_batch40": (MAIN, list(np.random.default_rng(5).integers(0, 300, 40)), 320),
     "main_no_shared_hard": (MAIN.with_(shared=False, variant="hard_concat"), [9, 129, 257], 384),
@@ -128,8 +137,8 @@ CASES = {
     # with 64 experts (nine queries in group 0)
     "wide_k4_qpw2": (WIDE.with_(k=4), [3, 200, 511], 512),
     "n64_k8_qpw3": (MAIN.with_(N=64, G=8, k=8), [0, 65, 300], 320),
-    # one CTA per (sequence, group) at d_h = 80
-    "dh80_direct_batch80": (MAIN.with_(d_h=80),
+    # d_h = 80 with four key chunks per (sequence, group)
+    "dh80_split4_batch80": (MAIN.with_(d_h=80),
                             list(np.random.default_rng(6).integers(0, 200, 80)), 256),
 }
 # every head dim the ABI accepts, split key chunks with ragged positions
