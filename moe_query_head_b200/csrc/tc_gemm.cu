@@ -48,10 +48,12 @@ struct Lay {
 };
 // Shared-memory ring: B stages hold up to BN rows, or 64 for the routed projection of a head
 // dimension up to 64 (NARROW), whose smaller stages buy a fourth stage in the same space:
-// these GEMMs are bound by load latency times the bytes in flight.
-template <bool NARROW>
+// these GEMMs are bound by load latency times the bytes in flight. DEEP: one CTA per SM
+// with twice the stages, for grids no larger than the SM count (the small-M GEMMs of a
+// decode step), whose few CTAs each walk all of K: fewer round trips over K.
+template <bool NARROW, bool DEEP = false>
 struct Ring {
-  static constexpr int STAGES = NARROW ? 4 : 3;
+  static constexpr int STAGES = (NARROW ? 4 : 3) * (DEEP ? 2 : 1);
   static constexpr int B_ROWS = NARROW ? 64 : BN;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
@@ -419,11 +421,11 @@ __device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0, int cset
 
 // ROUTE: the dense projection whose router tiles (problem 0) route (route_rows); a separate
 // instance, so the plain GEMMs carry none of that code.
-template <bool GATHER, bool ROUTE, bool NARROW>
-__global__ void __launch_bounds__(Lay<GATHER>::THREADS, CTAS_PER_SM)
+template <bool GATHER, bool ROUTE, bool NARROW, bool DEEP>
+__global__ void __launch_bounds__(Lay<GATHER>::THREADS, DEEP ? 1 : CTAS_PER_SM)
 tc_gemm_kernel(const __grid_constant__ Params P) {
   using L = Lay<GATHER>;
-  using R = Ring<NARROW>;
+  using R = Ring<NARROW, DEEP>;
   constexpr int STAGES = R::STAGES;
   constexpr int A_STAGE_BYTES = R::A_BYTES;
   constexpr int B_STAGE_BYTES = R::B_BYTES;
@@ -814,14 +816,20 @@ bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATHER, bool ROUTE = false, bool NARROW = false>
-int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
-  constexpr int smem = Ring<NARROW>::SMEM;
-  if (!set_smem_limit_once<tc_gemm_kernel<GATHER, ROUTE, NARROW>>(smem)) return -1;
-  return launch_pdl(tc_gemm_kernel<GATHER, ROUTE, NARROW>, dim3(grid),
+template <bool GATHER, bool ROUTE, bool NARROW, bool DEEP>
+int launch_ring(const Params& P, int grid, cudaStream_t st) {
+  constexpr int smem = Ring<NARROW, DEEP>::SMEM;
+  if (!set_smem_limit_once<tc_gemm_kernel<GATHER, ROUTE, NARROW, DEEP>>(smem)) return -1;
+  return launch_pdl(tc_gemm_kernel<GATHER, ROUTE, NARROW, DEEP>, dim3(grid),
                     dim3(Lay<GATHER>::THREADS), smem, st, P) == cudaSuccess
              ? 1
              : -1;
+}
+
+template <bool GATHER, bool ROUTE = false, bool NARROW = false>
+int launch(gqe_ctx* h, const Params& P, int grid, cudaStream_t st) {
+  return grid <= h->num_sms ? launch_ring<GATHER, ROUTE, NARROW, true>(P, grid, st)
+                            : launch_ring<GATHER, ROUTE, NARROW, false>(P, grid, st);
 }
 
 Problem make_problem(int N, OutMap out) {
