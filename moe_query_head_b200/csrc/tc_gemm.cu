@@ -375,15 +375,26 @@ __device__ void route_rows_any(const Params& P, uint32_t t_row, int t, bool vali
 // writes the routing statistics ("GQE" README, Algorithm Overview; the Switch-style
 // load-balancing loss): counts, mean_prob (fixed-point sum / M), offsets (e M) and
 //   L = (1/G) sum_e E f_e Pbar_e,  f = count / (M k),  Pbar = prob_sum / M.
-__device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0, int cset) {
+__device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0, double* s_ps) {
   const int N = P.nexp, M = P.M;
   const int tid = threadIdx.x;
   if (tid < N) {
+    // the set flag and both sets' counts (and, in CTA 0, probability sums) in one round
+    // trip; the flag then picks the call's set
+    const int flag = __ldcg(P.set_flag);
+    const int c0 = __ldcg(P.rc + tid), c1 = __ldcg(P.rc + kMaxExperts + tid);
+    long long p0 = 0, p1 = 0;
+    if (blockIdx.x == 0) {
+      p0 = __ldcg(reinterpret_cast<const long long*>(P.rpsum) + tid);
+      p1 = __ldcg(reinterpret_cast<const long long*>(P.rpsum) + kMaxExperts + tid);
+    }
+    const bool second = flag & 1;
     // a count above M would mean a cursor set that was not cleared: never reached, but the
     // bucket reads stay inside expert e's M slots whatever the cursors hold
-    const int c = __ldcg(P.rc + cset + tid);
+    const int c = second ? c1 : c0;
     s_cnt[tid] = min(max(c, 0), M);
     if (c < 0 || c > M) atomicExch(P.status, kStatusBadState);
+    if (blockIdx.x == 0) s_ps[tid] = (double)(second ? p1 : p0) / kProbFix;
   }
   __syncthreads();
   if (tid == 0) {
@@ -398,20 +409,15 @@ __device__ void routed_schedule(const Params& P, int* s_cnt, int* s_t0, int cset
     const StatsOut& S = P.so;
     const int G = N / P.E;
     if (tid < N) {
-      const double ps =
-          (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + cset + tid) / kProbFix;
       S.counts[tid] = s_cnt[tid];
       S.offsets[tid] = tid * M;
-      S.mean_prob[tid] = (float)(ps / M);
+      S.mean_prob[tid] = (float)(s_ps[tid] / M);
     }
     if (tid == 0) {
       S.offsets[N] = N * M;
       double L = 0.0;
-      for (int x = 0; x < N; ++x) {
-        const double ps =
-            (double)__ldcg(reinterpret_cast<const long long*>(P.rpsum) + cset + x) / kProbFix;
-        L += (double)P.E * ((double)s_cnt[x] / ((double)M * P.k)) * (ps / M);
-      }
+      for (int x = 0; x < N; ++x)
+        L += (double)P.E * ((double)s_cnt[x] / ((double)M * P.k)) * (s_ps[x] / M);
       if (S.aux) S.aux[0] = (float)(L / G);
     }
   }
@@ -477,21 +483,26 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   pdl_allow_next();
   int* s_cnt = reinterpret_cast<int*>(scratch);         // [kMaxExperts] routed schedule
   int* s_t0 = s_cnt + kMaxExperts;                      // [kMaxExperts + 1]
+  double* s_ps = reinterpret_cast<double*>(scratch + 528);  // [kMaxExperts] (CTA 0)
   int total = P.total_tiles;
   int cset = 0;  // this call's cursor set, as an offset into the two sets
   if constexpr (ROUTE) {
-    // this call's cursor set is zero; the other one (the previous call's) is cleared here
-    cset = (__ldcg(P.ro.set_flag) & 1) * kMaxExperts;
-    if (blockIdx.x == 0 && threadIdx.x < kMaxExperts) {
-      const int other = kMaxExperts - cset;
-      P.ro.cursor[other + threadIdx.x] = 0;
-      P.ro.psum_fx[other + threadIdx.x] = 0ull;
+    // Only the epilogue warps route, so only they read the set flag (the producer and MMA
+    // warps start at once). This call's set is zero; two epilogue warps of CTA 0 clear the
+    // other one (the previous call's, whose last reader has finished).
+    if (warp >= L::EPI0) {
+      cset = (__ldcg(P.ro.set_flag) & 1) * kMaxExperts;
+      const int e = threadIdx.x - L::EPI0 * 32;
+      if (blockIdx.x == 0 && e < kMaxExperts) {
+        const int other = kMaxExperts - cset;
+        P.ro.cursor[other + e] = 0;
+        P.ro.psum_fx[other + e] = 0ull;
+      }
     }
   }
   if constexpr (GATHER) {
     if (P.rc != nullptr) {
-      cset = (__ldcg(P.set_flag) & 1) * kMaxExperts;
-      routed_schedule(P, s_cnt, s_t0, cset);  // block-wide
+      routed_schedule(P, s_cnt, s_t0, s_ps);  // block-wide
       total = s_t0[P.nexp];
     } else {
       total = *P.tile_count;
