@@ -13,7 +13,8 @@
 // and its experts' buckets (still routing every group in the dense projection).
 //
 // One persistent kernel, two CTAs per SM (each CTA's pipeline hand-offs, fills and tail are
-// covered by the other CTA's work):
+// covered by the other CTA's work); grids of at most one CTA per SM (small M) run one CTA per
+// SM with a ring twice as deep:
 //   producers  dense: one warp issuing TMA tile loads of A and B. Routed projection: three
 //              warps gathering A rows through registers into the 128-byte swizzled
 //              layout (each warp fills every third stage), B by TMA;
