@@ -6,14 +6,16 @@
 // sparse query heads apply to each new token: for group g the new token has k routed query
 // streams (s = g*k + r) and, in group 0, the always-on shared stream (it reads KV head 0;
 // gist.science summary, Output Construction). A step for B sequences runs the forward's
-// projection, routing, combine and W_o kernels on the B new tokens; this file holds the part
-// that differs: the attention of stream s of sequence b over positions 0..L_b of its KV head,
-// where positions < L_b come from the cache and position L_b is the new token.
+// projection, routing and W_o kernels on the B new tokens; this file holds the parts that
+// differ: the attention of stream s of sequence b over positions 0..L_b of its KV head,
+// where positions < L_b come from the cache and position L_b is the new token, and the
+// combine of the key chunks and the gqe slot.
 //
 // The work is HBM-bound (every cached K/V row is read once, shared by all query streams of
 // its group), so it runs on CUDA cores. CTA (chunk c, group g, sequence b) streams its key
-// range in tiles of 64 rows through a two-stage cp.async ring in shared memory (rows padded
-// by 16 bytes). Each of the four warps takes 16 keys of every tile for all of the group's queries,
+// range in tiles of 64 rows through a two-stage cp.async ring in shared memory (dense rows
+// for d_h an odd multiple of 16, else rows padded by 16 bytes: see DecCfg). Each of the four
+// warps takes 16 keys of every tile for all of the group's queries,
 // so the work is spread evenly however few queries a group has (two at k = 1 in group 0,
 // one elsewhere): a score per (key, half of the head dims) lane pair, the online softmax
 // over the warp's keys with shuffles, P V with each lane owning pairs of head dimensions.
