@@ -62,6 +62,20 @@ struct Ring {
   static constexpr int SMEM =
       STAGES * (A_BYTES + B_BYTES) + 1024 + 256 + 16 * (kMaxExperts + 8) + 4 * kMaxExperts;
 };
+// Scratch after the barriers (routed schedule): s_cnt [kMaxExperts] and s_t0
+// [kMaxExperts + 1] ints, then CTA 0's probability sums, doubles, at kPsOffset.
+constexpr int kPsOffset = 528;
+static_assert(kPsOffset >= 4 * (2 * kMaxExperts + 1) && kPsOffset % 8 == 0,
+              "the probability sums follow the schedule arrays, 8-byte aligned");
+template <int STAGES>
+constexpr bool scratch_fits() {
+  // barriers (full, empty per stage; two accumulators' full and empty), the TMEM holder and
+  // abort flag (16 bytes), then the scratch, within the space SMEM reserves after the stages
+  return (2 * STAGES + 4) * 8 + 16 + kPsOffset + 8 * kMaxExperts <=
+         256 + 16 * (kMaxExperts + 8) + 4 * kMaxExperts;
+}
+static_assert(scratch_fits<Ring<true, true>::STAGES>() && scratch_fits<Ring<false, true>::STAGES>(),
+              "the routed schedule's scratch fits the deepest ring's shared memory");
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int MAX_PROBLEMS = 4;
 constexpr int MAX_COL_TILES = 32;  // column tiles over all problems of one GEMM
@@ -484,7 +498,7 @@ tc_gemm_kernel(const __grid_constant__ Params P) {
   pdl_allow_next();
   int* s_cnt = reinterpret_cast<int*>(scratch);         // [kMaxExperts] routed schedule
   int* s_t0 = s_cnt + kMaxExperts;                      // [kMaxExperts + 1]
-  double* s_ps = reinterpret_cast<double*>(scratch + 528);  // [kMaxExperts] (CTA 0)
+  double* s_ps = reinterpret_cast<double*>(scratch + kPsOffset);  // [kMaxExperts] (CTA 0)
   int total = P.total_tiles;
   int cset = 0;  // this call's cursor set, as an offset into the two sets
   if constexpr (ROUTE) {
