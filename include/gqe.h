@@ -375,7 +375,8 @@ const char* gqe_status_str(int status);
 int64_t gqe_workspace_bytes(int dim, int N, int G, int k, int d_h, gqe_dtype dtype,
                             int64_t max_tokens);
 
-/* gqe_kernel_launches — kernels the last gqe_forward on this handle launched. */
+/* gqe_kernel_launches — kernels the last gqe_forward or gqe_decode on this handle launched
+ * (-1 for a null handle). */
 int gqe_kernel_launches(gqe_handle h);
 
 #ifdef __cplusplus
