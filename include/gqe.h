@@ -190,7 +190,9 @@ gqe_status gqe_enable_backward(gqe_handle h);
  * Enqueued on `stream`; allocates nothing and does not synchronise. Hand-written kernels
  * form the combine/router backward and the attention backward (tcgen05); the dense weight
  * and input gradient GEMMs run in cuBLAS. The result is the same from run to run (no
- * atomics). Errors as gqe_forward.
+ * atomics). Errors as gqe_forward. A gqe_forward followed by this call may be captured in
+ * one CUDA graph and replayed as a training step (cuBLAS runs with the handle's preset
+ * workspace, so the capture allocates nothing).
  */
 gqe_status gqe_backward(gqe_handle h, const void* x, int B, int T, const void* W_r,
                         const void* W_q, const void* W_k, const void* W_v, const void* W_shared,
