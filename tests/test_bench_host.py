@@ -1,7 +1,7 @@
 """Host logic of bench.py that needs no GPU: the DRAM traffic of the attention and of the
 decode cache attention is reported only for the profiled workload and only while the
 kernel's sources hash to the value recorded with the ncu capture; the decode workload's
-shapes."""
+shapes; the reference arm's timing; the clock record read from nvidia-smi's samples."""
 import json
 import os
 
@@ -64,3 +64,44 @@ def test_reference_arm_reports_the_time_it_ran():
     wl = bench.W.WORKLOADS["tiny_f32"]
     assert line["config"] == bench.prefill_config(wl, 1)
     assert line["cpu_baseline"]["value"] == line["value"]
+
+
+def test_clock_sampler_reads_nvidia_smi_samples(tmp_path):
+    """The clock record beside a timed run: the median SM clock over the busy samples (idle
+    ones, under half the fastest, left out), the maximum clock, and every throttle reason
+    seen active (nvidia-smi's csv,noheader,nounits rows of ClockSampler.FIELDS)."""
+    import tempfile
+
+    class Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    rows = [
+        "345, 1965, 120.1, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",
+        "1965, 1965, 850.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1950, 1965, 990.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 870.4, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    s = object.__new__(bench.ClockSampler)
+    s.proc = Proc()
+    s.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False, dir=tmp_path)
+    s.file.write("\n".join(rows) + "\n")
+    rec = s.stop()
+    assert rec["samples"] == 4
+    assert rec["sm_mhz"] == 1965.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"]
+    # a hardware slowdown is reported by name, so the run can be rejected
+    s2 = object.__new__(bench.ClockSampler)
+    s2.proc = Proc()
+    s2.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False, dir=tmp_path)
+    s2.file.write("1500, 1965, 600, 0x8, Active, Not Active, Not Active, Not Active\n")
+    assert s2.stop()["reasons"] == ["hw_slowdown"]
+    # no nvidia-smi: no clock figures, and the record says why
+    s3 = object.__new__(bench.ClockSampler)
+    s3.proc = None
+    assert s3.stop() == {"sm_mhz": None, "sm_max_mhz": None,
+                         "reasons": ["nvidia-smi unavailable"]}
